@@ -1,0 +1,171 @@
+"""Pins for the CPU oracle (no GPU).  Each test ties an oracle function to a
+fact fixed by the report or by the mathematics, not to a retyped copy of it."""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import QUINTIC
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed=0):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _scalar_iterate(sig, coeffs, steps):
+    """Singular-value picture: Y -> aY + (bYY^T + c(YY^T)^2)Y maps each
+    singular value s of Y to a s + b s^3 + c s^5 and keeps the vectors."""
+    a, b, c = coeffs
+    for _ in range(steps):
+        sig = a * sig + b * sig ** 3 + c * sig ** 5
+    return sig
+
+
+@pytest.mark.parametrize("shape", [(8, 16), (16, 8), (32, 64), (64, 128), (1, 5), (5, 1), (24, 24)])
+@pytest.mark.parametrize("steps", [1, 2, 5])
+def test_newton_schulz_equals_polynomial_on_singular_values(shape, steps):
+    X = _rand(shape, seed=shape[0] * 1000 + shape[1])
+    eps = 1e-7
+    O = oracle.newton_schulz(X, steps, QUINTIC, eps)
+    U, s, Vt = np.linalg.svd(X / (np.linalg.norm(X) + eps), full_matrices=False)
+    expect = (U * _scalar_iterate(s, QUINTIC, steps)) @ Vt
+    assert O.shape == X.shape
+    assert np.linalg.norm(O - expect) <= 1e-10 * np.linalg.norm(expect)
+
+
+def test_newton_schulz_output_band():
+    """Tuned quintic, 5 steps: singular values of O lie in the image of the
+    scalar map over the input band (grid-evaluated here)."""
+    X = _rand((96, 200), seed=3)
+    O = oracle.newton_schulz(X, 5, QUINTIC, 1e-7)
+    s_in = np.linalg.svd(X / np.linalg.norm(X), compute_uv=False)
+    s_out = np.linalg.svd(O, compute_uv=False)
+    grid = np.linspace(s_in.min(), s_in.max(), 200001)
+    img = _scalar_iterate(grid, QUINTIC, 5)
+    assert s_out.min() >= img.min() - 1e-9 and s_out.max() <= img.max() + 1e-9
+    # the tuned map keeps every value of a well-spread spectrum near 1
+    assert 0.6 < s_out.min() and s_out.max() < 1.25
+
+
+@pytest.mark.parametrize("coeffs", [(1.5, -0.5, 0.0), (15 / 8, -10 / 8, 3 / 8)])
+def test_newton_schulz_converges_to_polar_factor(coeffs):
+    rng = np.random.default_rng(7)
+    U, _ = np.linalg.qr(rng.standard_normal((40, 40)))
+    V, _ = np.linalg.qr(rng.standard_normal((90, 40)))
+    s = np.geomspace(1.0, 0.1, 40)                       # condition number 10
+    X = (U * s) @ V.T
+    polar = U @ V.T
+    errs = [np.linalg.norm(oracle.newton_schulz(X, k, coeffs, 0.0) - polar) / np.linalg.norm(polar)
+            for k in range(0, 41, 5)]
+    assert all(e1 <= e0 + 1e-14 for e0, e1 in zip(errs, errs[1:]))
+    assert errs[-1] < 1e-10
+
+
+def test_tuned_quintic_does_not_converge():
+    """The tuned coefficients trade convergence for speed: p(1) != 1."""
+    assert abs(_scalar_iterate(np.array([1.0]), QUINTIC, 1)[0] - 0.701) < 1e-3
+
+
+def test_newton_schulz_transpose_and_scale():
+    X = _rand((20, 50), seed=11)
+    O = oracle.newton_schulz(X, 5, QUINTIC, 0.0)
+    Ot = oracle.newton_schulz(X.T.copy(), 5, QUINTIC, 0.0)
+    assert np.allclose(Ot, O.T, rtol=0, atol=1e-12)
+    O3 = oracle.newton_schulz(1e-3 * X, 5, QUINTIC, 0.0)
+    assert np.allclose(O3, O, rtol=0, atol=1e-12)
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            lhs, rhs = line.split("|")
+            rows.append(([float(v) for v in lhs.split()], [float(v) for v in rhs.split()]))
+    return rows
+
+
+def test_hyperball_hand_solved_cases():
+    rows = _golden_rows("hyperball_two_element.txt")
+    assert len(rows) == 3
+    for (w0, w1, o0, o1, lr, R), (n0, n1, elr) in rows:
+        W_new, st = oracle.hyperball_update(np.array([[w0, w1]]), np.array([[o0, o1]]), lr, R)
+        assert np.allclose(W_new, [[n0, n1]], rtol=0, atol=1e-14)
+        assert abs(st["elr"] - elr) < 1e-15
+
+
+def test_hyperball_invariants():
+    """||W_{t+1}|| = R and effective LR = lr (Sec. 3.3.1)."""
+    rng = np.random.default_rng(5)
+    for lr in (0.0, 1e-4, 0.012, 0.3):
+        W = rng.standard_normal((30, 70))
+        R = np.linalg.norm(W)
+        O = rng.standard_normal((30, 70))
+        W_new, st = oracle.hyperball_update(W, O, lr, R)
+        assert abs(np.linalg.norm(W_new) - R) <= 1e-13 * R
+        assert abs(st["elr"] - lr) <= 1e-14
+        assert abs(st["post_norm"] - R) <= 1e-13 * R
+        # the update is scale-free: O and 7 O give the same step
+        W7, _ = oracle.hyperball_update(W, 7.0 * O, lr, R)
+        assert np.allclose(W7, W_new, rtol=0, atol=1e-14)
+
+
+def test_momentum_geometric_sum():
+    """After k steps from M=0: M_k = sum_j beta^(k-j) G_j; X = G_k + beta M_k."""
+    beta = 0.95
+    Gs = [_rand((6, 9), seed=100 + j) for j in range(5)]
+    M = np.zeros((6, 9))
+    for k, G in enumerate(Gs):
+        M, X = oracle.momentum_update(M, G, beta, nesterov=True)
+        geo = sum(beta ** (k - j) * Gs[j] for j in range(k + 1))
+        assert np.allclose(M, geo, rtol=0, atol=1e-13)
+        assert np.allclose(X, Gs[k] + beta * geo, rtol=0, atol=1e-13)
+    _, Xp = oracle.momentum_update(np.zeros((6, 9)), Gs[0], 0.0, nesterov=True)
+    assert np.array_equal(Xp, Gs[0])
+    M2, X2 = oracle.momentum_update(M, Gs[0], beta, nesterov=False)
+    assert np.array_equal(X2, M2)
+
+
+def test_lerp_momentum_gives_the_same_direction():
+    beta = 0.9
+    G1, G2 = _rand((8, 12), 1), _rand((8, 12), 2)
+    _, Xs = oracle.momentum_update(oracle.momentum_update(np.zeros((8, 12)), G1, beta)[0], G2, beta)
+    Ml = (1 - beta) * G1                                   # lerp form, one step
+    Ml = beta * Ml + (1 - beta) * G2
+    Xl = (1 - beta) * G2 + beta * Ml
+    assert np.allclose(Xl, (1 - beta) * Xs, rtol=0, atol=1e-14)
+    assert np.allclose(oracle.newton_schulz(Xl, 5, QUINTIC, 0.0),
+                       oracle.newton_schulz(Xs, 5, QUINTIC, 0.0), rtol=0, atol=1e-12)
+
+
+def test_step_edge_cases():
+    W = _rand((4, 6), 9)
+    R = np.linalg.norm(W)
+    Z = np.zeros((4, 6))
+    # zero gradient and zero momentum: no displacement, re-projection only
+    W1, M1, O, st = oracle.muonh_step(W, Z, Z, 0.01, R)
+    assert st["flags"] & oracle.FLAG_ZERO_UPDATE and st["elr"] == 0.0
+    assert np.allclose(W1, W, rtol=0, atol=1e-15)
+    # non-finite gradient: W kept, flag raised
+    G = _rand((4, 6), 10)
+    G[1, 2] = np.nan
+    W2, M2, O2, st2 = oracle.muonh_step(W, Z, G, 0.01, R)
+    assert st2["flags"] & oracle.FLAG_NONFINITE_INPUT and np.array_equal(W2, W)
+    # lr = 0 re-projects onto the same sphere
+    W3, _, _, st3 = oracle.muonh_step(W, Z, _rand((4, 6), 12), 0.0, R)
+    assert st3["elr"] == 0.0 and np.allclose(W3, W, rtol=0, atol=1e-14)
+
+
+def test_multi_step_norm_stays_on_sphere():
+    shapes = [(16, 40), (40, 16)]
+    W0 = [_rand(s, 20 + i) * 0.02 for i, s in enumerate(shapes)]
+    out = oracle.run_steps(W0, lambda t, i: _rand(shapes[i], 1000 * t + i) * 1e-3, [0.01] * 6)
+    for i in range(2):
+        assert abs(np.linalg.norm(out["W"][i]) - out["R"][i]) <= 1e-12 * out["R"][i]
+        for st in out["stats"]:
+            assert abs(st[i]["elr"] - 0.01) < 1e-12
