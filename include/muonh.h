@@ -1,0 +1,170 @@
+/*
+ * muonh.h -- C ABI of the MuonH optimizer step for NVIDIA B200 (sm_100a).
+ *
+ * MuonH ("Muon with the Hyperball wrapper") is the optimizer the Puro-2B
+ * report applies to the attention and MLP matrices of a Qwen3-architecture
+ * model (arXiv HTML, Sec. 3.3 "Hyperball Optimization").  For each wrapped
+ * matrix W (m x n) one step computes
+ *
+ *   M_t   = beta M_{t-1} + G_t                      heavy-ball momentum
+ *   X     = G_t + beta M_t   (Nesterov)  or  M_t
+ *   O     = NS(X)                                   quintic Newton-Schulz:
+ *           Y = X/(||X||_F + eps) on the wide orientation, then ns_steps times
+ *           A = Y Y^T;  B = b A + c A A;  Y = a Y + B Y
+ *   u^    = O/||O||_F                               Sec. 3.3, Eq. (1)
+ *   W~    = W_t - lr R u^                           Sec. 3.3, Eq. (1)
+ *   W_t+1 = R W~/||W~||_F                           Sec. 3.3, Eq. (1)
+ *
+ * with the radius fixed at R = ||W_0||_F (Sec. 3.3).  The effective LR of
+ * Sec. 3.3.1 Eq. (4), ||lr R u^||_F/||W_t||_F, then equals lr, so `lr` is the
+ * prescribed effective LR (eta^H = m eta^base of Sec. 3.3.1; the caller
+ * applies the multiplier m and the schedule).  The pages name the Muon update
+ * but not its internals: momentum form, Nesterov, eps and the coefficients
+ * (a, b, c) are per-matrix inputs here.
+ *
+ * Conventions shared by every entry point
+ *   - All functions are host functions; `stream` is a cudaStream_t passed as
+ *     void* (NULL = the legacy default stream).  Work is enqueued
+ *     asynchronously on it; argument checking is synchronous.
+ *   - Device pointers are CUDA device (or managed) addresses on the current
+ *     device.  The library never frees memory it did not allocate.
+ *   - A non-OK status leaves every caller buffer untouched; the message of
+ *     the last failure on the calling thread is in muonh_last_error().
+ *   - Conditions found on the device (non-finite input, zero update, a
+ *     bounded wait that gave up) never abort a step: they set per-matrix
+ *     flags in muonh_stats and are reported by muonh_device_status().
+ */
+#ifndef MUONH_H_
+#define MUONH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MUONH_OK = 0,
+  MUONH_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size, bad enum value     */
+  MUONH_ERR_ALIGNMENT = 2,     /* pointer or stride not 16-byte aligned      */
+  MUONH_ERR_CUDA = 3,          /* a CUDA runtime call failed                 */
+  MUONH_ERR_OOM = 4,           /* workspace allocation failed                */
+  MUONH_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up         */
+  MUONH_ERR_UNSUPPORTED = 6    /* no sm_100 device, or a size beyond limits  */
+} muonh_status;
+
+/* Arithmetic of the Newton-Schulz GEMMs (tensor cores, fp32 accumulation).
+ *   FP16: operands stored as fp16 with exact power-of-two scaling (default)
+ *   BF16: operands stored as bf16
+ *   FP32: each operand split into an fp16 high and low part, three products
+ *         per GEMM (hi*hi + hi*lo + lo*hi), about fp32 accuracy, 3x the work */
+enum { MUONH_NS_FP16 = 0, MUONH_NS_BF16 = 1, MUONH_NS_FP32 = 2 };
+
+/* Per-matrix flags reported in muonh_stats.flags. */
+enum {
+  MUONH_FLAG_NONFINITE_INPUT = 1u,   /* X had NaN/Inf: W kept unchanged          */
+  MUONH_FLAG_ZERO_UPDATE = 2u,       /* ||X|| or ||O|| == 0: W only re-projected */
+  MUONH_FLAG_NONFINITE_UPDATE = 4u,  /* X finite, O not: W kept unchanged        */
+  MUONH_FLAG_DEGENERATE = 8u,        /* ||W~|| == 0: W kept unchanged            */
+  MUONH_FLAG_TIMEOUT = 16u           /* a device wait gave up during this step   */
+};
+
+/* One wrapped matrix.  w and m are caller-owned fp32 device buffers of
+ * rows x cols elements, row-major with row stride ld (elements, ld >= cols),
+ * 16-byte aligned base.  Rows are moved with 16-byte vector accesses when
+ * cols and ld are multiples of 4, element by element otherwise (slower, any
+ * ld).  The library updates them in
+ * place on every step and keeps the pointers: they must stay valid until
+ * muonh_destroy.  m must hold zeros before the first step (momentum starts
+ * at 0).  radius <= 0 asks muonh_init to use ||W_0||_F (the Sec. 3.3 rule);
+ * a positive value is used as R as given.  ns_steps in [0, 64]. */
+typedef struct {
+  float* w;
+  float* m;
+  int64_t rows;
+  int64_t cols;
+  int64_t ld;
+  float radius;
+  float beta;
+  int32_t nesterov;
+  int32_t ns_steps;
+  float ns_a;
+  float ns_b;
+  float ns_c;
+} muonh_matrix_desc;
+
+typedef struct {
+  int32_t ns_precision;   /* MUONH_NS_FP16 / _BF16 / _FP32                  */
+  float eps;              /* Newton-Schulz input: X/(||X||_F + eps), >= 0    */
+} muonh_config;
+
+/* Per-matrix result of one step (24 bytes, plain fp32 + uint32). */
+typedef struct {
+  float elr;          /* ||lr R u^||_F / ||W_t||_F  (Eq. (4) for Eq. (1))   */
+  float pre_norm;     /* ||W_t||_F                                          */
+  float post_norm;    /* ||W_t+1||_F, measured on the stored result         */
+  float update_norm;  /* ||O||_F, the Newton-Schulz output                  */
+  float input_norm;   /* ||X||_F, the Newton-Schulz input                   */
+  uint32_t flags;     /* MUONH_FLAG_*                                       */
+} muonh_stats;
+
+typedef struct muonh_ctx muonh_ctx;
+
+/* Build the step for n matrices: validates the descriptors, groups matrices
+ * of equal Newton-Schulz shape, allocates the device workspace (owned by the
+ * context, freed by muonh_destroy), computes R = ||W_0||_F where asked and
+ * ||W_0||_F^2 for every matrix, and synchronises `stream` once.
+ * *out receives the context; on failure *out is set to NULL. */
+muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t n,
+                        const muonh_config* cfg, void* stream);
+
+/* One MuonH step over all matrices (the hot path).
+ *   lr     host array of n floats: the effective LR (eta^H) of each matrix,
+ *          read before the call returns.
+ *   grads  host array of n device pointers to fp32 gradients, each laid out
+ *          like its matrix's w (same rows, cols, ld); read before return.
+ *   stats  NULL, or device-accessible memory (device, managed or mapped
+ *          pinned host) for n muonh_stats, written by the last kernel.
+ * Updates every w and m in place.  Enqueued on `stream`; the caller
+ * synchronises before reading w, m or stats. */
+muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* grads,
+                        muonh_stats* stats, void* stream);
+
+/* Copy the last step's per-matrix stats to host memory (n entries);
+ * synchronises the stream of the last step. */
+muonh_status muonh_get_stats(muonh_ctx* ctx, muonh_stats* host_out);
+
+/* Write matrix i's Newton-Schulz output O of the last step, unscaled and in
+ * the orientation of w (rows x cols), as fp32 into device memory `dst` with
+ * row stride ld (elements).  Enqueued on `stream`. */
+muonh_status muonh_get_update(muonh_ctx* ctx, int32_t i, float* dst, int64_t ld, void* stream);
+
+/* Host copy of the n radii R. */
+muonh_status muonh_get_radius(const muonh_ctx* ctx, float* host_R);
+
+/* Checkpointing of the library-held state (R[], ||W_t||^2[], step count).
+ * W and M are caller-owned and saved by the caller.  With buf == NULL,
+ * *len receives the size needed.  Export synchronises the last stream. */
+muonh_status muonh_export_state(muonh_ctx* ctx, void* buf, size_t* len);
+muonh_status muonh_import_state(muonh_ctx* ctx, const void* buf, size_t len);
+
+/* Synchronises the last stream and returns MUONH_ERR_TIMEOUT if a device
+ * wait gave up since the previous call (then clears the record), else OK. */
+muonh_status muonh_device_status(muonh_ctx* ctx);
+
+/* Number of kernel launches the last muonh_step enqueued. */
+int32_t muonh_last_launch_count(const muonh_ctx* ctx);
+
+void muonh_destroy(muonh_ctx* ctx);
+
+const char* muonh_status_string(muonh_status s);
+
+/* Message of the last failure on the calling thread ("" if none). */
+const char* muonh_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* MUONH_H_ */

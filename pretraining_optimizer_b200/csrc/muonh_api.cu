@@ -1,0 +1,641 @@
+// C ABI of the MuonH step and its host-side scheduler.
+//
+// muonh_init groups the matrices by their padded Newton-Schulz shape
+// (r_pad x c_pad, r = min(rows, cols) on the wide orientation, both padded
+// to multiples of 256), allocates one zero-filled workspace per shape class
+// ([count][r_pad][c_pad] iterate ping-pong buffers and [count][r_pad][r_pad]
+// Gram and polynomial buffers), encodes one TMA descriptor per buffer and
+// box shape, and builds the tile lists of the grouped GEMM launches.  Zero
+// padding is exact for the iteration: padded rows and columns of Y, A and B
+// stay zero, so no GEMM tile is ragged.
+//
+// muonh_step enqueues, on the caller's stream:
+//   momentum_norm  (M update, ||X||^2 partials)      -> finalize_input
+//   write_x        (X / (||X|| + eps), 16-bit, wide orientation)
+//   ns_steps x { GRAM, SQUARE, APPLY }               (tcgen05 GEMMs)
+//   update_dots    (||O||^2, <W, O> partials)        -> finalize_update
+//   project        (W <- R (W - lr R O/||O||) / ||.||, Eq. (1)) -> finalize_step
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "muonh_common.cuh"
+
+using namespace muonh;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+muonh_status fail(muonh_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+#define CUDA_TRY(call)                                                                                \
+  do {                                                                                                \
+    cudaError_t e_ = (call);                                                                          \
+    if (e_ != cudaSuccess) return fail(MUONH_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+constexpr int kRing = 4;
+constexpr int64_t kMaxDim = 1 << 20;
+constexpr int64_t kMaxRPad = 16384;
+constexpr int32_t kMaxNsSteps = 64;
+constexpr uint32_t kStateMagic = 0x484E554Du;   // "MUNH"
+
+struct TileList {
+  TileDesc* dev = nullptr;
+  int32_t count = 0;
+};
+
+struct ClassHost {
+  int32_t r_pad, c_pad, count = 0;
+  ClassDev dev{};
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Largest power-of-two exponent e with bound * 2^e <= 60000 (fp16 max 65504).
+int safe_exponent(double bound) {
+  if (!(bound > 0.0) || !std::isfinite(bound)) return 0;
+  int e = static_cast<int>(std::floor(std::log2(60000.0 / bound)));
+  return std::max(-24, std::min(15, e));
+}
+
+// Bounds on the entries of Y, A = Y Y^T and B = b A + c A^2 over all
+// iterations, from the scalar map sigma -> a s + b s^3 + c s^5 on the
+// singular values (entries are bounded by the spectral norm), starting from
+// sigma_max(Y_0) <= 1 after the Frobenius normalisation.
+void scale_exponents(float a, float b, float c, int steps, int prec, int32_t* ex, int32_t* ea, int32_t* eb) {
+  if (prec == P_BF16) {
+    *ex = *ea = *eb = 0;
+    return;
+  }
+  double smax = 1.0, s_all = 1.0;
+  for (int k = 0; k < steps; ++k) {
+    double m = 0.0;
+    const int n = 8192;
+    for (int i = 0; i <= n; ++i) {
+      const double s = smax * i / n;
+      m = std::max(m, std::fabs(a * s + b * s * s * s + c * s * s * s * s * s));
+    }
+    smax = std::max(m * 1.001, 1e-30);
+    s_all = std::max(s_all, smax);
+    if (!std::isfinite(s_all) || s_all > 1e6) break;
+  }
+  const double xmax = s_all * 1.02;
+  const double amax = xmax * xmax;
+  double bmax = 0.0;
+  for (int i = 0; i <= 8192; ++i) {
+    const double l = amax * i / 8192;
+    bmax = std::max(bmax, std::fabs(b * l + c * l * l));
+  }
+  *ex = safe_exponent(xmax);
+  *ea = safe_exponent(amax);
+  *eb = safe_exponent(std::max(bmax, 1e-30));
+}
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+}  // namespace
+
+struct muonh_ctx {
+  int32_t n = 0;
+  int32_t prec = 0;
+  float eps = 0.f;
+  int device = 0;
+  int sm_count = 148;
+  int32_t max_steps = 0;
+  int64_t n_et = 0;
+  int64_t step_count = 0;
+  int32_t last_launches = 0;
+  cudaStream_t last_stream = nullptr;
+
+  std::vector<MatDev> mats;
+  std::vector<ClassHost> classes;
+  std::vector<TileList> gram_lists, apply_lists;   // per Newton-Schulz iteration
+  std::vector<void*> allocs;
+
+  MatDev* d_mats = nullptr;
+  ClassDev* d_classes = nullptr;
+  MatScal* d_scal = nullptr;
+  MatStep* d_step = nullptr;
+  int32_t* d_et_mat = nullptr;
+  float* d_part = nullptr;
+  double* d_part64 = nullptr;
+  CUtensorMap* d_tmaps = nullptr;
+  int* d_err = nullptr;
+
+  MatStep* h_step[kRing] = {};
+  cudaEvent_t ev[kRing] = {};
+  int ring = 0;
+
+  EwParams ew(muonh_stats* stats_out) const {
+    EwParams p{};
+    p.mats = d_mats;
+    p.step = d_step;
+    p.scal = d_scal;
+    p.classes = d_classes;
+    p.et_mat = d_et_mat;
+    p.n_et = n_et;
+    p.part = d_part;
+    p.part64 = d_part64;
+    p.n = n;
+    p.eps = eps;
+    p.prec = prec;
+    p.stats_out = stats_out;
+    p.err = d_err;
+    return p;
+  }
+};
+
+namespace {
+
+cudaError_t dev_alloc(muonh_ctx* ctx, void** p, size_t bytes) {
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e == cudaSuccess) ctx->allocs.push_back(*p);
+  return e;
+}
+
+void release(muonh_ctx* ctx) {
+  if (!ctx) return;
+  for (void* p : ctx->allocs) cudaFree(p);
+  ctx->allocs.clear();
+  for (int i = 0; i < kRing; ++i) {
+    if (ctx->h_step[i]) cudaFreeHost(ctx->h_step[i]);
+    if (ctx->ev[i]) cudaEventDestroy(ctx->ev[i]);
+  }
+  delete ctx;
+}
+
+muonh_status encode_map(CUtensorMap* out, void* base, int prec16_is_bf16, int64_t inner, int64_t rows,
+                        int64_t count, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(count)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner * 2), static_cast<cuuint64_t>(inner * rows * 2)};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(out, prec16_is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return MUONH_OK;
+}
+
+muonh_status check_launch(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(MUONH_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return MUONH_OK;
+}
+
+#define LAUNCH_TRY(expr, name)                              \
+  do {                                                      \
+    muonh_status st_ = check_launch((expr), name);          \
+    if (st_ != MUONH_OK) return st_;                        \
+    ++launches;                                             \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* muonh_status_string(muonh_status s) {
+  switch (s) {
+    case MUONH_OK: return "ok";
+    case MUONH_ERR_INVALID_ARG: return "invalid argument";
+    case MUONH_ERR_ALIGNMENT: return "misaligned pointer or stride";
+    case MUONH_ERR_CUDA: return "CUDA error";
+    case MUONH_ERR_OOM: return "out of device memory";
+    case MUONH_ERR_TIMEOUT: return "device wait timed out";
+    case MUONH_ERR_UNSUPPORTED: return "unsupported device or size";
+  }
+  return "unknown status";
+}
+
+const char* muonh_last_error(void) { return g_last_error.c_str(); }
+
+muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t n, const muonh_config* cfg,
+                        void* stream) {
+  g_last_error.clear();
+  if (!out) return fail(MUONH_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!mats || n <= 0 || !cfg) return fail(MUONH_ERR_INVALID_ARG, "mats/cfg NULL or n <= 0");
+  if (cfg->ns_precision < 0 || cfg->ns_precision > 2)
+    return fail(MUONH_ERR_INVALID_ARG, "ns_precision %d is not FP16, BF16 or FP32", cfg->ns_precision);
+  if (!(cfg->eps >= 0.f) || !std::isfinite(cfg->eps)) return fail(MUONH_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  for (int32_t i = 0; i < n; ++i) {
+    const muonh_matrix_desc& d = mats[i];
+    if (!d.w || !d.m) return fail(MUONH_ERR_INVALID_ARG, "matrix %d: w or m is NULL", i);
+    if (d.rows <= 0 || d.cols <= 0 || d.rows > kMaxDim || d.cols > kMaxDim)
+      return fail(MUONH_ERR_INVALID_ARG, "matrix %d: rows/cols out of range (1..%lld)", i, (long long)kMaxDim);
+    if (d.ld < d.cols) return fail(MUONH_ERR_INVALID_ARG, "matrix %d: ld < cols", i);
+    if ((reinterpret_cast<uintptr_t>(d.w) & 15) || (reinterpret_cast<uintptr_t>(d.m) & 15))
+      return fail(MUONH_ERR_ALIGNMENT, "matrix %d: w and m must be 16-byte aligned", i);
+    if (d.ns_steps < 0 || d.ns_steps > kMaxNsSteps)
+      return fail(MUONH_ERR_INVALID_ARG, "matrix %d: ns_steps %d outside [0, %d]", i, d.ns_steps, kMaxNsSteps);
+    if (!std::isfinite(d.beta) || !std::isfinite(d.ns_a) || !std::isfinite(d.ns_b) || !std::isfinite(d.ns_c) ||
+        !std::isfinite(d.radius))
+      return fail(MUONH_ERR_INVALID_ARG, "matrix %d: beta, coefficients and radius must be finite", i);
+    if (round_up(std::min(d.rows, d.cols), kPad) > kMaxRPad)
+      return fail(MUONH_ERR_UNSUPPORTED, "matrix %d: min(rows, cols) above %lld", i, (long long)kMaxRPad);
+  }
+
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  CUDA_TRY(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10)
+    return fail(MUONH_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev, prop.major,
+                prop.minor);
+  CUDA_TRY(ns_gemm_set_attributes());
+
+  muonh_ctx* ctx = new muonh_ctx();
+  ctx->n = n;
+  ctx->prec = cfg->ns_precision;
+  ctx->eps = cfg->eps;
+  ctx->device = dev;
+  ctx->sm_count = prop.multiProcessorCount;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ctx->last_stream = s;
+
+  struct Guard {
+    muonh_ctx*& c;
+    bool ok = false;
+    ~Guard() {
+      if (!ok) release(c);
+    }
+  } guard{ctx};
+
+  // ---- per-matrix layout and shape classes
+  std::map<std::pair<int64_t, int64_t>, int> class_of;
+  ctx->mats.resize(n);
+  int64_t n_et = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const muonh_matrix_desc& d = mats[i];
+    MatDev& md = ctx->mats[i];
+    md = MatDev{};
+    md.w = d.w;
+    md.m = d.m;
+    md.rows = d.rows;
+    md.cols = d.cols;
+    md.ld = d.ld;
+    md.r = static_cast<int32_t>(std::min(d.rows, d.cols));
+    md.c = static_cast<int32_t>(std::max(d.rows, d.cols));
+    md.transposed = d.rows > d.cols ? 1 : 0;
+    md.vec = (d.cols % 4 == 0 && d.ld % 4 == 0) ? 1 : 0;
+    md.beta = d.beta;
+    md.nesterov = d.nesterov ? 1 : 0;
+    md.ns_steps = d.ns_steps;
+    md.a = d.ns_a;
+    md.b = d.ns_b;
+    md.c_coef = d.ns_c;
+    scale_exponents(d.ns_a, d.ns_b, d.ns_c, d.ns_steps, ctx->prec, &md.ex, &md.ea, &md.eb);
+    md.et_rows = static_cast<int32_t>((d.rows + kEwTile - 1) / kEwTile);
+    md.et_cols = static_cast<int32_t>((d.cols + kEwTile - 1) / kEwTile);
+    md.et_begin = n_et;
+    n_et += static_cast<int64_t>(md.et_rows) * md.et_cols;
+    const std::pair<int64_t, int64_t> key(round_up(md.r, kPad), round_up(md.c, kPad));
+    auto it = class_of.find(key);
+    if (it == class_of.end()) {
+      ClassHost ch;
+      ch.r_pad = static_cast<int32_t>(key.first);
+      ch.c_pad = static_cast<int32_t>(key.second);
+      it = class_of.emplace(key, static_cast<int>(ctx->classes.size())).first;
+      ctx->classes.push_back(ch);
+    }
+    md.cls = it->second;
+    md.z = ctx->classes[md.cls].count++;
+    ctx->max_steps = std::max(ctx->max_steps, d.ns_steps);
+  }
+  ctx->n_et = n_et;
+
+  // ---- workspace
+  const int parts = ctx->prec == P_FP32 ? 2 : 1;
+  for (ClassHost& ch : ctx->classes) {
+    ClassDev& cd = ch.dev;
+    cd.r_pad = ch.r_pad;
+    cd.c_pad = ch.c_pad;
+    cd.count = ch.count;
+    cd.x_stride = static_cast<int64_t>(ch.r_pad) * ch.c_pad;
+    cd.a_stride = static_cast<int64_t>(ch.r_pad) * ch.r_pad;
+    const size_t xb = static_cast<size_t>(cd.x_stride) * ch.count * 2;
+    const size_t ab = static_cast<size_t>(cd.a_stride) * ch.count * 2;
+    for (int part = 0; part < parts; ++part) {
+      for (int buf = 0; buf < 2; ++buf) {
+        if (dev_alloc(ctx, &cd.x[buf][part], xb) != cudaSuccess)
+          return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", xb);
+        CUDA_TRY(cudaMemsetAsync(cd.x[buf][part], 0, xb, s));
+      }
+      if (dev_alloc(ctx, &cd.a[part], ab) != cudaSuccess || dev_alloc(ctx, &cd.b[part], ab) != cudaSuccess)
+        return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", ab);
+      CUDA_TRY(cudaMemsetAsync(cd.a[part], 0, ab, s));
+      CUDA_TRY(cudaMemsetAsync(cd.b[part], 0, ab, s));
+    }
+  }
+
+  // ---- tensor maps: TM_PER_CLASS per class
+  std::vector<CUtensorMap> maps(ctx->classes.size() * TM_PER_CLASS);
+  std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
+  for (size_t ci = 0; ci < ctx->classes.size(); ++ci) {
+    ClassDev& cd = ctx->classes[ci].dev;
+    cd.tm_base = static_cast<int32_t>(ci * TM_PER_CLASS);
+    CUtensorMap* m = &maps[cd.tm_base];
+    for (int part = 0; part < parts; ++part) {
+      const int bf = (ctx->prec == P_BF16 && part == 0) ? 1 : 0;
+      for (int buf = 0; buf < 2; ++buf) {
+        muonh_status st;
+        if ((st = encode_map(&m[tm_x(TM_X_K128, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBM)))
+          return st;
+        if ((st = encode_map(&m[tm_x(TM_X_K256, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBN)))
+          return st;
+        if ((st = encode_map(&m[tm_x(TM_X_MN, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBK)))
+          return st;
+      }
+      muonh_status st;
+      if ((st = encode_map(&m[TM_A_K128 + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
+      if ((st = encode_map(&m[TM_A_K256 + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN))) return st;
+      if ((st = encode_map(&m[TM_B_K128 + part], cd.b[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
+    }
+  }
+
+  // ---- device tables
+  if (dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_tmaps), maps.size() * sizeof(CUtensorMap)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_mats), n * sizeof(MatDev)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_classes), ctx->classes.size() * sizeof(ClassDev)) !=
+          cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_scal), n * sizeof(MatScal)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_step), n * sizeof(MatStep)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_et_mat), n_et * sizeof(int32_t)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part), 2 * n_et * sizeof(float)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part64), n_et * sizeof(double)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), sizeof(int)) != cudaSuccess)
+    return fail(MUONH_ERR_OOM, "allocation of the device tables failed");
+
+  std::vector<ClassDev> cdev;
+  for (const ClassHost& ch : ctx->classes) cdev.push_back(ch.dev);
+  std::vector<int32_t> et_mat(n_et);
+  for (int32_t i = 0; i < n; ++i) {
+    const MatDev& md = ctx->mats[i];
+    std::fill(et_mat.begin() + md.et_begin, et_mat.begin() + md.et_begin + int64_t(md.et_rows) * md.et_cols, i);
+  }
+  std::vector<MatScal> scal(n);
+  for (int32_t i = 0; i < n; ++i) {
+    scal[i] = MatScal{};
+    scal[i].R = mats[i].radius > 0.f ? mats[i].radius : 0.f;
+  }
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_mats, ctx->mats.data(), n * sizeof(MatDev), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_classes, cdev.data(), cdev.size() * sizeof(ClassDev), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_et_mat, et_mat.data(), n_et * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_scal, scal.data(), n * sizeof(MatScal), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, sizeof(int), s));
+
+  // ---- Newton-Schulz tile lists, one pair per iteration (shared when equal)
+  std::vector<int32_t> prev_active;
+  for (int32_t k = 0; k < ctx->max_steps; ++k) {
+    std::vector<int32_t> active;
+    for (int32_t i = 0; i < n; ++i)
+      if (ctx->mats[i].ns_steps > k) active.push_back(i);
+    if (k > 0 && active == prev_active) {
+      ctx->gram_lists.push_back(ctx->gram_lists.back());
+      ctx->apply_lists.push_back(ctx->apply_lists.back());
+      continue;
+    }
+    prev_active = active;
+    // longest tiles first (the K extent), then matrix by matrix for L2 reuse
+    std::vector<int32_t> order = active;
+    std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+      const ClassHost& cx = ctx->classes[ctx->mats[x].cls];
+      const ClassHost& cy = ctx->classes[ctx->mats[y].cls];
+      if (cx.c_pad != cy.c_pad) return cx.c_pad > cy.c_pad;
+      return cx.r_pad > cy.r_pad;
+    });
+    std::vector<TileDesc> gram, apply;
+    for (int32_t i : order) {
+      const ClassHost& ch = ctx->classes[ctx->mats[i].cls];
+      for (int bi = 0; bi < ch.r_pad / kBM; ++bi)
+        for (int bj = 0; bj < ch.r_pad / kBN; ++bj)
+          if (bj * kBN + kBN - 1 >= bi * kBM) gram.push_back(TileDesc{i, int16_t(bi), int16_t(bj)});
+    }
+    std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+      return ctx->classes[ctx->mats[x].cls].r_pad > ctx->classes[ctx->mats[y].cls].r_pad;
+    });
+    for (int32_t i : order) {
+      const ClassHost& ch = ctx->classes[ctx->mats[i].cls];
+      for (int bi = 0; bi < ch.r_pad / kBM; ++bi)
+        for (int bj = 0; bj < ch.c_pad / kBN; ++bj) apply.push_back(TileDesc{i, int16_t(bi), int16_t(bj)});
+    }
+    TileList gl, al;
+    gl.count = static_cast<int32_t>(gram.size());
+    al.count = static_cast<int32_t>(apply.size());
+    if (dev_alloc(ctx, reinterpret_cast<void**>(&gl.dev), std::max<size_t>(1, gram.size()) * sizeof(TileDesc)) !=
+            cudaSuccess ||
+        dev_alloc(ctx, reinterpret_cast<void**>(&al.dev), std::max<size_t>(1, apply.size()) * sizeof(TileDesc)) !=
+            cudaSuccess)
+      return fail(MUONH_ERR_OOM, "tile list allocation failed");
+    if (!gram.empty())
+      CUDA_TRY(cudaMemcpyAsync(gl.dev, gram.data(), gram.size() * sizeof(TileDesc), cudaMemcpyHostToDevice, s));
+    if (!apply.empty())
+      CUDA_TRY(cudaMemcpyAsync(al.dev, apply.data(), apply.size() * sizeof(TileDesc), cudaMemcpyHostToDevice, s));
+    ctx->gram_lists.push_back(gl);
+    ctx->apply_lists.push_back(al);
+  }
+
+  // ---- pinned staging ring for the per-step table
+  for (int i = 0; i < kRing; ++i) {
+    CUDA_TRY(cudaMallocHost(reinterpret_cast<void**>(&ctx->h_step[i]), n * sizeof(MatStep)));
+    CUDA_TRY(cudaEventCreateWithFlags(&ctx->ev[i], cudaEventDisableTiming));
+  }
+
+  // ---- R = ||W_0||_F where asked, and ||W_0||^2 for every matrix
+  const EwParams p = ctx->ew(nullptr);
+  int launches = 0;
+  const int grid = ctx->sm_count * 8;
+  LAUNCH_TRY(launch_init_norm(p, grid, s), "init_norm");
+  LAUNCH_TRY(launch_finalize_init(p, s), "finalize_init");
+  CUDA_TRY(cudaStreamSynchronize(s));
+  guard.ok = true;
+  *out = ctx;
+  return MUONH_OK;
+}
+
+muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* grads, muonh_stats* stats,
+                        void* stream) {
+  g_last_error.clear();
+  if (!ctx || !lr || !grads) return fail(MUONH_ERR_INVALID_ARG, "ctx, lr or grads is NULL");
+  for (int32_t i = 0; i < ctx->n; ++i) {
+    if (!grads[i]) return fail(MUONH_ERR_INVALID_ARG, "grads[%d] is NULL", i);
+    if (reinterpret_cast<uintptr_t>(grads[i]) & 15) return fail(MUONH_ERR_ALIGNMENT, "grads[%d] not 16-byte aligned", i);
+    if (!std::isfinite(lr[i])) return fail(MUONH_ERR_INVALID_ARG, "lr[%d] is not finite", i);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // stage (grad pointer, lr) in a pinned slot; reuse waits only if the GPU is kRing steps behind
+  const int slot = ctx->ring;
+  ctx->ring = (ctx->ring + 1) % kRing;
+  CUDA_TRY(cudaEventSynchronize(ctx->ev[slot]));
+  for (int32_t i = 0; i < ctx->n; ++i) ctx->h_step[slot][i] = MatStep{grads[i], lr[i], 0.f};
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_step, ctx->h_step[slot], ctx->n * sizeof(MatStep), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaEventRecord(ctx->ev[slot], s));
+
+  const EwParams p = ctx->ew(stats);
+  const int grid = ctx->sm_count * 8;
+  int launches = 0;
+  LAUNCH_TRY(launch_momentum_norm(p, grid, s), "momentum_norm");
+  LAUNCH_TRY(launch_finalize_input(p, s), "finalize_input");
+  LAUNCH_TRY(launch_write_x(p, grid, s), "write_x");
+  for (int32_t k = 0; k < ctx->max_steps; ++k) {
+    NsParams np{};
+    np.mats = ctx->d_mats;
+    np.classes = ctx->d_classes;
+    np.tmaps = ctx->d_tmaps;
+    np.err = ctx->d_err;
+    np.src = k & 1;
+    np.tiles = ctx->gram_lists[k].dev;
+    np.ntiles = ctx->gram_lists[k].count;
+    const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
+    LAUNCH_TRY(launch_ns_gemm(M_GRAM, ctx->prec, np, ggrid, s), "ns_gram");
+    LAUNCH_TRY(launch_ns_gemm(M_SQUARE, ctx->prec, np, ggrid, s), "ns_square");
+    np.tiles = ctx->apply_lists[k].dev;
+    np.ntiles = ctx->apply_lists[k].count;
+    LAUNCH_TRY(launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), s), "ns_apply");
+  }
+  LAUNCH_TRY(launch_update_dots(p, grid, s), "update_dots");
+  LAUNCH_TRY(launch_finalize_update(p, s), "finalize_update");
+  LAUNCH_TRY(launch_project(p, grid, s), "project");
+  LAUNCH_TRY(launch_finalize_step(p, s), "finalize_step");
+  ctx->last_launches = launches;
+  ctx->last_stream = s;
+  ++ctx->step_count;
+  return MUONH_OK;
+}
+
+muonh_status muonh_get_stats(muonh_ctx* ctx, muonh_stats* host_out) {
+  g_last_error.clear();
+  if (!ctx || !host_out) return fail(MUONH_ERR_INVALID_ARG, "ctx or host_out is NULL");
+  CUDA_TRY(cudaStreamSynchronize(ctx->last_stream));
+  std::vector<MatScal> scal(ctx->n);
+  CUDA_TRY(cudaMemcpy(scal.data(), ctx->d_scal, ctx->n * sizeof(MatScal), cudaMemcpyDeviceToHost));
+  for (int32_t i = 0; i < ctx->n; ++i) host_out[i] = scal[i].stats;
+  return MUONH_OK;
+}
+
+muonh_status muonh_get_update(muonh_ctx* ctx, int32_t i, float* dst, int64_t ld, void* stream) {
+  g_last_error.clear();
+  if (!ctx || !dst) return fail(MUONH_ERR_INVALID_ARG, "ctx or dst is NULL");
+  if (i < 0 || i >= ctx->n) return fail(MUONH_ERR_INVALID_ARG, "matrix index %d out of range", i);
+  if (ld < ctx->mats[i].cols) return fail(MUONH_ERR_INVALID_ARG, "ld < cols");
+  int launches = 0;
+  LAUNCH_TRY(launch_export_update(ctx->ew(nullptr), i, dst, ld, static_cast<cudaStream_t>(stream)), "export_update");
+  return MUONH_OK;
+}
+
+muonh_status muonh_get_radius(const muonh_ctx* ctx, float* host_R) {
+  g_last_error.clear();
+  if (!ctx || !host_R) return fail(MUONH_ERR_INVALID_ARG, "ctx or host_R is NULL");
+  CUDA_TRY(cudaStreamSynchronize(ctx->last_stream));
+  std::vector<MatScal> scal(ctx->n);
+  CUDA_TRY(cudaMemcpy(scal.data(), ctx->d_scal, ctx->n * sizeof(MatScal), cudaMemcpyDeviceToHost));
+  for (int32_t i = 0; i < ctx->n; ++i) host_R[i] = scal[i].R;
+  return MUONH_OK;
+}
+
+muonh_status muonh_export_state(muonh_ctx* ctx, void* buf, size_t* len) {
+  g_last_error.clear();
+  if (!ctx || !len) return fail(MUONH_ERR_INVALID_ARG, "ctx or len is NULL");
+  const size_t need = 16 + static_cast<size_t>(ctx->n) * (sizeof(float) + sizeof(double));
+  if (!buf) {
+    *len = need;
+    return MUONH_OK;
+  }
+  if (*len < need) return fail(MUONH_ERR_INVALID_ARG, "buffer of %zu bytes, %zu needed", *len, need);
+  CUDA_TRY(cudaStreamSynchronize(ctx->last_stream));
+  std::vector<MatScal> scal(ctx->n);
+  CUDA_TRY(cudaMemcpy(scal.data(), ctx->d_scal, ctx->n * sizeof(MatScal), cudaMemcpyDeviceToHost));
+  uint8_t* o = static_cast<uint8_t*>(buf);
+  const uint32_t hdr[2] = {kStateMagic, static_cast<uint32_t>(ctx->n)};
+  std::memcpy(o, hdr, 8);
+  std::memcpy(o + 8, &ctx->step_count, 8);
+  o += 16;
+  for (int32_t i = 0; i < ctx->n; ++i) {
+    std::memcpy(o, &scal[i].R, sizeof(float));
+    std::memcpy(o + sizeof(float), &scal[i].wnorm2, sizeof(double));
+    o += sizeof(float) + sizeof(double);
+  }
+  *len = need;
+  return MUONH_OK;
+}
+
+muonh_status muonh_import_state(muonh_ctx* ctx, const void* buf, size_t len) {
+  g_last_error.clear();
+  if (!ctx || !buf) return fail(MUONH_ERR_INVALID_ARG, "ctx or buf is NULL");
+  const size_t need = 16 + static_cast<size_t>(ctx->n) * (sizeof(float) + sizeof(double));
+  if (len != need) return fail(MUONH_ERR_INVALID_ARG, "state of %zu bytes, %zu expected", len, need);
+  const uint8_t* in = static_cast<const uint8_t*>(buf);
+  uint32_t hdr[2];
+  std::memcpy(hdr, in, 8);
+  if (hdr[0] != kStateMagic || hdr[1] != static_cast<uint32_t>(ctx->n))
+    return fail(MUONH_ERR_INVALID_ARG, "state was not exported from a context with %d matrices", ctx->n);
+  CUDA_TRY(cudaStreamSynchronize(ctx->last_stream));
+  std::vector<MatScal> scal(ctx->n);
+  CUDA_TRY(cudaMemcpy(scal.data(), ctx->d_scal, ctx->n * sizeof(MatScal), cudaMemcpyDeviceToHost));
+  int64_t steps;
+  std::memcpy(&steps, in + 8, 8);
+  in += 16;
+  for (int32_t i = 0; i < ctx->n; ++i) {
+    std::memcpy(&scal[i].R, in, sizeof(float));
+    std::memcpy(&scal[i].wnorm2, in + sizeof(float), sizeof(double));
+    in += sizeof(float) + sizeof(double);
+  }
+  CUDA_TRY(cudaMemcpy(ctx->d_scal, scal.data(), ctx->n * sizeof(MatScal), cudaMemcpyHostToDevice));
+  ctx->step_count = steps;
+  return MUONH_OK;
+}
+
+muonh_status muonh_device_status(muonh_ctx* ctx) {
+  g_last_error.clear();
+  if (!ctx) return fail(MUONH_ERR_INVALID_ARG, "ctx is NULL");
+  CUDA_TRY(cudaStreamSynchronize(ctx->last_stream));
+  int err = 0;
+  CUDA_TRY(cudaMemcpy(&err, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (err) {
+    CUDA_TRY(cudaMemset(ctx->d_err, 0, sizeof(int)));
+    return fail(MUONH_ERR_TIMEOUT, "a device-side wait gave up (Newton-Schulz GEMM pipeline)");
+  }
+  return MUONH_OK;
+}
+
+int32_t muonh_last_launch_count(const muonh_ctx* ctx) { return ctx ? ctx->last_launches : 0; }
+
+void muonh_destroy(muonh_ctx* ctx) {
+  if (!ctx) return;
+  cudaDeviceSynchronize();
+  release(ctx);
+}
+
+}  // extern "C"

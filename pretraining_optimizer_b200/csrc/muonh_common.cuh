@@ -1,0 +1,272 @@
+// Internal definitions shared by the CUDA translation units of libmuonh:
+// device-side tables, launch parameters and inline-PTX wrappers for
+// mbarrier, TMA and tcgen05 (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/muonh.h"
+
+namespace muonh {
+
+// ------------------------------------------------------------------ sizes
+constexpr int kEwTile = 64;          // elementwise tiles: 64 x 64 elements of W
+constexpr int kEwThreads = 256;
+constexpr int kBM = 128;             // Newton-Schulz GEMM tile: 128 x 256 x 64
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr int kPad = 256;            // NS buffers are padded to multiples of 256
+constexpr int kGemmThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
+
+enum Prec { P_FP16 = 0, P_BF16 = 1, P_FP32 = 2 };
+enum Mode { M_GRAM = 0, M_SQUARE = 1, M_APPLY = 2 };
+
+// Tensor-map slots of one shape class.  "hi" buffers hold the 16-bit
+// operand (fp16/bf16), "lo" buffers the fp16 residual in FP32 mode.
+enum TmSlot {
+  TM_X_K128 = 0,   // X[buf] as K-major operand, 128-row box   (+buf, +2*part)
+  TM_X_K256 = 4,   // X[buf] as K-major operand, 256-row box
+  TM_X_MN = 8,     // X[buf] as MN-major operand, 64 x 64 box
+  TM_A_K128 = 12,  // A, 128-row box (+part)
+  TM_A_K256 = 14,  // A, 256-row box (+part)
+  TM_B_K128 = 16,  // B, 128-row box (+part)
+  TM_PER_CLASS = 18
+};
+__host__ __device__ inline int tm_x(int base, int buf, int part) { return base + buf + 2 * part; }
+
+struct MatDev {
+  float* w;
+  float* m;
+  int64_t rows, cols, ld;
+  int32_t r, c;              // Newton-Schulz orientation, r <= c
+  int32_t transposed;        // rows > cols: X holds the transpose
+  int32_t cls, z;            // shape class and slot within it
+  int32_t vec;               // cols % 4 == 0: float4 path
+  float beta;
+  int32_t nesterov;
+  int32_t ns_steps;
+  float a, b, c_coef;
+  int32_t ex, ea, eb;        // power-of-two scales of stored X, A, B
+  int32_t et_rows, et_cols;  // elementwise tile grid
+  int64_t et_begin;          // first elementwise tile
+};
+
+struct ClassDev {
+  int32_t r_pad, c_pad, count, tm_base;
+  void* x[2][2];             // [buf][part]
+  void* a[2];                // [part]
+  void* b[2];
+  int64_t x_stride, a_stride;   // elements per matrix
+};
+
+struct MatStep {             // per step, copied from the host
+  const float* g;
+  float lr;
+  float pad_;
+};
+
+struct MatScal {             // device-resident per-matrix scalars
+  float R;
+  float xscale;              // 2^ex / (||X|| + eps)
+  float kw, ko;              // projection: W <- kw W + ko O_stored
+  int32_t mode;              // 0 step, 1 re-project only, 2 keep W
+  uint32_t flags;
+  double wnorm2;             // ||W_t||^2 (measured on the stored W)
+  muonh_stats stats;
+};
+
+struct TileDesc {
+  int32_t mat;
+  int16_t bi, bj;
+};
+
+struct NsParams {
+  const TileDesc* tiles;
+  int32_t ntiles;
+  int32_t src;               // X buffer read by this phase
+  const MatDev* mats;
+  const ClassDev* classes;
+  const CUtensorMap* tmaps;
+  int* err;
+};
+
+struct EwParams {
+  const MatDev* mats;
+  const MatStep* step;
+  MatScal* scal;
+  const ClassDev* classes;
+  const int32_t* et_mat;     // elementwise tile -> matrix
+  int64_t n_et;
+  float* part;               // per-tile partials
+  double* part64;
+  int32_t n;
+  float eps;
+  int32_t prec;
+  muonh_stats* stats_out;
+  const int* err;
+};
+
+// -------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity; gives up after kWaitLimitNs or
+// when another role already recorded an error.  Returns false on give-up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 255u) == 0u) {
+      if (*reinterpret_cast<volatile int*>(err) != 0) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        atomicOr(err, 1);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (fp16 or bf16 in, fp32 accumulate)
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on `bar` once all previously issued MMAs of this thread completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i gets lane (base+i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;   // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A K-major, B K- or MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n, int ab_bf16, int b_mn_major) {
+  return (1u << 4) | (static_cast<uint32_t>(ab_bf16) << 7) | (static_cast<uint32_t>(ab_bf16) << 10) |
+         (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// --------------------------------------------------------- launch helpers
+cudaError_t launch_ns_gemm(int mode, int prec, const NsParams& p, int grid, cudaStream_t s);
+size_t ns_gemm_smem_bytes(int prec);
+cudaError_t ns_gemm_set_attributes();
+
+cudaError_t launch_init_norm(const EwParams& p, int grid, cudaStream_t s);
+cudaError_t launch_finalize_init(const EwParams& p, cudaStream_t s);
+cudaError_t launch_momentum_norm(const EwParams& p, int grid, cudaStream_t s);
+cudaError_t launch_finalize_input(const EwParams& p, cudaStream_t s);
+cudaError_t launch_write_x(const EwParams& p, int grid, cudaStream_t s);
+cudaError_t launch_update_dots(const EwParams& p, int grid, cudaStream_t s);
+cudaError_t launch_finalize_update(const EwParams& p, cudaStream_t s);
+cudaError_t launch_project(const EwParams& p, int grid, cudaStream_t s);
+cudaError_t launch_finalize_step(const EwParams& p, cudaStream_t s);
+cudaError_t launch_export_update(const EwParams& p, int mat, float* dst, int64_t ld, cudaStream_t s);
+
+}  // namespace muonh

@@ -1,0 +1,548 @@
+// HBM-bound kernels of the MuonH step (sm_100a): momentum, the Frobenius
+// normalisation of the Newton-Schulz input, the hyperball projection of the
+// Puro-2B report (Sec. 3.3, Eq. (1)) and the per-matrix reductions.
+//
+// Every kernel walks 64 x 64 tiles of the weights' own layout (rows x cols,
+// row stride ld) in a persistent grid; a tile belongs to one matrix, so all
+// branches on matrix properties are block-uniform.  Per-tile partial sums go
+// to a fixed slot; the finalize kernels (one block per matrix) add the slots
+// of a matrix in a fixed order in fp64, so every result is bitwise
+// reproducible run to run.
+#include "muonh_common.cuh"
+
+namespace muonh {
+namespace {
+
+constexpr int kTy = kEwThreads / 16;    // 16 rows per pass, 16 threads x float4 per row
+
+struct TileCoord {
+  int mi;
+  int64_t r0, c0;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const EwParams& p, int64_t e) {
+  TileCoord t;
+  t.mi = p.et_mat[e];
+  const MatDev& md = p.mats[t.mi];
+  const int64_t local = e - md.et_begin;
+  t.r0 = (local / md.et_cols) * kEwTile;
+  t.c0 = (local % md.et_cols) * kEwTile;
+  return t;
+}
+
+// Load 4 consecutive fp32 (row, col..col+3), zero outside the matrix.
+__device__ __forceinline__ float4 load4(const float* base, const MatDev& md, int64_t row, int64_t col) {
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (row >= md.rows) return v;
+  const float* src = base + row * md.ld + col;
+  if (md.vec) {
+    if (col < md.cols) v = *reinterpret_cast<const float4*>(src);
+  } else {
+    if (col + 0 < md.cols) v.x = src[0];
+    if (col + 1 < md.cols) v.y = src[1];
+    if (col + 2 < md.cols) v.z = src[2];
+    if (col + 3 < md.cols) v.w = src[3];
+  }
+  return v;
+}
+
+__device__ __forceinline__ void store4(float* base, const MatDev& md, int64_t row, int64_t col, float4 v) {
+  if (row >= md.rows) return;
+  float* dst = base + row * md.ld + col;
+  if (md.vec) {
+    if (col < md.cols) *reinterpret_cast<float4*>(dst) = v;
+  } else {
+    if (col + 0 < md.cols) dst[0] = v.x;
+    if (col + 1 < md.cols) dst[1] = v.y;
+    if (col + 2 < md.cols) dst[2] = v.z;
+    if (col + 3 < md.cols) dst[3] = v.w;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ T block_sum(T v, T* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5;
+  __syncthreads();   // red may still be read by a previous call
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  T s = 0;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kEwThreads / 32; ++i) s += red[i];
+  return s;   // valid in thread 0
+}
+
+// ---------------------------------------------------- 16-bit X storage
+__device__ __forceinline__ void put16(void* hi, void* lo, int64_t off, float v, int prec) {
+  if (prec == P_BF16) {
+    reinterpret_cast<__nv_bfloat16*>(hi)[off] = __float2bfloat16_rn(v);
+  } else {
+    const __half h = __float2half_rn(v);
+    reinterpret_cast<__half*>(hi)[off] = h;
+    if (prec == P_FP32) reinterpret_cast<__half*>(lo)[off] = __float2half_rn(v - __half2float(h));
+  }
+}
+
+__device__ __forceinline__ float get16(const void* hi, const void* lo, int64_t off, int prec) {
+  if (prec == P_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(hi)[off]);
+  float v = __half2float(reinterpret_cast<const __half*>(hi)[off]);
+  if (prec == P_FP32) v += __half2float(reinterpret_cast<const __half*>(lo)[off]);
+  return v;
+}
+
+struct XView {
+  void* hi;
+  void* lo;
+  int64_t ld;   // c_pad
+};
+
+__device__ __forceinline__ XView x_view(const EwParams& p, const MatDev& md, int buf) {
+  const ClassDev& cd = p.classes[md.cls];
+  XView v;
+  const int64_t off = md.z * cd.x_stride * 2;
+  v.hi = static_cast<uint8_t*>(cd.x[buf][0]) + off;
+  v.lo = cd.x[buf][1] ? static_cast<uint8_t*>(cd.x[buf][1]) + off : nullptr;
+  v.ld = cd.c_pad;
+  return v;
+}
+
+// Read the 64 x 64 tile of O (W orientation, stored scale) into tile[r][c].
+__device__ __forceinline__ void load_o_tile(const EwParams& p, const MatDev& md, const TileCoord& tc,
+                                            float (*tile)[kEwTile + 1]) {
+  const XView xv = x_view(p, md, md.ns_steps & 1);
+  if (!md.transposed) {
+    // O(p, q) = X[p][q]
+    for (int i = threadIdx.x; i < kEwTile * kEwTile; i += kEwThreads) {
+      const int r = i / kEwTile, c = i % kEwTile;
+      tile[r][c] = get16(xv.hi, xv.lo, (tc.r0 + r) * xv.ld + tc.c0 + c, p.prec);
+    }
+  } else {
+    // O(p, q) = X[q][p]: read X rows q (coalesced along p), write transposed
+    for (int i = threadIdx.x; i < kEwTile * kEwTile; i += kEwThreads) {
+      const int q = i / kEwTile, r = i % kEwTile;
+      tile[r][q] = get16(xv.hi, xv.lo, (tc.c0 + q) * xv.ld + tc.r0 + r, p.prec);
+    }
+  }
+}
+
+// ------------------------------------------------------------- kernels
+__global__ void __launch_bounds__(kEwThreads) init_norm_kernel(const EwParams p) {
+  __shared__ double red[kEwThreads / 32];
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+    const TileCoord tc = tile_coord(p, e);
+    const MatDev& md = p.mats[tc.mi];
+    double acc = 0.0;
+    for (int j = 0; j < kEwTile / kTy; ++j) {
+      const float4 w = load4(md.w, md, tc.r0 + ty + kTy * j, tc.c0 + tx * 4);
+      acc += (double)w.x * w.x + (double)w.y * w.y + (double)w.z * w.z + (double)w.w * w.w;
+    }
+    const double s = block_sum(acc, red);
+    if (threadIdx.x == 0) p.part64[e] = s;
+  }
+}
+
+// M <- beta M + G; X = G + beta M (Nesterov) or M; partial ||X||^2.
+__global__ void __launch_bounds__(kEwThreads) momentum_norm_kernel(const EwParams p) {
+  __shared__ float red[kEwThreads / 32];
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+    const TileCoord tc = tile_coord(p, e);
+    const MatDev& md = p.mats[tc.mi];
+    const float* g = p.step[tc.mi].g;
+    const float beta = md.beta;
+    constexpr int J = kEwTile / kTy;
+    float4 gv[J], mv[J];
+    // issue every load of the tile before the first store
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int64_t row = tc.r0 + ty + kTy * j, col = tc.c0 + tx * 4;
+      gv[j] = load4(g, md, row, col);
+      mv[j] = load4(md.m, md, row, col);
+    }
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int64_t row = tc.r0 + ty + kTy * j, col = tc.c0 + tx * 4;
+      float4 m = mv[j];
+      m.x = fmaf(beta, m.x, gv[j].x);
+      m.y = fmaf(beta, m.y, gv[j].y);
+      m.z = fmaf(beta, m.z, gv[j].z);
+      m.w = fmaf(beta, m.w, gv[j].w);
+      store4(md.m, md, row, col, m);
+      float4 x = m;
+      if (md.nesterov) {
+        x.x = fmaf(beta, m.x, gv[j].x);
+        x.y = fmaf(beta, m.y, gv[j].y);
+        x.z = fmaf(beta, m.z, gv[j].z);
+        x.w = fmaf(beta, m.w, gv[j].w);
+      }
+      acc = fmaf(x.x, x.x, acc);
+      acc = fmaf(x.y, x.y, acc);
+      acc = fmaf(x.z, x.z, acc);
+      acc = fmaf(x.w, x.w, acc);
+    }
+    const float s = block_sum(acc, red);
+    if (threadIdx.x == 0) p.part[e] = s;
+  }
+}
+
+// X_stored = xscale * X into NS buffer 0 (wide orientation, transposed for tall W).
+__global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
+  __shared__ float tile[kEwTile][kEwTile + 1];
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+    const TileCoord tc = tile_coord(p, e);
+    const MatDev& md = p.mats[tc.mi];
+    const float* g = p.step[tc.mi].g;
+    const float beta = md.beta;
+    const float xs = p.scal[tc.mi].xscale;
+    const XView xv = x_view(p, md, 0);
+    if (!md.transposed) {
+#pragma unroll
+      for (int j = 0; j < kEwTile / kTy; ++j) {
+        const int64_t row = tc.r0 + ty + kTy * j, col = tc.c0 + tx * 4;
+        const float4 gv = load4(g, md, row, col);
+        const float4 mv = load4(md.m, md, row, col);
+        float4 x = mv;
+        if (md.nesterov) {
+          x.x = fmaf(beta, mv.x, gv.x);
+          x.y = fmaf(beta, mv.y, gv.y);
+          x.z = fmaf(beta, mv.z, gv.z);
+          x.w = fmaf(beta, mv.w, gv.w);
+        }
+        const int64_t off = row * xv.ld + col;
+        if (p.prec == P_FP16) {
+          __half2 h01 = __floats2half2_rn(x.x * xs, x.y * xs);
+          __half2 h23 = __floats2half2_rn(x.z * xs, x.w * xs);
+          uint2 u;
+          u.x = *reinterpret_cast<uint32_t*>(&h01);
+          u.y = *reinterpret_cast<uint32_t*>(&h23);
+          *reinterpret_cast<uint2*>(static_cast<__half*>(xv.hi) + off) = u;
+        } else {
+          put16(xv.hi, xv.lo, off + 0, x.x * xs, p.prec);
+          put16(xv.hi, xv.lo, off + 1, x.y * xs, p.prec);
+          put16(xv.hi, xv.lo, off + 2, x.z * xs, p.prec);
+          put16(xv.hi, xv.lo, off + 3, x.w * xs, p.prec);
+        }
+      }
+    } else {
+      __syncthreads();   // previous tile's readers are done with `tile`
+#pragma unroll
+      for (int j = 0; j < kEwTile / kTy; ++j) {
+        const int r = ty + kTy * j;
+        const int64_t row = tc.r0 + r, col = tc.c0 + tx * 4;
+        const float4 gv = load4(g, md, row, col);
+        const float4 mv = load4(md.m, md, row, col);
+        float4 x = mv;
+        if (md.nesterov) {
+          x.x = fmaf(beta, mv.x, gv.x);
+          x.y = fmaf(beta, mv.y, gv.y);
+          x.z = fmaf(beta, mv.z, gv.z);
+          x.w = fmaf(beta, mv.w, gv.w);
+        }
+        tile[r][tx * 4 + 0] = x.x * xs;
+        tile[r][tx * 4 + 1] = x.y * xs;
+        tile[r][tx * 4 + 2] = x.z * xs;
+        tile[r][tx * 4 + 3] = x.w * xs;
+      }
+      __syncthreads();
+      // X[q][p] = tile[p][q]: thread writes 16 consecutive p of one q
+      const int q = threadIdx.x / 4, p0 = (threadIdx.x % 4) * 16;
+      const int64_t off = (tc.c0 + q) * xv.ld + tc.r0 + p0;
+      if (p.prec == P_FP16) {
+        uint4 u[2];
+        __half* h = reinterpret_cast<__half*>(u);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) h[i] = __float2half_rn(tile[p0 + i][q]);
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(xv.hi) + off);
+        dst[0] = u[0];
+        dst[1] = u[1];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) put16(xv.hi, xv.lo, off + i, tile[p0 + i][q], p.prec);
+      }
+    }
+  }
+}
+
+// Partial ||O||^2 and <W, O> (O at its stored scale).
+__global__ void __launch_bounds__(kEwThreads) update_dots_kernel(const EwParams p) {
+  __shared__ float tile[kEwTile][kEwTile + 1];
+  __shared__ float red[kEwThreads / 32];
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+    const TileCoord tc = tile_coord(p, e);
+    const MatDev& md = p.mats[tc.mi];
+    if (p.scal[tc.mi].flags & MUONH_FLAG_NONFINITE_INPUT) {
+      if (threadIdx.x == 0) {
+        p.part[2 * e] = 0.f;
+        p.part[2 * e + 1] = 0.f;
+      }
+      continue;
+    }
+    __syncthreads();
+    load_o_tile(p, md, tc, tile);
+    __syncthreads();
+    float oo = 0.f, wo = 0.f;
+#pragma unroll
+    for (int j = 0; j < kEwTile / kTy; ++j) {
+      const int r = ty + kTy * j;
+      const float4 w = load4(md.w, md, tc.r0 + r, tc.c0 + tx * 4);
+      const float* o = &tile[r][tx * 4];
+      oo = fmaf(o[0], o[0], oo);
+      oo = fmaf(o[1], o[1], oo);
+      oo = fmaf(o[2], o[2], oo);
+      oo = fmaf(o[3], o[3], oo);
+      wo = fmaf(w.x, o[0], wo);
+      wo = fmaf(w.y, o[1], wo);
+      wo = fmaf(w.z, o[2], wo);
+      wo = fmaf(w.w, o[3], wo);
+    }
+    const float s_oo = block_sum(oo, red);
+    const float s_wo = block_sum(wo, red);
+    if (threadIdx.x == 0) {
+      p.part[2 * e] = s_oo;
+      p.part[2 * e + 1] = s_wo;
+    }
+  }
+}
+
+// W <- kw W + ko O (Eq. (1) with both normalisations folded into kw, ko).
+__global__ void __launch_bounds__(kEwThreads) project_kernel(const EwParams p) {
+  __shared__ float tile[kEwTile][kEwTile + 1];
+  __shared__ float red[kEwThreads / 32];
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+    const TileCoord tc = tile_coord(p, e);
+    const MatDev& md = p.mats[tc.mi];
+    const MatScal& sc = p.scal[tc.mi];
+    const int mode = sc.mode;
+    if (mode == 2) {
+      if (threadIdx.x == 0) p.part[e] = 0.f;
+      continue;
+    }
+    const float kw = sc.kw, ko = sc.ko;
+    if (mode == 0) {
+      __syncthreads();
+      load_o_tile(p, md, tc, tile);
+      __syncthreads();
+    }
+    constexpr int J = kEwTile / kTy;
+    float4 wv[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) wv[j] = load4(md.w, md, tc.r0 + ty + kTy * j, tc.c0 + tx * 4);
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int r = ty + kTy * j;
+      const int64_t row = tc.r0 + r, col = tc.c0 + tx * 4;
+      float4 w = wv[j];
+      if (mode == 0) {
+        const float* o = &tile[r][tx * 4];
+        w.x = fmaf(ko, o[0], kw * w.x);
+        w.y = fmaf(ko, o[1], kw * w.y);
+        w.z = fmaf(ko, o[2], kw * w.z);
+        w.w = fmaf(ko, o[3], kw * w.w);
+      } else {
+        w.x *= kw;
+        w.y *= kw;
+        w.z *= kw;
+        w.w *= kw;
+      }
+      store4(md.w, md, row, col, w);
+      acc = fmaf(w.x, w.x, acc);
+      acc = fmaf(w.y, w.y, acc);
+      acc = fmaf(w.z, w.z, acc);
+      acc = fmaf(w.w, w.w, acc);
+    }
+    const float s = block_sum(acc, red);
+    if (threadIdx.x == 0) p.part[e] = s;
+  }
+}
+
+// dst (rows x cols, fp32, row stride ld) = O of one matrix, unscaled.
+__global__ void __launch_bounds__(kEwThreads) export_update_kernel(const EwParams p, int mi, float* dst,
+                                                                   int64_t ld) {
+  __shared__ float tile[kEwTile][kEwTile + 1];
+  const MatDev& md = p.mats[mi];
+  const float unscale = exp2f(static_cast<float>(-md.ex));
+  const int64_t n_tiles = static_cast<int64_t>(md.et_rows) * md.et_cols;
+  for (int64_t local = blockIdx.x; local < n_tiles; local += gridDim.x) {
+    const int64_t e = md.et_begin + local;
+    const TileCoord tc = tile_coord(p, e);
+    __syncthreads();
+    load_o_tile(p, md, tc, tile);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kEwTile * kEwTile; i += kEwThreads) {
+      const int r = i / kEwTile, c = i % kEwTile;
+      const int64_t row = tc.r0 + r, col = tc.c0 + c;
+      if (row < md.rows && col < md.cols) dst[row * ld + col] = tile[r][c] * unscale;
+    }
+  }
+}
+
+// ------------------------------------------------------ finalize kernels
+template <typename T>
+__device__ double matrix_sum(const T* part, int64_t begin, int64_t count, int stride, int comp, double* red) {
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < count; i += kEwThreads) s += static_cast<double>(part[(begin + i) * stride + comp]);
+  return block_sum(s, red);
+}
+
+__global__ void __launch_bounds__(kEwThreads) finalize_init_kernel(const EwParams p) {
+  __shared__ double red[kEwThreads / 32];
+  const int mi = blockIdx.x;
+  const MatDev& md = p.mats[mi];
+  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
+  const double s = matrix_sum(p.part64, md.et_begin, cnt, 1, 0, red);
+  if (threadIdx.x == 0) {
+    MatScal& sc = p.scal[mi];
+    sc.wnorm2 = s;
+    if (!(sc.R > 0.f)) sc.R = static_cast<float>(sqrt(s));
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwParams p) {
+  __shared__ double red[kEwThreads / 32];
+  const int mi = blockIdx.x;
+  const MatDev& md = p.mats[mi];
+  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
+  const double s = matrix_sum(p.part, md.et_begin, cnt, 1, 0, red);
+  if (threadIdx.x == 0) {
+    MatScal& sc = p.scal[mi];
+    sc.flags = 0u;
+    sc.mode = 0;
+    const double xn = sqrt(s);
+    sc.stats.input_norm = static_cast<float>(xn);
+    if (!isfinite(s)) {
+      sc.flags |= MUONH_FLAG_NONFINITE_INPUT;
+      sc.xscale = 0.f;
+    } else if (s == 0.0) {
+      sc.flags |= MUONH_FLAG_ZERO_UPDATE;
+      sc.xscale = 0.f;
+    } else {
+      sc.xscale = static_cast<float>(ldexp(1.0, md.ex) / (xn + static_cast<double>(p.eps)));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads) finalize_update_kernel(const EwParams p) {
+  __shared__ double red[kEwThreads / 32];
+  const int mi = blockIdx.x;
+  const MatDev& md = p.mats[mi];
+  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
+  const double soo = matrix_sum(p.part, md.et_begin, cnt, 2, 0, red);
+  const double swo = matrix_sum(p.part, md.et_begin, cnt, 2, 1, red);
+  if (threadIdx.x == 0) {
+    MatScal& sc = p.scal[mi];
+    const double unscale = ldexp(1.0, -md.ex);
+    const double oo = soo * unscale * unscale;
+    const double wo = swo * unscale;
+    const double on = sqrt(oo);
+    const double wn2 = sc.wnorm2;
+    const double wn = sqrt(wn2);
+    const double R = sc.R;
+    const double lr = p.step[mi].lr;
+    sc.kw = 1.f;
+    sc.ko = 0.f;
+    double elr = 0.0;
+    if (sc.flags & MUONH_FLAG_NONFINITE_INPUT) {
+      sc.mode = 2;
+    } else if (!isfinite(oo) || !isfinite(wo)) {
+      sc.flags |= MUONH_FLAG_NONFINITE_UPDATE;
+      sc.mode = 2;
+    } else if (oo == 0.0) {
+      sc.flags |= MUONH_FLAG_ZERO_UPDATE;
+      if (wn > 0.0) {
+        sc.mode = 1;
+        sc.kw = static_cast<float>(R / wn);
+      } else {
+        sc.flags |= MUONH_FLAG_DEGENERATE;
+        sc.mode = 2;
+      }
+    } else {
+      const double alpha = lr * R / on;
+      const double wt2 = wn2 - 2.0 * alpha * wo + alpha * alpha * oo;
+      if (!(wt2 > 0.0)) {
+        sc.flags |= MUONH_FLAG_DEGENERATE;
+        sc.mode = 2;
+      } else {
+        const double kw = R / sqrt(wt2);
+        sc.mode = 0;
+        sc.kw = static_cast<float>(kw);
+        sc.ko = static_cast<float>(-kw * alpha * unscale);
+        elr = alpha * on / wn;
+      }
+    }
+    sc.stats.elr = static_cast<float>(elr);
+    sc.stats.pre_norm = static_cast<float>(wn);
+    sc.stats.update_norm = (sc.flags & MUONH_FLAG_NONFINITE_INPUT) ? 0.f : static_cast<float>(on);
+  }
+}
+
+__global__ void __launch_bounds__(kEwThreads) finalize_step_kernel(const EwParams p) {
+  __shared__ double red[kEwThreads / 32];
+  const int mi = blockIdx.x;
+  const MatDev& md = p.mats[mi];
+  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
+  const double s = matrix_sum(p.part, md.et_begin, cnt, 1, 0, red);
+  if (threadIdx.x == 0) {
+    MatScal& sc = p.scal[mi];
+    if (sc.mode != 2) sc.wnorm2 = s;
+    sc.stats.post_norm = static_cast<float>(sqrt(sc.wnorm2));
+    if (*reinterpret_cast<const volatile int*>(p.err) != 0) sc.flags |= MUONH_FLAG_TIMEOUT;
+    sc.stats.flags = sc.flags;
+    if (p.stats_out) p.stats_out[mi] = sc.stats;
+  }
+}
+
+inline int ew_grid(int64_t n_et, int grid) {
+  return static_cast<int>(n_et < grid ? (n_et > 0 ? n_et : 1) : grid);
+}
+
+}  // namespace
+
+cudaError_t launch_init_norm(const EwParams& p, int grid, cudaStream_t s) {
+  init_norm_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_finalize_init(const EwParams& p, cudaStream_t s) {
+  finalize_init_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_momentum_norm(const EwParams& p, int grid, cudaStream_t s) {
+  momentum_norm_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_finalize_input(const EwParams& p, cudaStream_t s) {
+  finalize_input_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_write_x(const EwParams& p, int grid, cudaStream_t s) {
+  write_x_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_update_dots(const EwParams& p, int grid, cudaStream_t s) {
+  update_dots_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_finalize_update(const EwParams& p, cudaStream_t s) {
+  finalize_update_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_project(const EwParams& p, int grid, cudaStream_t s) {
+  project_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_finalize_step(const EwParams& p, cudaStream_t s) {
+  finalize_step_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_export_update(const EwParams& p, int mat, float* dst, int64_t ld, cudaStream_t s) {
+  export_update_kernel<<<256, kEwThreads, 0, s>>>(p, mat, dst, ld);
+  return cudaGetLastError();
+}
+
+}  // namespace muonh

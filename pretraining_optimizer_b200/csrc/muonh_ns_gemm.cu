@@ -1,0 +1,389 @@
+// Grouped Newton-Schulz GEMMs on the 5th-generation tensor cores (sm_100a).
+//
+// One Newton-Schulz iteration on a wide matrix Y (r x c) is three products
+// (quintic iteration of the Muon update; the MuonH wrapper of the Puro-2B
+// report, Sec. 3.3, normalises its output):
+//   GRAM    A  = Y Y^T                 M = r, N = r, K = c   (symmetric)
+//   SQUARE  B  = b A + c A A           M = r, N = r, K = r   (symmetric)
+//   APPLY   Y' = a Y + B Y             M = r, N = c, K = r
+// Every launch covers the tiles of all matrices of the step (grouped), in a
+// persistent grid of one CTA per SM.  Symmetric products compute only the
+// 128 x 256 tiles that touch the upper triangle and write each element of
+// the upper triangle once directly and once mirrored.
+//
+// Per CTA: warp 0 issues TMA loads into a ring of shared-memory stages,
+// warp 1 (one thread) issues tcgen05.mma into one of two TMEM accumulators
+// (128 lanes x 256 fp32 columns each), warps 2-5 drain the other
+// accumulator with tcgen05.ld, apply the polynomial epilogue and store.
+// Every wait is bounded (muonh::mbar_wait) and records a timeout in *err.
+//
+// Storage: fp16 operands hold the value times 2^e (e per matrix and per
+// operand, chosen on the host so that no entry can overflow); products of
+// scaled operands are rescaled exactly in the fp32 epilogue.  In FP32 mode
+// each operand is a pair (hi, lo) of fp16 arrays, value = hi + lo, and each
+// tile accumulates hi*hi + hi*lo + lo*hi.
+#include "muonh_common.cuh"
+
+namespace muonh {
+namespace {
+
+template <int PREC>
+struct Store16;
+template <>
+struct Store16<P_FP16> {
+  using T = __half;
+  static __device__ __forceinline__ T cvt(float v) { return __float2half_rn(v); }
+  static __device__ __forceinline__ float back(T v) { return __half2float(v); }
+};
+template <>
+struct Store16<P_BF16> {
+  using T = __nv_bfloat16;
+  static __device__ __forceinline__ T cvt(float v) { return __float2bfloat16_rn(v); }
+  static __device__ __forceinline__ float back(T v) { return __bfloat162float(v); }
+};
+template <>
+struct Store16<P_FP32> : Store16<P_FP16> {};
+
+template <int PREC>
+struct Cfg {
+  static constexpr int kParts = (PREC == P_FP32) ? 2 : 1;
+  static constexpr int kStages = (PREC == P_FP32) ? 2 : 4;
+  static constexpr int kABytes = kBM * kBK * 2;                    // 16 KB
+  static constexpr int kBBytes = kBN * kBK * 2;                    // 32 KB
+  static constexpr int kStageBytes = kParts * (kABytes + kBBytes);
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kSmem = kBarOffset + 256 + 1024;            // + barriers + alignment slack
+};
+
+// 32 consecutive values of one row, stored as 16-bit (and the fp16 residual in FP32 mode).
+template <int PREC>
+__device__ __forceinline__ void store_row32(void* hi_base, void* lo_base, int64_t off, const float (&v)[32]) {
+  using S = Store16<PREC>;
+  using T = typename S::T;
+  uint4 hbuf[4], lbuf[4];
+  T* h = reinterpret_cast<T*>(hbuf);
+  __half* l = reinterpret_cast<__half*>(lbuf);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    T hv = S::cvt(v[j]);
+    h[j] = hv;
+    if (PREC == P_FP32) l[j] = __float2half_rn(v[j] - S::back(hv));
+  }
+  uint4* dh = reinterpret_cast<uint4*>(reinterpret_cast<T*>(hi_base) + off);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) dh[q] = hbuf[q];
+  if (PREC == P_FP32) {
+    uint4* dl = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(lo_base) + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dl[q] = lbuf[q];
+  }
+}
+
+template <int PREC>
+__device__ __forceinline__ void store_one(void* hi_base, void* lo_base, int64_t off, float v) {
+  using S = Store16<PREC>;
+  using T = typename S::T;
+  T hv = S::cvt(v);
+  reinterpret_cast<T*>(hi_base)[off] = hv;
+  if (PREC == P_FP32) reinterpret_cast<__half*>(lo_base)[off] = __float2half_rn(v - S::back(hv));
+}
+
+template <int PREC>
+__device__ __forceinline__ void load_row32(const void* hi_base, const void* lo_base, int64_t off, float (&v)[32]) {
+  using S = Store16<PREC>;
+  using T = typename S::T;
+  uint4 hbuf[4], lbuf[4];
+  const uint4* sh = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(hi_base) + off);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) hbuf[q] = sh[q];
+  const T* h = reinterpret_cast<const T*>(hbuf);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = S::back(h[j]);
+  if (PREC == P_FP32) {
+    const uint4* sl = reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(lo_base) + off);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) lbuf[q] = sl[q];
+    const __half* l = reinterpret_cast<const __half*>(lbuf);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] += __half2float(l[j]);
+  }
+}
+
+// Symmetric output: element (row, col) of the upper triangle (col >= row)
+// is stored at [row][col]; for col > row also at [col][row].
+template <int PREC>
+__device__ __forceinline__ void store_symmetric(void* hi, void* lo, int ld, int row, int col0,
+                                                const float (&v)[32]) {
+  const int64_t roff = static_cast<int64_t>(row) * ld;
+  if (col0 >= row) {
+    store_row32<PREC>(hi, lo, roff + col0, v);
+  } else if (col0 + 31 >= row) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j >= row) store_one<PREC>(hi, lo, roff + col0 + j, v[j]);
+  }
+  if (col0 + 31 > row) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j > row) store_one<PREC>(hi, lo, static_cast<int64_t>(col0 + j) * ld + row, v[j]);
+  }
+}
+
+template <int MODE, int PREC>
+__global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_constant__ NsParams p) {
+  using C = Cfg<PREC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_parity[C::kStages];
+      bool issued[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) issued[s] = false;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
+        const TileDesc td = p.tiles[t];
+        const MatDev& md = p.mats[td.mat];
+        const ClassDev& cd = p.classes[md.cls];
+        const int z = md.z;
+        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) { ok = false; break; }
+          mbar_expect_tx(&full[stage], C::kStageBytes);
+          uint8_t* sa = smem + stage * C::kStageBytes;
+          uint8_t* sb = sa + C::kParts * C::kABytes;
+          const int k0 = kb * kBK;
+          for (int part = 0; part < C::kParts; ++part) {
+            uint8_t* a_dst = sa + part * C::kABytes;
+            uint8_t* b_dst = sb + part * C::kBBytes;
+            if (MODE == M_GRAM) {
+              tma_load_3d(a_dst, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, part), &full[stage], k0,
+                          td.bi * kBM, z);
+              tma_load_3d(b_dst, p.tmaps + tm_x(cd.tm_base + TM_X_K256, p.src, part), &full[stage], k0,
+                          td.bj * kBN, z);
+            } else if (MODE == M_SQUARE) {
+              tma_load_3d(a_dst, p.tmaps + cd.tm_base + TM_A_K128 + part, &full[stage], k0, td.bi * kBM, z);
+              tma_load_3d(b_dst, p.tmaps + cd.tm_base + TM_A_K256 + part, &full[stage], k0, td.bj * kBN, z);
+            } else {
+              tma_load_3d(a_dst, p.tmaps + cd.tm_base + TM_B_K128 + part, &full[stage], k0, td.bi * kBM, z);
+              const CUtensorMap* xm = p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, part);
+#pragma unroll
+              for (int q = 0; q < kBN / 64; ++q)
+                tma_load_3d(b_dst + q * (64 * kBK * 2), xm, &full[stage], td.bj * kBN + q * 64, k0, z);
+            }
+          }
+          issued[stage] = true;
+          issued_parity[stage] = phase;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // let the copies already in flight land before the CTA exits
+        for (int s = 0; s < C::kStages; ++s)
+          if (issued[s]) {
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&full[s], issued_parity[s]) && globaltimer() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, PREC == P_BF16 ? 1 : 0, MODE == M_APPLY ? 1 : 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++local) {
+        const TileDesc td = p.tiles[t];
+        const MatDev& md = p.mats[td.mat];
+        const ClassDev& cd = p.classes[md.cls];
+        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kBN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kParts * C::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+#pragma unroll
+            for (int prod = 0; prod < (C::kParts == 2 ? 3 : 1); ++prod) {
+              // products: hi*hi, hi*lo, lo*hi
+              const int pa = (prod == 2) ? 1 : 0;
+              const int pb = (prod == 1) ? 1 : 0;
+              const uint64_t adesc = sdesc_sw128(sa + pa * C::kABytes + k * 32, 16, 1024);
+              uint64_t bdesc;
+              if (MODE == M_APPLY)
+                bdesc = sdesc_sw128(sb + pb * C::kBBytes + k * 16 * 128, 64 * kBK * 2, 1024);
+              else
+                bdesc = sdesc_sw128(sb + pb * C::kBBytes + k * 32, 16, 1024);
+              umma_f16(d_tmem, adesc, bdesc, kIdesc, (kb | k | prod) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+      // make sure no MMA is still writing TMEM when the CTA deallocates it
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int lrow = quarter * 32 + lane;    // row within the tile
+    int local = 0;
+    for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++local) {
+      const TileDesc td = p.tiles[t];
+      const MatDev& md = p.mats[td.mat];
+      const ClassDev& cd = p.classes[md.cls];
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
+      tc_fence_after();
+      const int row = td.bi * kBM + lrow;
+      // tcgen05.ld is warp-collective: chunk skips below depend on the warp's
+      // first row only, so a warp never splits around it.
+      const int warp_row0 = row - lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
+      if (MODE == M_GRAM) {
+        const float sc = exp2f(static_cast<float>(md.ea - 2 * md.ex));
+        void* hi = static_cast<uint8_t*>(cd.a[0]) + md.z * cd.a_stride * 2;
+        void* lo = cd.a[1] ? static_cast<uint8_t*>(cd.a[1]) + md.z * cd.a_stride * 2 : nullptr;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int col0 = td.bj * kBN + ch * 32;
+          if (col0 + 31 < warp_row0) continue;   // whole chunk below the diagonal for this warp
+          float v[32];
+          tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= sc;
+          store_symmetric<PREC>(hi, lo, cd.r_pad, row, col0, v);
+        }
+      } else if (MODE == M_SQUARE) {
+        const float kb_ = md.b * exp2f(static_cast<float>(md.eb - md.ea));
+        const float kc_ = md.c_coef * exp2f(static_cast<float>(md.eb - 2 * md.ea));
+        const void* ahi = static_cast<const uint8_t*>(cd.a[0]) + md.z * cd.a_stride * 2;
+        const void* alo = cd.a[1] ? static_cast<const uint8_t*>(cd.a[1]) + md.z * cd.a_stride * 2 : nullptr;
+        void* bhi = static_cast<uint8_t*>(cd.b[0]) + md.z * cd.a_stride * 2;
+        void* blo = cd.b[1] ? static_cast<uint8_t*>(cd.b[1]) + md.z * cd.a_stride * 2 : nullptr;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int col0 = td.bj * kBN + ch * 32;
+          if (col0 + 31 < warp_row0) continue;   // whole chunk below the diagonal for this warp
+          float v[32], a[32];
+          tmem_ld32(taddr + ch * 32, v);
+          load_row32<PREC>(ahi, alo, static_cast<int64_t>(row) * cd.r_pad + col0, a);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = fmaf(kc_, v[j], kb_ * a[j]);
+          store_symmetric<PREC>(bhi, blo, cd.r_pad, row, col0, v);
+        }
+      } else {
+        const float ks = exp2f(static_cast<float>(-md.eb));
+        const float ca = md.a;
+        const int64_t xo = md.z * cd.x_stride * 2;
+        const void* xhi = static_cast<const uint8_t*>(cd.x[p.src][0]) + xo;
+        const void* xlo = cd.x[p.src][1] ? static_cast<const uint8_t*>(cd.x[p.src][1]) + xo : nullptr;
+        void* yhi = static_cast<uint8_t*>(cd.x[p.src ^ 1][0]) + xo;
+        void* ylo = cd.x[p.src ^ 1][1] ? static_cast<uint8_t*>(cd.x[p.src ^ 1][1]) + xo : nullptr;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int col0 = td.bj * kBN + ch * 32;
+          const int64_t off = static_cast<int64_t>(row) * cd.c_pad + col0;
+          float v[32], x[32];
+          tmem_ld32(taddr + ch * 32, v);
+          load_row32<PREC>(xhi, xlo, off, x);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = fmaf(ks, v[j], ca * x[j]);
+          store_row32<PREC>(yhi, ylo, off, v);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+}  // namespace
+
+template <int MODE, int PREC>
+static cudaError_t set_attr() {
+  return cudaFuncSetAttribute(ns_gemm_kernel<MODE, PREC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<PREC>::kSmem);
+}
+
+cudaError_t ns_gemm_set_attributes() {
+  cudaError_t e;
+#define MUONH_SET(MD, PR) \
+  if ((e = set_attr<MD, PR>()) != cudaSuccess) return e;
+  MUONH_SET(M_GRAM, P_FP16) MUONH_SET(M_SQUARE, P_FP16) MUONH_SET(M_APPLY, P_FP16)
+  MUONH_SET(M_GRAM, P_BF16) MUONH_SET(M_SQUARE, P_BF16) MUONH_SET(M_APPLY, P_BF16)
+  MUONH_SET(M_GRAM, P_FP32) MUONH_SET(M_SQUARE, P_FP32) MUONH_SET(M_APPLY, P_FP32)
+#undef MUONH_SET
+  return cudaSuccess;
+}
+
+size_t ns_gemm_smem_bytes(int prec) {
+  return prec == P_FP32 ? Cfg<P_FP32>::kSmem : Cfg<P_FP16>::kSmem;
+}
+
+cudaError_t launch_ns_gemm(int mode, int prec, const NsParams& p, int grid, cudaStream_t s) {
+  if (p.ntiles <= 0) return cudaSuccess;
+  const size_t smem = ns_gemm_smem_bytes(prec);
+#define MUONH_LAUNCH(MD, PR)                                                   \
+  if (mode == MD && prec == PR) {                                              \
+    ns_gemm_kernel<MD, PR><<<grid, kGemmThreads, smem, s>>>(p);                \
+    return cudaGetLastError();                                                 \
+  }
+  MUONH_LAUNCH(M_GRAM, P_FP16) MUONH_LAUNCH(M_SQUARE, P_FP16) MUONH_LAUNCH(M_APPLY, P_FP16)
+  MUONH_LAUNCH(M_GRAM, P_BF16) MUONH_LAUNCH(M_SQUARE, P_BF16) MUONH_LAUNCH(M_APPLY, P_BF16)
+  MUONH_LAUNCH(M_GRAM, P_FP32) MUONH_LAUNCH(M_SQUARE, P_FP32) MUONH_LAUNCH(M_APPLY, P_FP32)
+#undef MUONH_LAUNCH
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace muonh

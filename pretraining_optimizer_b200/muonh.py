@@ -1,0 +1,226 @@
+"""ctypes binding of libmuonh.so: argument marshalling only.
+
+Every step of the optimizer runs in the library's CUDA kernels; PyTorch is
+used for device memory (the caller's weight, momentum and gradient tensors)
+and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, Structure, c_char_p, c_float, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+
+QUINTIC = (3.4445, -4.7750, 2.0315)
+NS_FP16, NS_BF16, NS_FP32 = 0, 1, 2
+_PREC = {"fp16": NS_FP16, "bf16": NS_BF16, "fp32": NS_FP32}
+FLAG_NONFINITE_INPUT = 1
+FLAG_ZERO_UPDATE = 2
+FLAG_NONFINITE_UPDATE = 4
+FLAG_DEGENERATE = 8
+FLAG_TIMEOUT = 16
+
+EXPORTED_SYMBOLS = (
+    "muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
+    "muonh_export_state", "muonh_import_state", "muonh_device_status", "muonh_last_launch_count",
+    "muonh_destroy", "muonh_status_string", "muonh_last_error",
+)
+
+
+class MatrixDesc(Structure):
+    _fields_ = [("w", c_void_p), ("m", c_void_p), ("rows", c_int64), ("cols", c_int64),
+                ("ld", c_int64), ("radius", c_float), ("beta", c_float), ("nesterov", c_int32),
+                ("ns_steps", c_int32), ("ns_a", c_float), ("ns_b", c_float), ("ns_c", c_float)]
+
+
+class Config(Structure):
+    _fields_ = [("ns_precision", c_int32), ("eps", c_float)]
+
+
+class Stats(Structure):
+    _fields_ = [("elr", c_float), ("pre_norm", c_float), ("post_norm", c_float),
+                ("update_norm", c_float), ("input_norm", c_float), ("flags", c_uint32)]
+
+
+class MuonHError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"muonh status {status}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuonh.so")
+
+
+_LIB = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libmuonh.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m pretraining_optimizer_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.muonh_init.argtypes = [POINTER(c_void_p), POINTER(MatrixDesc), c_int32, POINTER(Config), c_void_p]
+    lib.muonh_step.argtypes = [c_void_p, POINTER(c_float), POINTER(c_void_p), c_void_p, c_void_p]
+    lib.muonh_get_stats.argtypes = [c_void_p, POINTER(Stats)]
+    lib.muonh_get_update.argtypes = [c_void_p, c_int32, c_void_p, c_int64, c_void_p]
+    lib.muonh_get_radius.argtypes = [c_void_p, POINTER(c_float)]
+    lib.muonh_export_state.argtypes = [c_void_p, c_void_p, POINTER(c_size_t)]
+    lib.muonh_import_state.argtypes = [c_void_p, c_void_p, c_size_t]
+    lib.muonh_device_status.argtypes = [c_void_p]
+    lib.muonh_last_launch_count.argtypes = [c_void_p]
+    lib.muonh_last_launch_count.restype = c_int32
+    lib.muonh_destroy.argtypes = [c_void_p]
+    lib.muonh_destroy.restype = None
+    lib.muonh_status_string.argtypes = [c_int32]
+    lib.muonh_status_string.restype = c_char_p
+    lib.muonh_last_error.argtypes = []
+    lib.muonh_last_error.restype = c_char_p
+    for name in ("muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
+                 "muonh_export_state", "muonh_import_state", "muonh_device_status"):
+        getattr(lib, name).restype = c_int32
+    _LIB = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        lib = library()
+        msg = lib.muonh_last_error().decode() or lib.muonh_status_string(status).decode()
+        raise MuonHError(status, msg)
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _matrix_view(t, what: str):
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_cuda or t.dim() != 2:
+        raise TypeError(f"{what} must be a 2-D fp32 CUDA tensor")
+    if t.stride(1) != 1:
+        raise ValueError(f"{what} must have unit column stride")
+    return t.data_ptr(), t.shape[0], t.shape[1], max(t.stride(0), t.shape[1])
+
+
+class MuonH:
+    """MuonH over a list of fp32 CUDA weight matrices (updated in place).
+
+    lr passed to step() is the effective LR eta^H of each matrix
+    (the caller applies the hyperball multiplier and the schedule)."""
+
+    def __init__(self, weights, momenta=None, *, beta=0.95, nesterov=True, ns_steps=5,
+                 ns_coeffs=QUINTIC, eps=1e-7, ns_precision="fp16", radii=None, stream=None):
+        import torch
+        self._lib = library()
+        self.weights = list(weights)
+        n = len(self.weights)
+        if momenta is None:
+            momenta = [torch.zeros_like(w) for w in self.weights]
+        self.momenta = list(momenta)
+        if len(self.momenta) != n:
+            raise ValueError("one momentum tensor per weight")
+        prec = _PREC[ns_precision] if isinstance(ns_precision, str) else int(ns_precision)
+        descs = (MatrixDesc * n)()
+        self.shapes = []
+        for i, (w, m) in enumerate(zip(self.weights, self.momenta)):
+            wp, rows, cols, ld = _matrix_view(w, f"weights[{i}]")
+            mp, mr, mc, mld = _matrix_view(m, f"momenta[{i}]")
+            if (mr, mc, mld) != (rows, cols, ld):
+                raise ValueError(f"momenta[{i}] must match weights[{i}] in shape and stride")
+            R = 0.0 if radii is None else float(radii[i])
+            a, b, c = ns_coeffs if not isinstance(ns_coeffs[0], (tuple, list)) else ns_coeffs[i]
+            steps = ns_steps if isinstance(ns_steps, int) else ns_steps[i]
+            bt = beta if isinstance(beta, (int, float)) else beta[i]
+            descs[i] = MatrixDesc(wp, mp, rows, cols, ld, R, bt, int(bool(nesterov)), steps, a, b, c)
+            self.shapes.append((rows, cols, ld))
+        cfg = Config(prec, eps)
+        ctx = c_void_p()
+        _check(self._lib.muonh_init(ctypes.byref(ctx), descs, n, ctypes.byref(cfg), _stream_handle(stream)))
+        self._ctx = ctx
+        self.n = n
+        self._lr = (c_float * n)()
+        self._g = (c_void_p * n)()
+
+    # ---------------------------------------------------------------- step
+    def step(self, grads, lr, stats=None, stream=None) -> None:
+        """grads: list of fp32 CUDA tensors shaped like the weights; lr: float or
+        per-matrix sequence; stats: None or a CUDA tensor of >= 24*n bytes."""
+        n = self.n
+        if len(grads) != n:
+            raise ValueError("one gradient per weight")
+        if isinstance(lr, (int, float)):
+            for i in range(n):
+                self._lr[i] = lr
+        else:
+            for i in range(n):
+                self._lr[i] = lr[i]
+        for i, g in enumerate(grads):
+            gp, r, c, ld = _matrix_view(g, f"grads[{i}]")
+            if (r, c, ld) != self.shapes[i]:
+                raise ValueError(f"grads[{i}] must match weights[{i}] in shape and stride")
+            self._g[i] = gp
+        sp = None
+        if stats is not None:
+            if not stats.is_cuda or stats.numel() * stats.element_size() < 24 * n:
+                raise ValueError("stats must be a CUDA tensor of at least 24*n bytes")
+            sp = stats.data_ptr()
+        _check(self._lib.muonh_step(self._ctx, self._lr, self._g, sp, _stream_handle(stream)))
+
+    def step_raw(self, grad_ptrs, lr_values, stats_ptr=None, stream_handle=0) -> None:
+        """Lowest-overhead step: pointers and values already marshalled."""
+        _check(self._lib.muonh_step(self._ctx, lr_values, grad_ptrs, stats_ptr, stream_handle))
+
+    # ---------------------------------------------------------- inspection
+    def stats(self) -> list[dict]:
+        out = (Stats * self.n)()
+        _check(self._lib.muonh_get_stats(self._ctx, out))
+        return [dict(elr=s.elr, pre_norm=s.pre_norm, post_norm=s.post_norm, update_norm=s.update_norm,
+                     input_norm=s.input_norm, flags=s.flags) for s in out]
+
+    def update(self, i: int, stream=None):
+        """Matrix i's Newton-Schulz output O of the last step (fp32, W's shape)."""
+        import torch
+        rows, cols, _ = self.shapes[i]
+        dst = torch.empty((rows, cols), dtype=torch.float32, device=self.weights[i].device)
+        _check(self._lib.muonh_get_update(self._ctx, i, dst.data_ptr(), cols, _stream_handle(stream)))
+        return dst
+
+    def radii(self) -> list[float]:
+        out = (c_float * self.n)()
+        _check(self._lib.muonh_get_radius(self._ctx, out))
+        return list(out)
+
+    def last_launch_count(self) -> int:
+        return int(self._lib.muonh_last_launch_count(self._ctx))
+
+    def device_status(self) -> None:
+        _check(self._lib.muonh_device_status(self._ctx))
+
+    def export_state(self) -> bytes:
+        size = c_size_t(0)
+        _check(self._lib.muonh_export_state(self._ctx, None, ctypes.byref(size)))
+        buf = ctypes.create_string_buffer(size.value)
+        _check(self._lib.muonh_export_state(self._ctx, buf, ctypes.byref(size)))
+        return buf.raw[: size.value]
+
+    def import_state(self, blob: bytes) -> None:
+        buf = ctypes.create_string_buffer(blob, len(blob))
+        _check(self._lib.muonh_import_state(self._ctx, buf, len(blob)))
+
+    def close(self) -> None:
+        if getattr(self, "_ctx", None):
+            self._lib.muonh_destroy(self._ctx)
+            self._ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

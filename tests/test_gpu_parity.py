@@ -1,0 +1,161 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs (B200 only)."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity_helpers import (FP16_NS_TOL, FP32_NS_TOL, NORM_TOL, W_TOL_10, rel_fro, run_gpu,
+                            run_oracle)
+
+pytestmark = pytest.mark.gpu
+
+
+def _single():
+    wl = synth.workload("single_256x512")
+    W0 = [wl.weight(0)]
+    return wl, W0
+
+
+@pytest.mark.parametrize("prec,ns_tol,w_tol", [("fp16", FP16_NS_TOL, W_TOL_10),
+                                               ("fp32", FP32_NS_TOL, 1e-5)])
+def test_single_matrix_ten_steps(prec, ns_tol, w_tol):
+    """256 x 512, 10 steps, lr 0.01, beta 0.95 Nesterov, tuned quintic x 5."""
+    wl, W0 = _single()
+    keep = (0, 4, 9)
+    g = run_gpu(W0, wl.grad, wl.lrs, prec=prec, keep_updates=keep)
+    o = run_oracle(W0, wl.grad, wl.lrs, keep_updates=keep)
+    R = o["R"][0]
+    assert abs(g["R"][0] - R) <= NORM_TOL * R
+    for t in keep:
+        assert rel_fro(g["O"][t][0], o["O"][t][0]) <= ns_tol, (t, rel_fro(g["O"][t][0], o["O"][t][0]))
+        # element by element: no entry off by more than a few times the typical error
+        err = np.abs(g["O"][t][0] - o["O"][t][0]).max()
+        assert err <= 10 * ns_tol * np.abs(o["O"][t][0]).max(), (t, err)
+    for t in range(len(wl.lrs)):
+        gs, os_ = g["stats"][t][0], o["stats"][t][0]
+        assert gs["flags"] == 0
+        assert abs(gs["elr"] - os_["elr"]) <= NORM_TOL * os_["elr"]
+        assert abs(gs["post_norm"] - R) <= NORM_TOL * R
+        assert abs(gs["pre_norm"] - os_["pre_norm"]) <= NORM_TOL * R
+        assert abs(gs["input_norm"] - os_["input_norm"]) <= NORM_TOL * os_["input_norm"]
+        assert abs(gs["update_norm"] - os_["update_norm"]) <= ns_tol * os_["update_norm"]
+    assert np.linalg.norm(g["W"][0] - o["W"][0]) / R <= w_tol
+    assert rel_fro(g["M"][0], o["M"][0]) <= 1e-6
+
+
+def test_single_matrix_bf16_operands():
+    """bf16 operand storage: measured ~1% NS error on this case (see design notes), 3e-2 bound."""
+    wl, W0 = _single()
+    g = run_gpu(W0, wl.grad, wl.lrs[:3], prec="bf16", keep_updates=(0, 2))
+    o = run_oracle(W0, wl.grad, wl.lrs[:3], keep_updates=(0, 2))
+    for t in (0, 2):
+        assert rel_fro(g["O"][t][0], o["O"][t][0]) <= 3e-2
+    assert abs(g["stats"][2][0]["post_norm"] - o["R"][0]) <= NORM_TOL * o["R"][0]
+
+
+@pytest.mark.parametrize("coeffs,tol", [((1.0, 0.0, 0.0), 2e-3),    # O = X0: K1 path only
+                                        ((0.0, 1.0, 0.0), 4e-3),    # O = (X X^T) X: GRAM + APPLY
+                                        ((0.0, 0.0, 1.0), 6e-3),    # O = (X X^T)^2 X: SQUARE
+                                        ((3.4445, -4.7750, 2.0315), 5e-3)])
+@pytest.mark.parametrize("shape", [(256, 512), (512, 256), (384, 1000), (1000, 300)])
+def test_one_iteration_isolates_each_gemm(coeffs, tol, shape):
+    W0 = [synth.initial_weight(0, *shape)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shape)
+    g = run_gpu(W0, grad, [0.01], ns_steps=1, coeffs=coeffs, keep_updates=(0,))
+    o = run_oracle(W0, grad, [0.01], ns_steps=1, coeffs=coeffs, keep_updates=(0,))
+    assert rel_fro(g["O"][0][0], o["O"][0][0]) <= tol
+
+
+@pytest.mark.parametrize("prec", ["fp16", "fp32"])
+def test_mixed_shapes_grouped_in_one_context(prec):
+    """Several shape classes, tall and wide, ragged sizes, a strided view,
+    odd column counts (scalar path), a 1 x n and an n x 1 matrix."""
+    shapes = [(256, 512), (512, 256), (256, 512), (1000, 300), (130, 70), (1, 300), (300, 1),
+              (96, 301), (640, 384)]
+    strides = [None, None, 520, None, None, None, None, None, 400]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    lrs = [[0.01 + 0.001 * i for i in range(len(shapes))]] * 3
+    tol = FP16_NS_TOL if prec == "fp16" else FP32_NS_TOL
+    g = run_gpu(W0, grad, lrs, prec=prec, keep_updates=(2,), strides=strides)
+    o = run_oracle(W0, grad, lrs, keep_updates=(2,))
+    for i, s in enumerate(shapes):
+        assert rel_fro(g["O"][2][i], o["O"][2][i]) <= tol, (i, s, rel_fro(g["O"][2][i], o["O"][2][i]))
+        R = o["R"][i]
+        assert abs(g["stats"][2][i]["post_norm"] - R) <= NORM_TOL * R, (i, s)
+        assert abs(g["stats"][2][i]["elr"] - o["stats"][2][i]["elr"]) <= NORM_TOL * o["stats"][2][i]["elr"]
+        assert np.linalg.norm(g["W"][i] - o["W"][i]) / R <= (1e-3 if prec == "fp16" else 1e-5), (i, s)
+
+
+def test_edge_cases_zero_nan_and_zero_lr():
+    shapes = [(128, 256)] * 4
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+
+    def grad(t, i):
+        gr = synth.gaussian_gradient(t, i, *shapes[i])
+        if i == 0:
+            return np.zeros_like(gr)            # zero gradient, zero momentum
+        if i == 1:
+            gr[3, 7] = np.nan                   # non-finite gradient
+        return gr
+
+    lrs = [[0.01, 0.01, 0.0, 0.02]]
+    g = run_gpu(W0, grad, lrs, keep_updates=(0,))
+    o = run_oracle(W0, grad, lrs)
+    st = g["stats"][0]
+    assert st[0]["flags"] & oracle.FLAG_ZERO_UPDATE and st[0]["elr"] == 0.0
+    assert np.allclose(g["W"][0], W0[0], rtol=1e-6, atol=1e-7)
+    assert st[1]["flags"] & oracle.FLAG_NONFINITE_INPUT
+    assert np.array_equal(g["W"][1], W0[1])
+    assert st[2]["flags"] == 0 and st[2]["elr"] == 0.0
+    assert np.allclose(g["W"][2], o["W"][2], rtol=0, atol=1e-6)
+    assert st[3]["flags"] == 0 and abs(st[3]["elr"] - 0.02) <= NORM_TOL * 0.02
+
+
+def test_convergent_coefficients_reach_the_polar_factor():
+    """With (15/8, -10/8, 3/8) the iteration converges to U V^T (fp32 NS mode, 30 steps)."""
+    rng = np.random.default_rng(3)
+    U, _ = np.linalg.qr(rng.standard_normal((128, 128)))
+    V, _ = np.linalg.qr(rng.standard_normal((384, 128)))
+    G = ((U * np.geomspace(1.0, 0.05, 128)) @ V.T).astype(np.float32)
+    W0 = [synth.initial_weight(0, 128, 384)]
+    g = run_gpu(W0, lambda t, i: G, [0.01], prec="fp32", ns_steps=30,
+                coeffs=(15 / 8, -10 / 8, 3 / 8), keep_updates=(0,), beta=0.0)
+    polar = U @ V.T
+    assert rel_fro(g["O"][0][0], polar) <= 1e-5
+
+
+def test_bitwise_deterministic():
+    wl, W0 = _single()
+    a = run_gpu(W0, wl.grad, wl.lrs[:3], keep_updates=(2,))
+    b = run_gpu(W0, wl.grad, wl.lrs[:3], keep_updates=(2,))
+    assert np.array_equal(a["W"][0], b["W"][0]) and np.array_equal(a["O"][2][0], b["O"][2][0])
+
+
+def test_checkpoint_resume_is_bitwise():
+    """10 straight steps == 5 steps, export/import into a new context, 5 steps."""
+    import torch
+    from pretraining_optimizer_b200 import MuonH
+    wl, W0 = _single()
+    grads = [[torch.from_numpy(wl.grad(t, 0)).cuda()] for t in range(10)]
+    W = [torch.from_numpy(W0[0]).cuda()]
+    opt = MuonH(W)
+    for t in range(10):
+        opt.step(grads[t], wl.lrs[t])
+    straight = W[0].cpu().numpy()
+    opt.close()
+    W2 = [torch.from_numpy(W0[0]).cuda()]
+    M2 = [torch.zeros_like(W2[0])]
+    opt = MuonH(W2, M2)
+    for t in range(5):
+        opt.step(grads[t], wl.lrs[t])
+    blob = opt.export_state()
+    w_ck, m_ck = W2[0].clone(), M2[0].clone()
+    opt.close()
+    opt = MuonH([w_ck], [m_ck], radii=[1.0])       # radius replaced by the imported state
+    opt.import_state(blob)
+    for t in range(5, 10):
+        opt.step(grads[t], wl.lrs[t])
+    torch.cuda.synchronize()
+    assert np.array_equal(w_ck.cpu().numpy(), straight)
+    opt.close()
