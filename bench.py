@@ -1,0 +1,377 @@
+#!/usr/bin/env python
+"""MuonH optimizer-step benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen3_1.7b|qwen3_0.6b|single_256x512] [--ns-precision fp16|bf16|fp32]
+
+One step = one muonh_step over the whole matrix set (momentum, Newton-Schulz,
+hyperball projection of every matrix).  Inputs are synthetic (W0 ~ N(0,0.02^2),
+gradients ~ N(0,1e-3^2)), resident in HBM when the timed region starts, and
+far larger than L2 (the 1.7B set moves ~34 GB of algorithmic traffic per
+step), so no L2 flush is needed between steps.  With N > 1 (torchrun) every
+rank runs an independent replica of the workload (no data-path collective);
+the timed region is bracketed by barriers and the max over ranks is taken.
+
+Rank 0 prints one JSON line.  --impl reference times the CPU oracle instead
+(rank 0 only, no GPU work).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MuonH steps/s for Qwen3-1.7B matrix set on 1 B200; NS TFLOP/s & HBM GB/s vs peak"
+UNIT = "steps/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# bytes per element actually moved by each elementwise kernel of this design
+KERNEL_BYTES = {
+    "momentum_norm": 12,   # read G, M; write M
+    "write_x": 10,         # read G, M; write 16-bit X
+    "update_dots": 6,      # read W, 16-bit O
+    "project": 10,         # read W, O; write W
+}
+# algorithmic bytes per element of the whole step (read G, M, W, O; write M, X, W)
+ALGO_BYTES_PER_ELEM = 24
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3_1.7b")
+    ap.add_argument("--ns-precision", default="fp16", choices=["fp16", "bf16", "fp32"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_desc(name):
+    import synth
+    wl = synth.workload(name)
+    shapes = [(m.rows, m.cols) for m in wl.matrices]
+    return wl, shapes
+
+
+def ns_flops(shapes, steps):
+    """Dense-convention Newton-Schulz FLOPs: per iteration 4 r^2 c + 2 r^3."""
+    tot = 0
+    for rr, cc in shapes:
+        r, c = min(rr, cc), max(rr, cc)
+        tot += steps * (4 * r * r * c + 2 * r ** 3)
+    return tot
+
+
+def apply_flops(shapes):
+    """One APPLY launch (Y' = aY + BY for every matrix): 2 r^2 c per matrix."""
+    return sum(2 * min(a, b) ** 2 * max(a, b) for a, b in shapes)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, indices):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", ",".join(str(i) for i in indices)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, power = [], [], set(), []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def committed_traffic(kernel_file, workload, prec):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    or None when the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    key = f"ns_apply/{workload}/{prec}"
+    if key not in d:
+        return None
+    src = os.path.join(ROOT, "pretraining_optimizer_b200", "csrc", kernel_file)
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if d[key].get("source_sha256") != digest:
+        return None
+    return d[key]["dram_bytes_per_launch"]
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample_rate(shapes, wl, sample_idx, steps=1):
+    """Time the oracle (as it stands, fp64) on a sample of the set for `steps`
+    steps; return (steps/s scaled to the whole set, seconds, sample FLOPs share)."""
+    import numpy as np
+    import oracle
+    W0 = {i: wl.weight(i) for i in sample_idx}
+    Gs = {(t, i): wl.grad(t, i) for t in range(steps) for i in sample_idx}
+    M = {i: np.zeros_like(W0[i], dtype=np.float64) for i in sample_idx}
+    W = {i: W0[i].astype(np.float64) for i in sample_idx}
+    R = {i: oracle.radius(W0[i]) for i in sample_idx}
+    t0 = time.perf_counter()
+    for t in range(steps):
+        for i in sample_idx:
+            W[i], M[i], _, _ = oracle.muonh_step(W[i], M[i], Gs[(t, i)], wl.lrs[t % len(wl.lrs)], R[i],
+                                                 wl.beta, wl.nesterov, wl.ns_steps, wl.ns_coeffs)
+    dt = time.perf_counter() - t0
+    share = ns_flops([shapes[i] for i in sample_idx], wl.ns_steps) / ns_flops(shapes, wl.ns_steps)
+    return steps * share / dt, dt, share
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((d.get("num_threads", 1) for d in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl, shapes = workload_desc(args.workload)
+    layer0 = list(range(min(7, len(shapes))))
+    times, shares = [], []
+    for k in range(args.warmup + args.steps):
+        idx = [layer0[k % len(layer0)]]           # one matrix of layer 0 per step, in rotation
+        _, dt, share = oracle_sample_rate(shapes, wl, idx)
+        if k >= args.warmup:
+            times.append(dt)
+            shares.append(share)
+    # each sampled step stands for share of a full step: full-step time = dt / share
+    full_step_s = sum(times) / sum(shares)
+    value = 1.0 / full_step_s
+    cores = blas_threads()
+    sample = (f"one layer-0 matrix per step in rotation ({len(layer0)} matrices), fp64 NumPy oracle, "
+              f"time scaled to the whole {len(shapes)}-matrix set by Newton-Schulz FLOP share")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * full_step_s,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "ns_steps": wl.ns_steps},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from pretraining_optimizer_b200 import MuonH
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl, shapes = workload_desc(args.workload)
+    n = len(shapes)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + rank)
+    W = [torch.randn(s, generator=gen, device=dev) * 0.02 for s in shapes]
+    M = [torch.zeros_like(w) for w in W]
+    G = [torch.randn(s, generator=gen, device=dev) * 1e-3 for s in shapes]
+    opt = MuonH(W, M, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps, ns_coeffs=wl.ns_coeffs,
+                ns_precision=args.ns_precision)
+    lrs = wl.lrs
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for k in range(args.warmup):
+        opt.step(G, lrs[k % len(lrs)])
+    torch.cuda.synchronize()
+    launches_per_step = opt.last_launch_count()
+    opt.phase_times()          # clear any record
+
+    # ---------------- timed region (device events on the launching stream)
+    opt.enable_timing(True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(range(world)) if rank == 0 else None
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        opt.step(G, lrs[k % len(lrs)])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    opt.enable_timing(False)
+    ms = t_start.elapsed_time(t_end)
+    phases = opt.phase_times()
+    opt.device_status()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1000.0)
+
+    # ---------------- end to end through the public API, host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = [torch.empty(s, dtype=torch.float32, pin_memory=True) for s in shapes]
+        for h, g in zip(host, G):
+            h.copy_(g)
+        stats_dev = torch.empty(n * 6, dtype=torch.int32, device=dev)
+        stats_host = torch.empty(n * 6, dtype=torch.int32, pin_memory=True)
+        e2e_steps = max(1, min(args.steps, 10))
+        opt.step(G, lrs[0])
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(e2e_steps):
+            for g, h in zip(G, host):
+                g.copy_(h, non_blocking=True)
+            opt.step(G, lrs[k % len(lrs)], stats=stats_dev)
+            stats_host.copy_(stats_dev, non_blocking=True)
+            stream.synchronize()                  # the caller reads the step's stats
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(4 * a * b for a, b in shapes)
+        e2e = {"value": world * e2e_steps / (e_ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": 24 * n, "steps": e2e_steps}
+        del host
+
+    # ---------------- rooflines from the live per-kernel events
+    peaks, peak_src = load_peaks()
+    elems = sum(a * b for a, b in shapes)
+    kernels = {}
+    for name, (tms, cnt) in phases.items():
+        if cnt == 0:
+            continue
+        entry = {"ms_per_launch": tms / cnt, "launches": cnt, "share": tms / sum(v[0] for v in phases.values())}
+        if name in KERNEL_BYTES:
+            entry["gbps"] = KERNEL_BYTES[name] * elems / (tms / cnt / 1000.0) / 1e9
+        kernels[name] = entry
+    apply_ms, apply_n = phases["ns_apply"]
+    ap_flops = apply_flops(shapes)
+    achieved = ap_flops / (apply_ms / apply_n / 1000.0) / 1e12
+    peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    roofline = {"bound": "tensor", "kernel": "ns_apply", "achieved": achieved, "peak": peak_t,
+                "unit": "TFLOP/s", "frac": achieved / peak_t,
+                "traffic": committed_traffic("muonh_ns_gemm.cu", args.workload, args.ns_precision),
+                "peak_source": f"bf16_tflops_sustained ({peak_src}); fp16 operands run at the bf16 rate"}
+    ns_ms = sum(phases[k][0] for k in ("ns_gram", "ns_square", "ns_apply")) / args.steps
+    ew_ms = sum(phases[k][0] for k in KERNEL_BYTES) / args.steps
+    summary = {
+        "ns_tflops_dense": ns_flops(shapes, wl.ns_steps) / (ns_ms / 1000.0) / 1e12,
+        "ns_ms_per_step": ns_ms,
+        "elementwise_ms_per_step": ew_ms,
+        "elementwise_gbps_algorithmic": ALGO_BYTES_PER_ELEM * elems / (ew_ms / 1000.0) / 1e9,
+        "hbm_peak_gbps": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+    }
+
+    # ---------------- CPU baseline: the oracle on layer 0, rank 0, N = 1
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = list(range(min(7, n)))
+        rate, dt, share = oracle_sample_rate(shapes, wl, sample)
+        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"layer 0 ({len(sample)} of {n} matrices, {share:.4f} of the NS FLOPs), one fp64 step "
+                         f"({dt:.1f} s), scaled to the whole set"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f16" if args.ns_precision == "fp16" else
+                ("bf16" if args.ns_precision == "bf16" else "f32"),
+                "data": "synthetic",
+                "config": {"workload": args.workload, "matrices": n, "params": elems,
+                           "ns_steps": wl.ns_steps, "ns_precision": args.ns_precision,
+                           "state": "fp32 W, M, G", "lr": "workload schedule",
+                           "l2": "inputs larger than L2 (no flush)",
+                           "parallelism": f"{world} independent replica(s)"},
+                "roofline": roofline, "summary": summary, "kernels": kernels, "clocks": clocks,
+                "gpu_launches": launches_per_step * args.steps, "e2e": e2e, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

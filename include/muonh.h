@@ -156,6 +156,32 @@ muonh_status muonh_device_status(muonh_ctx* ctx);
 /* Number of kernel launches the last muonh_step enqueued. */
 int32_t muonh_last_launch_count(const muonh_ctx* ctx);
 
+/* Kernel phases of one step, in launch order (ns_* repeat ns_steps times). */
+enum {
+  MUONH_PHASE_MOMENTUM_NORM = 0,   /* M update, ||X||^2 partials            */
+  MUONH_PHASE_FINALIZE_INPUT = 1,  /* per-matrix 1/(||X|| + eps)            */
+  MUONH_PHASE_WRITE_X = 2,         /* normalised 16-bit X, wide orientation */
+  MUONH_PHASE_NS_GRAM = 3,         /* A = Y Y^T                             */
+  MUONH_PHASE_NS_SQUARE = 4,       /* B = b A + c A A                       */
+  MUONH_PHASE_NS_APPLY = 5,        /* Y = a Y + B Y                         */
+  MUONH_PHASE_UPDATE_DOTS = 6,     /* ||O||^2, <W, O> partials              */
+  MUONH_PHASE_FINALIZE_UPDATE = 7, /* Eq. (1) scalars per matrix            */
+  MUONH_PHASE_PROJECT = 8,         /* W <- R (W - lr R u^)/||.||            */
+  MUONH_PHASE_FINALIZE_STEP = 9,   /* ||W_t+1||, stats                      */
+  MUONH_NUM_PHASES = 10
+};
+
+/* With enable != 0, every following muonh_step brackets each kernel with a
+ * pair of CUDA events on its stream (a few microseconds per step); 0 stops
+ * recording.  Recorded pairs are kept until muonh_phase_times reads them. */
+muonh_status muonh_enable_timing(muonh_ctx* ctx, int32_t enable);
+
+/* Synchronises the last stream and returns, per phase, the summed kernel
+ * time in ms (ms_out[MUONH_NUM_PHASES]) and the number of launches timed
+ * (launches_out[MUONH_NUM_PHASES], may be NULL) since the previous call;
+ * then clears the record. */
+muonh_status muonh_phase_times(muonh_ctx* ctx, float* ms_out, int64_t* launches_out);
+
 void muonh_destroy(muonh_ctx* ctx);
 
 const char* muonh_status_string(muonh_status s);

@@ -4,7 +4,7 @@
 // (r_pad x c_pad, r = min(rows, cols) on the wide orientation, both padded
 // to multiples of 256), allocates one zero-filled workspace per shape class
 // ([count][r_pad][c_pad] iterate ping-pong buffers and [count][r_pad][r_pad]
-// Gram and polynomial buffers), encodes one TMA descriptor per buffer and
+// buffers for A = Y Y^T, C = b I + c A and B' = a I + A C), encodes one TMA descriptor per buffer and
 // box shape, and builds the tile lists of the grouped GEMM launches.  Zero
 // padding is exact for the iteration: padded rows and columns of Y, A and B
 // stay zero, so no GEMM tile is ragged.
@@ -87,13 +87,15 @@ int safe_exponent(double bound) {
   return std::max(-24, std::min(15, e));
 }
 
-// Bounds on the entries of Y, A = Y Y^T and B = b A + c A^2 over all
-// iterations, from the scalar map sigma -> a s + b s^3 + c s^5 on the
-// singular values (entries are bounded by the spectral norm), starting from
+// Bounds on the entries of the stored operands over all iterations: Y,
+// A = Y Y^T, C = b I + c A and B' = a I + b A + c A^2.  Entries are bounded
+// by spectral norms, which follow from the scalar map
+// s -> a s + b s^3 + c s^5 on the singular values, starting from
 // sigma_max(Y_0) <= 1 after the Frobenius normalisation.
-void scale_exponents(float a, float b, float c, int steps, int prec, int32_t* ex, int32_t* ea, int32_t* eb) {
+void scale_exponents(float a, float b, float c, int steps, int prec, int32_t* ex, int32_t* ea, int32_t* ec,
+                     int32_t* eb) {
   if (prec == P_BF16) {
-    *ex = *ea = *eb = 0;
+    *ex = *ea = *ec = *eb = 0;
     return;
   }
   double smax = 1.0, s_all = 1.0;
@@ -110,13 +112,15 @@ void scale_exponents(float a, float b, float c, int steps, int prec, int32_t* ex
   }
   const double xmax = s_all * 1.02;
   const double amax = xmax * xmax;
-  double bmax = 0.0;
+  double cmax = 0.0, bmax = 0.0;
   for (int i = 0; i <= 8192; ++i) {
     const double l = amax * i / 8192;
-    bmax = std::max(bmax, std::fabs(b * l + c * l * l));
+    cmax = std::max(cmax, std::fabs(b + c * l));
+    bmax = std::max(bmax, std::fabs(a + b * l + c * l * l));
   }
   *ex = safe_exponent(xmax);
   *ea = safe_exponent(amax);
+  *ec = safe_exponent(std::max(cmax, 1e-30));
   *eb = safe_exponent(std::max(bmax, 1e-30));
 }
 
@@ -155,6 +159,26 @@ struct muonh_ctx {
   cudaEvent_t ev[kRing] = {};
   int ring = 0;
 
+  // optional per-kernel timing: (phase, begin event, end event)
+  bool timing = false;
+  struct Timed {
+    int phase;
+    cudaEvent_t begin, end;
+  };
+  std::vector<Timed> timed;
+  std::vector<cudaEvent_t> event_pool;
+
+  cudaEvent_t take_event() {
+    if (!event_pool.empty()) {
+      cudaEvent_t e = event_pool.back();
+      event_pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+
   EwParams ew(muonh_stats* stats_out) const {
     EwParams p{};
     p.mats = d_mats;
@@ -190,6 +214,11 @@ void release(muonh_ctx* ctx) {
     if (ctx->h_step[i]) cudaFreeHost(ctx->h_step[i]);
     if (ctx->ev[i]) cudaEventDestroy(ctx->ev[i]);
   }
+  for (auto& t : ctx->timed) {
+    cudaEventDestroy(t.begin);
+    cudaEventDestroy(t.end);
+  }
+  for (cudaEvent_t e : ctx->event_pool) cudaEventDestroy(e);
   delete ctx;
 }
 
@@ -219,6 +248,22 @@ muonh_status check_launch(cudaError_t e, const char* what) {
     muonh_status st_ = check_launch((expr), name);          \
     if (st_ != MUONH_OK) return st_;                        \
     ++launches;                                             \
+  } while (0)
+
+// A launch of the step, bracketed by events when timing is on.
+#define STEP_LAUNCH(phase, expr, name)                                   \
+  do {                                                                   \
+    cudaEvent_t ev_b = nullptr, ev_e = nullptr;                          \
+    if (ctx->timing) {                                                   \
+      ev_b = ctx->take_event();                                          \
+      ev_e = ctx->take_event();                                          \
+      CUDA_TRY(cudaEventRecord(ev_b, s));                                \
+    }                                                                    \
+    LAUNCH_TRY(expr, name);                                              \
+    if (ctx->timing) {                                                   \
+      CUDA_TRY(cudaEventRecord(ev_e, s));                                \
+      ctx->timed.push_back(muonh_ctx::Timed{phase, ev_b, ev_e});         \
+    }                                                                    \
   } while (0)
 
 }  // namespace
@@ -315,9 +360,17 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
     md.a = d.ns_a;
     md.b = d.ns_b;
     md.c_coef = d.ns_c;
-    scale_exponents(d.ns_a, d.ns_b, d.ns_c, d.ns_steps, ctx->prec, &md.ex, &md.ea, &md.eb);
-    md.et_rows = static_cast<int32_t>((d.rows + kEwTile - 1) / kEwTile);
-    md.et_cols = static_cast<int32_t>((d.cols + kEwTile - 1) / kEwTile);
+    scale_exponents(d.ns_a, d.ns_b, d.ns_c, d.ns_steps, ctx->prec, &md.ex, &md.ea, &md.ec, &md.eb);
+    if (md.transposed) {
+      md.et_th = md.et_tw = kEwTile;
+    } else {
+      int tw = kEwTile;
+      while (tw < 512 && tw < d.cols) tw *= 2;
+      md.et_tw = tw;
+      md.et_th = kEwTile * kEwTile / tw;
+    }
+    md.et_rows = static_cast<int32_t>((d.rows + md.et_th - 1) / md.et_th);
+    md.et_cols = static_cast<int32_t>((d.cols + md.et_tw - 1) / md.et_tw);
     md.et_begin = n_et;
     n_et += static_cast<int64_t>(md.et_rows) * md.et_cols;
     const std::pair<int64_t, int64_t> key(round_up(md.r, kPad), round_up(md.c, kPad));
@@ -352,9 +405,11 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", xb);
         CUDA_TRY(cudaMemsetAsync(cd.x[buf][part], 0, xb, s));
       }
-      if (dev_alloc(ctx, &cd.a[part], ab) != cudaSuccess || dev_alloc(ctx, &cd.b[part], ab) != cudaSuccess)
+      if (dev_alloc(ctx, &cd.a[part], ab) != cudaSuccess || dev_alloc(ctx, &cd.c[part], ab) != cudaSuccess ||
+          dev_alloc(ctx, &cd.b[part], ab) != cudaSuccess)
         return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", ab);
       CUDA_TRY(cudaMemsetAsync(cd.a[part], 0, ab, s));
+      CUDA_TRY(cudaMemsetAsync(cd.c[part], 0, ab, s));
       CUDA_TRY(cudaMemsetAsync(cd.b[part], 0, ab, s));
     }
   }
@@ -379,7 +434,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       }
       muonh_status st;
       if ((st = encode_map(&m[TM_A_K128 + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
-      if ((st = encode_map(&m[TM_A_K256 + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN))) return st;
+      if ((st = encode_map(&m[TM_C_K256 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN))) return st;
       if ((st = encode_map(&m[TM_B_K128 + part], cd.b[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
     }
   }
@@ -506,9 +561,9 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
   const EwParams p = ctx->ew(stats);
   const int grid = ctx->sm_count * 8;
   int launches = 0;
-  LAUNCH_TRY(launch_momentum_norm(p, grid, s), "momentum_norm");
-  LAUNCH_TRY(launch_finalize_input(p, s), "finalize_input");
-  LAUNCH_TRY(launch_write_x(p, grid, s), "write_x");
+  STEP_LAUNCH(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_norm(p, grid, s), "momentum_norm");
+  STEP_LAUNCH(MUONH_PHASE_FINALIZE_INPUT, launch_finalize_input(p, s), "finalize_input");
+  STEP_LAUNCH(MUONH_PHASE_WRITE_X, launch_write_x(p, grid, s), "write_x");
   for (int32_t k = 0; k < ctx->max_steps; ++k) {
     NsParams np{};
     np.mats = ctx->d_mats;
@@ -519,16 +574,18 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
     np.tiles = ctx->gram_lists[k].dev;
     np.ntiles = ctx->gram_lists[k].count;
     const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
-    LAUNCH_TRY(launch_ns_gemm(M_GRAM, ctx->prec, np, ggrid, s), "ns_gram");
-    LAUNCH_TRY(launch_ns_gemm(M_SQUARE, ctx->prec, np, ggrid, s), "ns_square");
+    STEP_LAUNCH(MUONH_PHASE_NS_GRAM, launch_ns_gemm(M_GRAM, ctx->prec, np, ggrid, s), "ns_gram");
+    STEP_LAUNCH(MUONH_PHASE_NS_SQUARE, launch_ns_gemm(M_SQUARE, ctx->prec, np, ggrid, s), "ns_square");
     np.tiles = ctx->apply_lists[k].dev;
     np.ntiles = ctx->apply_lists[k].count;
-    LAUNCH_TRY(launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), s), "ns_apply");
+    STEP_LAUNCH(MUONH_PHASE_NS_APPLY,
+                launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), s),
+                "ns_apply");
   }
-  LAUNCH_TRY(launch_update_dots(p, grid, s), "update_dots");
-  LAUNCH_TRY(launch_finalize_update(p, s), "finalize_update");
-  LAUNCH_TRY(launch_project(p, grid, s), "project");
-  LAUNCH_TRY(launch_finalize_step(p, s), "finalize_step");
+  STEP_LAUNCH(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, s), "update_dots");
+  STEP_LAUNCH(MUONH_PHASE_FINALIZE_UPDATE, launch_finalize_update(p, s), "finalize_update");
+  STEP_LAUNCH(MUONH_PHASE_PROJECT, launch_project(p, grid, s), "project");
+  STEP_LAUNCH(MUONH_PHASE_FINALIZE_STEP, launch_finalize_step(p, s), "finalize_step");
   ctx->last_launches = launches;
   ctx->last_stream = s;
   ++ctx->step_count;
@@ -631,6 +688,35 @@ muonh_status muonh_device_status(muonh_ctx* ctx) {
 }
 
 int32_t muonh_last_launch_count(const muonh_ctx* ctx) { return ctx ? ctx->last_launches : 0; }
+
+muonh_status muonh_enable_timing(muonh_ctx* ctx, int32_t enable) {
+  g_last_error.clear();
+  if (!ctx) return fail(MUONH_ERR_INVALID_ARG, "ctx is NULL");
+  ctx->timing = enable != 0;
+  return MUONH_OK;
+}
+
+muonh_status muonh_phase_times(muonh_ctx* ctx, float* ms_out, int64_t* launches_out) {
+  g_last_error.clear();
+  if (!ctx || !ms_out) return fail(MUONH_ERR_INVALID_ARG, "ctx or ms_out is NULL");
+  CUDA_TRY(cudaStreamSynchronize(ctx->last_stream));
+  double acc[MUONH_NUM_PHASES] = {};
+  int64_t cnt[MUONH_NUM_PHASES] = {};
+  for (auto& t : ctx->timed) {
+    float ms = 0.f;
+    CUDA_TRY(cudaEventElapsedTime(&ms, t.begin, t.end));
+    acc[t.phase] += ms;
+    cnt[t.phase] += 1;
+    ctx->event_pool.push_back(t.begin);
+    ctx->event_pool.push_back(t.end);
+  }
+  ctx->timed.clear();
+  for (int i = 0; i < MUONH_NUM_PHASES; ++i) {
+    ms_out[i] = static_cast<float>(acc[i]);
+    if (launches_out) launches_out[i] = cnt[i];
+  }
+  return MUONH_OK;
+}
 
 void muonh_destroy(muonh_ctx* ctx) {
   if (!ctx) return;

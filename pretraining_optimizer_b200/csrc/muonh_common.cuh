@@ -33,8 +33,8 @@ enum TmSlot {
   TM_X_K256 = 4,   // X[buf] as K-major operand, 256-row box
   TM_X_MN = 8,     // X[buf] as MN-major operand, 64 x 64 box
   TM_A_K128 = 12,  // A, 128-row box (+part)
-  TM_A_K256 = 14,  // A, 256-row box (+part)
-  TM_B_K128 = 16,  // B, 128-row box (+part)
+  TM_C_K256 = 14,  // C = b I + c A, 256-row box (+part)
+  TM_B_K128 = 16,  // B' = a I + A C, 128-row box (+part)
   TM_PER_CLASS = 18
 };
 __host__ __device__ inline int tm_x(int base, int buf, int part) { return base + buf + 2 * part; }
@@ -51,16 +51,18 @@ struct MatDev {
   int32_t nesterov;
   int32_t ns_steps;
   float a, b, c_coef;
-  int32_t ex, ea, eb;        // power-of-two scales of stored X, A, B
+  int32_t ex, ea, ec, eb;    // power-of-two scales of stored X, A, C, B'
   int32_t et_rows, et_cols;  // elementwise tile grid
+  int32_t et_th, et_tw;      // elementwise tile shape: 64 x 64 for tall W, <= 8 x 512 rows otherwise
   int64_t et_begin;          // first elementwise tile
 };
 
 struct ClassDev {
   int32_t r_pad, c_pad, count, tm_base;
   void* x[2][2];             // [buf][part]
-  void* a[2];                // [part]
-  void* b[2];
+  void* a[2];                // [part]: A = Y Y^T
+  void* c[2];                // C = b I + c A
+  void* b[2];                // B' = a I + A C
   int64_t x_stride, a_stride;   // elements per matrix
 };
 

@@ -13,11 +13,16 @@
 namespace muonh {
 namespace {
 
-constexpr int kTy = kEwThreads / 16;    // 16 rows per pass, 16 threads x float4 per row
+// Every tile holds 4096 elements: 64 x 64 for tall matrices (whose X/O is
+// the transpose), th x tw with tw = min(512, cols rounded up to 64) rows
+// otherwise.  A thread covers 4 consecutive columns in each of 4 passes.
+constexpr int kPasses = 4;
 
 struct TileCoord {
   int mi;
   int64_t r0, c0;
+  int rin, cin;     // this thread's first row / column inside the tile
+  int rstep;        // rows between passes
 };
 
 __device__ __forceinline__ TileCoord tile_coord(const EwParams& p, int64_t e) {
@@ -25,8 +30,12 @@ __device__ __forceinline__ TileCoord tile_coord(const EwParams& p, int64_t e) {
   t.mi = p.et_mat[e];
   const MatDev& md = p.mats[t.mi];
   const int64_t local = e - md.et_begin;
-  t.r0 = (local / md.et_cols) * kEwTile;
-  t.c0 = (local % md.et_cols) * kEwTile;
+  t.r0 = (local / md.et_cols) * md.et_th;
+  t.c0 = (local % md.et_cols) * md.et_tw;
+  const int tpr = md.et_tw / 4;    // threads per tile row
+  t.rin = threadIdx.x / tpr;
+  t.cin = (threadIdx.x % tpr) * 4;
+  t.rstep = kEwThreads / tpr;
   return t;
 }
 
@@ -84,13 +93,6 @@ __device__ __forceinline__ void put16(void* hi, void* lo, int64_t off, float v, 
   }
 }
 
-__device__ __forceinline__ float get16(const void* hi, const void* lo, int64_t off, int prec) {
-  if (prec == P_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(hi)[off]);
-  float v = __half2float(reinterpret_cast<const __half*>(hi)[off]);
-  if (prec == P_FP32) v += __half2float(reinterpret_cast<const __half*>(lo)[off]);
-  return v;
-}
-
 struct XView {
   void* hi;
   void* lo;
@@ -107,35 +109,91 @@ __device__ __forceinline__ XView x_view(const EwParams& p, const MatDev& md, int
   return v;
 }
 
-// Read the 64 x 64 tile of O (W orientation, stored scale) into tile[r][c].
-__device__ __forceinline__ void load_o_tile(const EwParams& p, const MatDev& md, const TileCoord& tc,
-                                            float (*tile)[kEwTile + 1]) {
-  const XView xv = x_view(p, md, md.ns_steps & 1);
-  if (!md.transposed) {
-    // O(p, q) = X[p][q]
-    for (int i = threadIdx.x; i < kEwTile * kEwTile; i += kEwThreads) {
-      const int r = i / kEwTile, c = i % kEwTile;
-      tile[r][c] = get16(xv.hi, xv.lo, (tc.r0 + r) * xv.ld + tc.c0 + c, p.prec);
-    }
+// Four consecutive stored values X[row][col..col+3] (8-byte aligned).
+__device__ __forceinline__ float4 x4(const XView& xv, int64_t off, int prec) {
+  float4 r;
+  const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(xv.hi) + off);
+  if (prec == P_BF16) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    r = make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
   } else {
-    // O(p, q) = X[q][p]: read X rows q (coalesced along p), write transposed
-    for (int i = threadIdx.x; i < kEwTile * kEwTile; i += kEwThreads) {
-      const int q = i / kEwTile, r = i % kEwTile;
-      tile[r][q] = get16(xv.hi, xv.lo, (tc.c0 + q) * xv.ld + tc.r0 + r, p.prec);
+    const __half2 a = *reinterpret_cast<const __half2*>(&u.x);
+    const __half2 b = *reinterpret_cast<const __half2*>(&u.y);
+    r = make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+    if (prec == P_FP32) {
+      const uint2 l = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(xv.lo) + off);
+      const __half2 c = *reinterpret_cast<const __half2*>(&l.x);
+      const __half2 d = *reinterpret_cast<const __half2*>(&l.y);
+      r.x += __low2float(c);
+      r.y += __high2float(c);
+      r.z += __low2float(d);
+      r.w += __high2float(d);
     }
   }
+  return r;
+}
+
+// O(r0 + i, c0 + j) = X[c0 + j][r0 + i] of a tall matrix into tile[i][j]
+// (64 x 64), with 16-byte loads along X's rows.
+__device__ __forceinline__ void load_o_tile_t(const XView& xv, const TileCoord& tc, int prec,
+                                              float (*tile)[kEwTile + 1]) {
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int q = threadIdx.x / 8 + 32 * pass;
+    const int p0 = (threadIdx.x % 8) * 8;
+    const int64_t off = (tc.c0 + q) * xv.ld + tc.r0 + p0;
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(xv.hi) + off);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (prec == P_BF16) {
+        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[k]);
+        v[2 * k] = __low2float(h);
+        v[2 * k + 1] = __high2float(h);
+      } else {
+        const __half2 h = *reinterpret_cast<const __half2*>(&w[k]);
+        v[2 * k] = __low2float(h);
+        v[2 * k + 1] = __high2float(h);
+      }
+    }
+    if (prec == P_FP32) {
+      const uint4 l = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(xv.lo) + off);
+      const uint32_t lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&lw[k]);
+        v[2 * k] += __low2float(h);
+        v[2 * k + 1] += __high2float(h);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tile[p0 + i][q] = v[i];
+  }
+}
+
+// O at W coordinates (row, col..col+3), stored scale: direct for wide
+// matrices, from the transposed smem tile for tall ones.
+__device__ __forceinline__ float4 o_at(const XView& xv, const MatDev& md, const TileCoord& tc, int r, int c,
+                                       int prec, float (*tile)[kEwTile + 1]) {
+  if (!md.transposed) {
+    // tiles may reach past the padded width when cols is not a multiple of the tile width
+    if (tc.c0 + c >= xv.ld) return make_float4(0.f, 0.f, 0.f, 0.f);
+    return x4(xv, (tc.r0 + r) * xv.ld + tc.c0 + c, prec);
+  }
+  return make_float4(tile[r][c], tile[r][c + 1], tile[r][c + 2], tile[r][c + 3]);
 }
 
 // ------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kEwThreads) init_norm_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     double acc = 0.0;
-    for (int j = 0; j < kEwTile / kTy; ++j) {
-      const float4 w = load4(md.w, md, tc.r0 + ty + kTy * j, tc.c0 + tx * 4);
+    for (int j = 0; j < kPasses; ++j) {
+      const float4 w = load4(md.w, md, tc.r0 + tc.rin + tc.rstep * j, tc.c0 + tc.cin);
       acc += (double)w.x * w.x + (double)w.y * w.y + (double)w.z * w.z + (double)w.w * w.w;
     }
     const double s = block_sum(acc, red);
@@ -146,25 +204,24 @@ __global__ void __launch_bounds__(kEwThreads) init_norm_kernel(const EwParams p)
 // M <- beta M + G; X = G + beta M (Nesterov) or M; partial ||X||^2.
 __global__ void __launch_bounds__(kEwThreads) momentum_norm_kernel(const EwParams p) {
   __shared__ float red[kEwThreads / 32];
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     const float* g = p.step[tc.mi].g;
     const float beta = md.beta;
-    constexpr int J = kEwTile / kTy;
+    constexpr int J = kPasses;
     float4 gv[J], mv[J];
     // issue every load of the tile before the first store
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-      const int64_t row = tc.r0 + ty + kTy * j, col = tc.c0 + tx * 4;
+      const int64_t row = tc.r0 + tc.rin + tc.rstep * j, col = tc.c0 + tc.cin;
       gv[j] = load4(g, md, row, col);
       mv[j] = load4(md.m, md, row, col);
     }
     float acc = 0.f;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-      const int64_t row = tc.r0 + ty + kTy * j, col = tc.c0 + tx * 4;
+      const int64_t row = tc.r0 + tc.rin + tc.rstep * j, col = tc.c0 + tc.cin;
       float4 m = mv[j];
       m.x = fmaf(beta, m.x, gv[j].x);
       m.y = fmaf(beta, m.y, gv[j].y);
@@ -191,7 +248,6 @@ __global__ void __launch_bounds__(kEwThreads) momentum_norm_kernel(const EwParam
 // X_stored = xscale * X into NS buffer 0 (wide orientation, transposed for tall W).
 __global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
@@ -201,8 +257,8 @@ __global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
     const XView xv = x_view(p, md, 0);
     if (!md.transposed) {
 #pragma unroll
-      for (int j = 0; j < kEwTile / kTy; ++j) {
-        const int64_t row = tc.r0 + ty + kTy * j, col = tc.c0 + tx * 4;
+      for (int j = 0; j < kPasses; ++j) {
+        const int64_t row = tc.r0 + tc.rin + tc.rstep * j, col = tc.c0 + tc.cin;
         const float4 gv = load4(g, md, row, col);
         const float4 mv = load4(md.m, md, row, col);
         float4 x = mv;
@@ -212,6 +268,7 @@ __global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
           x.z = fmaf(beta, mv.z, gv.z);
           x.w = fmaf(beta, mv.w, gv.w);
         }
+        if (col >= xv.ld) continue;   // past the padded width (see o_at)
         const int64_t off = row * xv.ld + col;
         if (p.prec == P_FP16) {
           __half2 h01 = __floats2half2_rn(x.x * xs, x.y * xs);
@@ -229,9 +286,10 @@ __global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
       }
     } else {
       __syncthreads();   // previous tile's readers are done with `tile`
+      const int tx = tc.cin / 4;
 #pragma unroll
-      for (int j = 0; j < kEwTile / kTy; ++j) {
-        const int r = ty + kTy * j;
+      for (int j = 0; j < kPasses; ++j) {
+        const int r = tc.rin + tc.rstep * j;
         const int64_t row = tc.r0 + r, col = tc.c0 + tx * 4;
         const float4 gv = load4(g, md, row, col);
         const float4 mv = load4(md.m, md, row, col);
@@ -271,34 +329,23 @@ __global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
 __global__ void __launch_bounds__(kEwThreads) update_dots_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   __shared__ float red[kEwThreads / 32];
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
-    if (p.scal[tc.mi].flags & MUONH_FLAG_NONFINITE_INPUT) {
-      if (threadIdx.x == 0) {
-        p.part[2 * e] = 0.f;
-        p.part[2 * e + 1] = 0.f;
-      }
-      continue;
+    const XView xv = x_view(p, md, md.ns_steps & 1);
+    if (md.transposed) {
+      __syncthreads();
+      load_o_tile_t(xv, tc, p.prec, tile);
+      __syncthreads();
     }
-    __syncthreads();
-    load_o_tile(p, md, tc, tile);
-    __syncthreads();
     float oo = 0.f, wo = 0.f;
 #pragma unroll
-    for (int j = 0; j < kEwTile / kTy; ++j) {
-      const int r = ty + kTy * j;
-      const float4 w = load4(md.w, md, tc.r0 + r, tc.c0 + tx * 4);
-      const float* o = &tile[r][tx * 4];
-      oo = fmaf(o[0], o[0], oo);
-      oo = fmaf(o[1], o[1], oo);
-      oo = fmaf(o[2], o[2], oo);
-      oo = fmaf(o[3], o[3], oo);
-      wo = fmaf(w.x, o[0], wo);
-      wo = fmaf(w.y, o[1], wo);
-      wo = fmaf(w.z, o[2], wo);
-      wo = fmaf(w.w, o[3], wo);
+    for (int j = 0; j < kPasses; ++j) {
+      const int r = tc.rin + tc.rstep * j;
+      const float4 w = load4(md.w, md, tc.r0 + r, tc.c0 + tc.cin);
+      const float4 o = o_at(xv, md, tc, r, tc.cin, p.prec, tile);
+      oo = fmaf(o.x, o.x, fmaf(o.y, o.y, fmaf(o.z, o.z, fmaf(o.w, o.w, oo))));
+      wo = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, wo))));
     }
     const float s_oo = block_sum(oo, red);
     const float s_wo = block_sum(wo, red);
@@ -313,7 +360,6 @@ __global__ void __launch_bounds__(kEwThreads) update_dots_kernel(const EwParams 
 __global__ void __launch_bounds__(kEwThreads) project_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   __shared__ float red[kEwThreads / 32];
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
@@ -324,38 +370,31 @@ __global__ void __launch_bounds__(kEwThreads) project_kernel(const EwParams p) {
       continue;
     }
     const float kw = sc.kw, ko = sc.ko;
-    if (mode == 0) {
+    const XView xv = x_view(p, md, md.ns_steps & 1);
+    if (mode == 0 && md.transposed) {
       __syncthreads();
-      load_o_tile(p, md, tc, tile);
+      load_o_tile_t(xv, tc, p.prec, tile);
       __syncthreads();
     }
-    constexpr int J = kEwTile / kTy;
-    float4 wv[J];
+    float4 wv[kPasses], ov[kPasses];
 #pragma unroll
-    for (int j = 0; j < J; ++j) wv[j] = load4(md.w, md, tc.r0 + ty + kTy * j, tc.c0 + tx * 4);
+    for (int j = 0; j < kPasses; ++j) {
+      const int r = tc.rin + tc.rstep * j;
+      wv[j] = load4(md.w, md, tc.r0 + r, tc.c0 + tc.cin);
+      ov[j] = mode == 0 ? o_at(xv, md, tc, r, tc.cin, p.prec, tile) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int r = ty + kTy * j;
-      const int64_t row = tc.r0 + r, col = tc.c0 + tx * 4;
+    for (int j = 0; j < kPasses; ++j) {
+      const int r = tc.rin + tc.rstep * j;
       float4 w = wv[j];
-      if (mode == 0) {
-        const float* o = &tile[r][tx * 4];
-        w.x = fmaf(ko, o[0], kw * w.x);
-        w.y = fmaf(ko, o[1], kw * w.y);
-        w.z = fmaf(ko, o[2], kw * w.z);
-        w.w = fmaf(ko, o[3], kw * w.w);
-      } else {
-        w.x *= kw;
-        w.y *= kw;
-        w.z *= kw;
-        w.w *= kw;
-      }
-      store4(md.w, md, row, col, w);
-      acc = fmaf(w.x, w.x, acc);
-      acc = fmaf(w.y, w.y, acc);
-      acc = fmaf(w.z, w.z, acc);
-      acc = fmaf(w.w, w.w, acc);
+      const float4 o = ov[j];
+      w.x = fmaf(ko, o.x, kw * w.x);
+      w.y = fmaf(ko, o.y, kw * w.y);
+      w.z = fmaf(ko, o.z, kw * w.z);
+      w.w = fmaf(ko, o.w, kw * w.w);
+      store4(md.w, md, tc.r0 + r, tc.c0 + tc.cin, w);
+      acc = fmaf(w.x, w.x, fmaf(w.y, w.y, fmaf(w.z, w.z, fmaf(w.w, w.w, acc))));
     }
     const float s = block_sum(acc, red);
     if (threadIdx.x == 0) p.part[e] = s;
@@ -368,17 +407,23 @@ __global__ void __launch_bounds__(kEwThreads) export_update_kernel(const EwParam
   __shared__ float tile[kEwTile][kEwTile + 1];
   const MatDev& md = p.mats[mi];
   const float unscale = exp2f(static_cast<float>(-md.ex));
+  const XView xv = x_view(p, md, md.ns_steps & 1);
   const int64_t n_tiles = static_cast<int64_t>(md.et_rows) * md.et_cols;
   for (int64_t local = blockIdx.x; local < n_tiles; local += gridDim.x) {
-    const int64_t e = md.et_begin + local;
-    const TileCoord tc = tile_coord(p, e);
-    __syncthreads();
-    load_o_tile(p, md, tc, tile);
-    __syncthreads();
-    for (int i = threadIdx.x; i < kEwTile * kEwTile; i += kEwThreads) {
-      const int r = i / kEwTile, c = i % kEwTile;
-      const int64_t row = tc.r0 + r, col = tc.c0 + c;
-      if (row < md.rows && col < md.cols) dst[row * ld + col] = tile[r][c] * unscale;
+    const TileCoord tc = tile_coord(p, md.et_begin + local);
+    if (md.transposed) {
+      __syncthreads();
+      load_o_tile_t(xv, tc, p.prec, tile);
+      __syncthreads();
+    }
+    for (int j = 0; j < kPasses; ++j) {
+      const int r = tc.rin + tc.rstep * j;
+      const float4 o = o_at(xv, md, tc, r, tc.cin, p.prec, tile);
+      const int64_t row = tc.r0 + r, col = tc.c0 + tc.cin;
+      if (row >= md.rows) continue;
+      const float ov[4] = {o.x, o.y, o.z, o.w};
+      for (int k = 0; k < 4; ++k)
+        if (col + k < md.cols) dst[row * ld + col + k] = ov[k] * unscale;
     }
   }
 }

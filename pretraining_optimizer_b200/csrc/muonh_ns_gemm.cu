@@ -1,11 +1,13 @@
 // Grouped Newton-Schulz GEMMs on the 5th-generation tensor cores (sm_100a).
 //
-// One Newton-Schulz iteration on a wide matrix Y (r x c) is three products
+// One Newton-Schulz iteration on a wide matrix Y (r x c),
+//   Y' = a Y + (b A + c A A) Y,   A = Y Y^T
 // (quintic iteration of the Muon update; the MuonH wrapper of the Puro-2B
-// report, Sec. 3.3, normalises its output):
-//   GRAM    A  = Y Y^T                 M = r, N = r, K = c   (symmetric)
-//   SQUARE  B  = b A + c A A           M = r, N = r, K = r   (symmetric)
-//   APPLY   Y' = a Y + B Y             M = r, N = c, K = r
+// report, Sec. 3.3, normalises its output), runs as three products with the
+// polynomial folded into the operands so that no epilogue reads memory:
+//   GRAM    A  = Y Y^T,  and  C = b I + c A      M = r, N = r, K = c   (symmetric)
+//   SQUARE  B' = A C + a I                       M = r, N = r, K = r   (symmetric)
+//   APPLY   Y' = B' Y                            M = r, N = c, K = r
 // Every launch covers the tiles of all matrices of the step (grouped), in a
 // persistent grid of one CTA per SM.  Symmetric products compute only the
 // 128 x 256 tiles that touch the upper triangle and write each element of
@@ -86,27 +88,6 @@ __device__ __forceinline__ void store_one(void* hi_base, void* lo_base, int64_t 
   T hv = S::cvt(v);
   reinterpret_cast<T*>(hi_base)[off] = hv;
   if (PREC == P_FP32) reinterpret_cast<__half*>(lo_base)[off] = __float2half_rn(v - S::back(hv));
-}
-
-template <int PREC>
-__device__ __forceinline__ void load_row32(const void* hi_base, const void* lo_base, int64_t off, float (&v)[32]) {
-  using S = Store16<PREC>;
-  using T = typename S::T;
-  uint4 hbuf[4], lbuf[4];
-  const uint4* sh = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(hi_base) + off);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) hbuf[q] = sh[q];
-  const T* h = reinterpret_cast<const T*>(hbuf);
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = S::back(h[j]);
-  if (PREC == P_FP32) {
-    const uint4* sl = reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(lo_base) + off);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) lbuf[q] = sl[q];
-    const __half* l = reinterpret_cast<const __half*>(lbuf);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] += __half2float(l[j]);
-  }
 }
 
 // Symmetric output: element (row, col) of the upper triangle (col >= row)
@@ -193,7 +174,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
                           td.bj * kBN, z);
             } else if (MODE == M_SQUARE) {
               tma_load_3d(a_dst, p.tmaps + cd.tm_base + TM_A_K128 + part, &full[stage], k0, td.bi * kBM, z);
-              tma_load_3d(b_dst, p.tmaps + cd.tm_base + TM_A_K256 + part, &full[stage], k0, td.bj * kBN, z);
+              tma_load_3d(b_dst, p.tmaps + cd.tm_base + TM_C_K256 + part, &full[stage], k0, td.bj * kBN, z);
             } else {
               tma_load_3d(a_dst, p.tmaps + cd.tm_base + TM_B_K128 + part, &full[stage], k0, td.bi * kBM, z);
               const CUtensorMap* xm = p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, part);
@@ -289,52 +270,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       const int warp_row0 = row - lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       if (MODE == M_GRAM) {
-        const float sc = exp2f(static_cast<float>(md.ea - 2 * md.ex));
-        void* hi = static_cast<uint8_t*>(cd.a[0]) + md.z * cd.a_stride * 2;
-        void* lo = cd.a[1] ? static_cast<uint8_t*>(cd.a[1]) + md.z * cd.a_stride * 2 : nullptr;
+        // acc = 2^(2ex) A;  A_s = 2^ea A;  C_s = 2^ec (b I + c A)
+        const float sa = exp2f(static_cast<float>(md.ea - 2 * md.ex));
+        const float sc = md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
+        const float diag = md.b * exp2f(static_cast<float>(md.ec));
+        const int64_t mo = md.z * cd.a_stride * 2;
+        void* ahi = static_cast<uint8_t*>(cd.a[0]) + mo;
+        void* alo = cd.a[1] ? static_cast<uint8_t*>(cd.a[1]) + mo : nullptr;
+        void* chi = static_cast<uint8_t*>(cd.c[0]) + mo;
+        void* clo = cd.c[1] ? static_cast<uint8_t*>(cd.c[1]) + mo : nullptr;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int col0 = td.bj * kBN + ch * 32;
+          if (col0 + 31 < warp_row0) continue;   // whole chunk below the diagonal for this warp
+          float v[32], w[32];
+          tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            w[j] = sc * v[j];
+            v[j] *= sa;
+          }
+          const int dj = row - col0;   // diagonal element of this row, if in the chunk
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j == dj) w[j] += diag;
+          store_symmetric<PREC>(ahi, alo, cd.r_pad, row, col0, v);
+          store_symmetric<PREC>(chi, clo, cd.r_pad, row, col0, w);
+        }
+      } else if (MODE == M_SQUARE) {
+        // acc = 2^(ea+ec) A C;  B'_s = 2^eb (A C + a I)
+        const float sb = exp2f(static_cast<float>(md.eb - md.ea - md.ec));
+        const float diag = md.a * exp2f(static_cast<float>(md.eb));
+        const int64_t mo = md.z * cd.a_stride * 2;
+        void* bhi = static_cast<uint8_t*>(cd.b[0]) + mo;
+        void* blo = cd.b[1] ? static_cast<uint8_t*>(cd.b[1]) + mo : nullptr;
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
           if (col0 + 31 < warp_row0) continue;   // whole chunk below the diagonal for this warp
           float v[32];
           tmem_ld32(taddr + ch * 32, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= sc;
-          store_symmetric<PREC>(hi, lo, cd.r_pad, row, col0, v);
-        }
-      } else if (MODE == M_SQUARE) {
-        const float kb_ = md.b * exp2f(static_cast<float>(md.eb - md.ea));
-        const float kc_ = md.c_coef * exp2f(static_cast<float>(md.eb - 2 * md.ea));
-        const void* ahi = static_cast<const uint8_t*>(cd.a[0]) + md.z * cd.a_stride * 2;
-        const void* alo = cd.a[1] ? static_cast<const uint8_t*>(cd.a[1]) + md.z * cd.a_stride * 2 : nullptr;
-        void* bhi = static_cast<uint8_t*>(cd.b[0]) + md.z * cd.a_stride * 2;
-        void* blo = cd.b[1] ? static_cast<uint8_t*>(cd.b[1]) + md.z * cd.a_stride * 2 : nullptr;
-        for (int ch = 0; ch < kBN / 32; ++ch) {
-          const int col0 = td.bj * kBN + ch * 32;
-          if (col0 + 31 < warp_row0) continue;   // whole chunk below the diagonal for this warp
-          float v[32], a[32];
-          tmem_ld32(taddr + ch * 32, v);
-          load_row32<PREC>(ahi, alo, static_cast<int64_t>(row) * cd.r_pad + col0, a);
+          for (int j = 0; j < 32; ++j) v[j] *= sb;
+          const int dj = row - col0;   // diagonal element of this row, if in the chunk
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = fmaf(kc_, v[j], kb_ * a[j]);
+          for (int j = 0; j < 32; ++j)
+            if (j == dj) v[j] += diag;
           store_symmetric<PREC>(bhi, blo, cd.r_pad, row, col0, v);
         }
       } else {
+        // acc = 2^(eb+ex) B' Y;  Y'_s = 2^ex B' Y
         const float ks = exp2f(static_cast<float>(-md.eb));
-        const float ca = md.a;
         const int64_t xo = md.z * cd.x_stride * 2;
-        const void* xhi = static_cast<const uint8_t*>(cd.x[p.src][0]) + xo;
-        const void* xlo = cd.x[p.src][1] ? static_cast<const uint8_t*>(cd.x[p.src][1]) + xo : nullptr;
         void* yhi = static_cast<uint8_t*>(cd.x[p.src ^ 1][0]) + xo;
         void* ylo = cd.x[p.src ^ 1][1] ? static_cast<uint8_t*>(cd.x[p.src ^ 1][1]) + xo : nullptr;
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
-          const int64_t off = static_cast<int64_t>(row) * cd.c_pad + col0;
-          float v[32], x[32];
+          float v[32];
           tmem_ld32(taddr + ch * 32, v);
-          load_row32<PREC>(xhi, xlo, off, x);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = fmaf(ks, v[j], ca * x[j]);
-          store_row32<PREC>(yhi, ylo, off, v);
+          for (int j = 0; j < 32; ++j) v[j] *= ks;
+          store_row32<PREC>(yhi, ylo, static_cast<int64_t>(row) * cd.c_pad + col0, v);
         }
       }
       tc_fence_before();

@@ -22,8 +22,10 @@ FLAG_TIMEOUT = 16
 EXPORTED_SYMBOLS = (
     "muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
     "muonh_export_state", "muonh_import_state", "muonh_device_status", "muonh_last_launch_count",
-    "muonh_destroy", "muonh_status_string", "muonh_last_error",
+    "muonh_enable_timing", "muonh_phase_times", "muonh_destroy", "muonh_status_string", "muonh_last_error",
 )
+PHASES = ("momentum_norm", "finalize_input", "write_x", "ns_gram", "ns_square", "ns_apply",
+          "update_dots", "finalize_update", "project", "finalize_step")
 
 
 class MatrixDesc(Structure):
@@ -73,6 +75,8 @@ def library() -> ctypes.CDLL:
     lib.muonh_device_status.argtypes = [c_void_p]
     lib.muonh_last_launch_count.argtypes = [c_void_p]
     lib.muonh_last_launch_count.restype = c_int32
+    lib.muonh_enable_timing.argtypes = [c_void_p, c_int32]
+    lib.muonh_phase_times.argtypes = [c_void_p, POINTER(c_float), POINTER(c_int64)]
     lib.muonh_destroy.argtypes = [c_void_p]
     lib.muonh_destroy.restype = None
     lib.muonh_status_string.argtypes = [c_int32]
@@ -80,7 +84,8 @@ def library() -> ctypes.CDLL:
     lib.muonh_last_error.argtypes = []
     lib.muonh_last_error.restype = c_char_p
     for name in ("muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
-                 "muonh_export_state", "muonh_import_state", "muonh_device_status"):
+                 "muonh_export_state", "muonh_import_state", "muonh_device_status",
+                 "muonh_enable_timing", "muonh_phase_times"):
         getattr(lib, name).restype = c_int32
     _LIB = lib
     return lib
@@ -199,6 +204,16 @@ class MuonH:
 
     def last_launch_count(self) -> int:
         return int(self._lib.muonh_last_launch_count(self._ctx))
+
+    def enable_timing(self, enable: bool = True) -> None:
+        _check(self._lib.muonh_enable_timing(self._ctx, int(bool(enable))))
+
+    def phase_times(self) -> dict:
+        """{phase: (total ms, launches)} recorded since the previous call."""
+        ms = (c_float * len(PHASES))()
+        cnt = (c_int64 * len(PHASES))()
+        _check(self._lib.muonh_phase_times(self._ctx, ms, cnt))
+        return {name: (float(ms[i]), int(cnt[i])) for i, name in enumerate(PHASES)}
 
     def device_status(self) -> None:
         _check(self._lib.muonh_device_status(self._ctx))

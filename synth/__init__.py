@@ -185,6 +185,13 @@ class Workload:
 
 
 def workload(name: str) -> Workload:
+    """Named workloads; "<set>:L" keeps the first L layers of a Qwen3 set."""
+    if ":" in name:
+        base, layers = name.split(":")
+        wl = workload(base)
+        keep = 7 * int(layers)
+        return Workload(name, wl.matrices[:keep], wl.lrs, wl.gradient, wl.beta, wl.nesterov,
+                        wl.ns_steps, wl.ns_coeffs)
     if name == "single_256x512":
         return Workload(name, single_256x512(), constant_lr(10, 0.01))
     if name == "qwen3_0.6b":

@@ -112,6 +112,20 @@ def test_edge_cases_zero_nan_and_zero_lr():
     assert st[3]["flags"] == 0 and abs(st[3]["elr"] - 0.02) <= NORM_TOL * 0.02
 
 
+def test_zero_newton_schulz_steps_uses_the_normalised_input():
+    """ns_steps = 0: O = X/(||X|| + eps) (fp16 storage), mixed with a matrix that iterates."""
+    shapes = [(256, 512), (512, 256)]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    for steps in (0, 1):
+        g = run_gpu(W0, grad, [0.01, 0.01], ns_steps=steps, keep_updates=(1,))
+        o = run_oracle(W0, grad, [0.01, 0.01], ns_steps=steps, keep_updates=(1,))
+        for i in range(2):
+            assert rel_fro(g["O"][1][i], o["O"][1][i]) <= (1e-3 if steps == 0 else 4e-3)
+            assert abs(g["stats"][1][i]["post_norm"] - o["R"][i]) <= NORM_TOL * o["R"][i]
+            assert np.linalg.norm(g["W"][i] - o["W"][i]) / o["R"][i] <= 1e-4
+
+
 def test_convergent_coefficients_reach_the_polar_factor():
     """With (15/8, -10/8, 3/8) the iteration converges to U V^T (fp32 NS mode, 30 steps)."""
     rng = np.random.default_rng(3)
