@@ -182,6 +182,28 @@ muonh_status muonh_enable_timing(muonh_ctx* ctx, int32_t enable);
  * then clears the record. */
 muonh_status muonh_phase_times(muonh_ctx* ctx, float* ms_out, int64_t* launches_out);
 
+/* Allocation-free momentum stage for one matrix (the report has no
+ * counterpart; this is a deployment convenience).  Computes, like the first
+ * kernel of muonh_step, M <- beta M + G in place and writes ||X||_F of the
+ * Newton-Schulz input X = G + beta M (nesterov != 0) or X = M to the device
+ * double *x_norm.  For callers that cannot call cudaMalloc -- code running
+ * under global-mode stream capture, programs whose device memory is owned
+ * entirely by a framework allocator or a fixed arena, loops that must not
+ * take the driver's allocation locks -- it allocates nothing: its scratch
+ * (one fp32 partial sum per 4096-element tile) is a 256 KB array compiled
+ * into the library, held by every device that loads it until exit.
+ *   m, g   fp32 device buffers, rows x cols, row stride ld, 16-byte aligned;
+ *          m is updated in place, g is read.
+ *   limit  at most 65,536 tiles (268,435,456 elements); a larger matrix
+ *          returns MUONH_ERR_UNSUPPORTED and touches nothing.
+ * The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the one scratch array, so calls whose kernels overlap on
+ * the GPU (different streams without ordering) race; calls on one stream are
+ * ordered and safe.  Enqueued on `stream`. */
+muonh_status muonh_momentum_norm_noalloc(float* m, const float* g, int64_t rows, int64_t cols, int64_t ld,
+                                         float beta, int32_t nesterov, double* x_norm, void* stream);
+
 void muonh_destroy(muonh_ctx* ctx);
 
 const char* muonh_status_string(muonh_status s);

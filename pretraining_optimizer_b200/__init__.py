@@ -8,5 +8,5 @@ built library raises.
 from .muonh import (  # noqa: F401
     MuonH, MuonHError, QUINTIC, NS_FP16, NS_BF16, NS_FP32,
     FLAG_NONFINITE_INPUT, FLAG_ZERO_UPDATE, FLAG_NONFINITE_UPDATE, FLAG_DEGENERATE,
-    FLAG_TIMEOUT, PHASES, library, library_path, EXPORTED_SYMBOLS,
+    FLAG_TIMEOUT, PHASES, library, library_path, EXPORTED_SYMBOLS, momentum_norm_noalloc,
 )

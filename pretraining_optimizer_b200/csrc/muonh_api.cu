@@ -128,6 +128,8 @@ int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 }  // namespace
 
+void muonh::set_error_message(const char* msg) { g_last_error = msg; }
+
 struct muonh_ctx {
   int32_t n = 0;
   int32_t prec = 0;

@@ -255,6 +255,9 @@ __host__ __device__ constexpr uint32_t idesc_f16(int m, int n, int ab_bf16, int 
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// Message returned by muonh_last_error() on the calling thread.
+void set_error_message(const char* msg);
+
 // --------------------------------------------------------- launch helpers
 cudaError_t launch_ns_gemm(int mode, int prec, const NsParams& p, int grid, cudaStream_t s);
 size_t ns_gemm_smem_bytes(int prec);

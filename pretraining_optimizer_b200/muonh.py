@@ -22,7 +22,8 @@ FLAG_TIMEOUT = 16
 EXPORTED_SYMBOLS = (
     "muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
     "muonh_export_state", "muonh_import_state", "muonh_device_status", "muonh_last_launch_count",
-    "muonh_enable_timing", "muonh_phase_times", "muonh_destroy", "muonh_status_string", "muonh_last_error",
+    "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc", "muonh_destroy",
+    "muonh_status_string", "muonh_last_error",
 )
 PHASES = ("momentum_norm", "finalize_input", "write_x", "ns_gram", "ns_square", "ns_apply",
           "update_dots", "finalize_update", "project", "finalize_step")
@@ -77,6 +78,8 @@ def library() -> ctypes.CDLL:
     lib.muonh_last_launch_count.restype = c_int32
     lib.muonh_enable_timing.argtypes = [c_void_p, c_int32]
     lib.muonh_phase_times.argtypes = [c_void_p, POINTER(c_float), POINTER(c_int64)]
+    lib.muonh_momentum_norm_noalloc.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_float,
+                                                c_int32, c_void_p, c_void_p]
     lib.muonh_destroy.argtypes = [c_void_p]
     lib.muonh_destroy.restype = None
     lib.muonh_status_string.argtypes = [c_int32]
@@ -85,7 +88,7 @@ def library() -> ctypes.CDLL:
     lib.muonh_last_error.restype = c_char_p
     for name in ("muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
                  "muonh_export_state", "muonh_import_state", "muonh_device_status",
-                 "muonh_enable_timing", "muonh_phase_times"):
+                 "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc"):
         getattr(lib, name).restype = c_int32
     _LIB = lib
     return lib
@@ -112,6 +115,22 @@ def _matrix_view(t, what: str):
     if t.stride(1) != 1:
         raise ValueError(f"{what} must have unit column stride")
     return t.data_ptr(), t.shape[0], t.shape[1], max(t.stride(0), t.shape[1])
+
+
+def momentum_norm_noalloc(m, g, beta=0.95, nesterov=True, x_norm=None, stream=None):
+    """Allocation-free momentum stage for one matrix (no context, no device
+    allocation inside the library): m <- beta m + g in place; returns the
+    device fp64 tensor holding ||X||_F of the Newton-Schulz input."""
+    import torch
+    mp, rows, cols, ld = _matrix_view(m, "m")
+    gp, gr, gc, gld = _matrix_view(g, "g")
+    if (gr, gc, gld) != (rows, cols, ld):
+        raise ValueError("g must match m in shape and stride")
+    if x_norm is None:
+        x_norm = torch.empty((), dtype=torch.float64, device=m.device)
+    _check(library().muonh_momentum_norm_noalloc(mp, gp, rows, cols, ld, float(beta), int(bool(nesterov)),
+                                                 x_norm.data_ptr(), _stream_handle(stream)))
+    return x_norm
 
 
 class MuonH:
