@@ -55,6 +55,11 @@ struct Cfg {
   static constexpr int kStageBytes = kParts * (kABytes + kBBytes);
   static constexpr int kBarOffset = kStages * kStageBytes;
   static constexpr int kSmem = kBarOffset + 256 + 1024;            // + barriers + alignment slack
+  // FP32 mode: the tensor cores accumulate kChunkBlocks k-blocks (128 of K)
+  // into a scratch accumulator; the epilogue adds each chunk to the running
+  // sum in IEEE fp32 (the hardware accumulation truncates, with an error
+  // that grows with the number of accumulated products).
+  static constexpr int kChunkBlocks = 2;
 };
 
 // 32 consecutive values of one row, stored as 16-bit (and the fp16 residual in FP32 mode).
@@ -201,7 +206,68 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && PREC == P_FP32) {
+      // accumulator S (columns 0..255) holds chunk 0 and the running sum;
+      // chunks 1.. go to C (columns 256..511) and are merged by the epilogue.
+      constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, 0, MODE == M_APPLY ? 1 : 0);
+      uint64_t* cready = &tfull[0];
+      uint64_t* sdone = &tfull[1];
+      uint64_t* cfree = &tempty[0];
+      uint64_t* sfree = &tempty[1];
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0, cuse = 0;
+      for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x, ++local) {
+        const TileDesc td = p.tiles[t];
+        const MatDev& md = p.mats[td.mat];
+        const ClassDev& cd = p.classes[md.cls];
+        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
+        if (local > 0 && !mbar_wait(sfree, (local - 1) & 1, p.err)) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < nk && ok; ++kb) {
+          const int chunk = kb / C::kChunkBlocks;
+          const bool chunk_start = (kb % C::kChunkBlocks) == 0;
+          if (chunk >= 1 && chunk_start) {
+            if (cuse > 0 && !mbar_wait(cfree, (cuse - 1) & 1, p.err)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const uint32_t d_tmem = tmem_base + (chunk == 0 ? 0 : kBN);
+          if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kParts * C::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+#pragma unroll
+            for (int prod = 0; prod < 3; ++prod) {
+              const int pa = (prod == 2) ? 1 : 0;
+              const int pb = (prod == 1) ? 1 : 0;
+              const uint64_t adesc = sdesc_sw128(sa + pa * C::kABytes + k * 32, 16, 1024);
+              uint64_t bdesc;
+              if (MODE == M_APPLY)
+                bdesc = sdesc_sw128(sb + pb * C::kBBytes + k * 16 * 128, 64 * kBK * 2, 1024);
+              else
+                bdesc = sdesc_sw128(sb + pb * C::kBBytes + k * 32, 16, 1024);
+              umma_f16(d_tmem, adesc, bdesc, kIdesc, (chunk_start && k == 0 && prod == 0) ? 0u : 1u);
+            }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          const bool chunk_end = ((kb + 1) % C::kChunkBlocks) == 0 || kb + 1 == nk;
+          if (chunk >= 1 && chunk_end) {
+            umma_commit(cready);
+            ++cuse;
+          }
+        }
+        if (!ok) break;
+        umma_commit(sdone);
+      }
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+    } else if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, PREC == P_BF16 ? 1 : 0, MODE == M_APPLY ? 1 : 0);
       int stage = 0;
       uint32_t phase = 0;
@@ -256,13 +322,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int lrow = quarter * 32 + lane;    // row within the tile
     int local = 0;
+    int merges = 0;                          // FP32 mode: chunk merges so far
     for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++local) {
       const TileDesc td = p.tiles[t];
       const MatDev& md = p.mats[td.mat];
       const ClassDev& cd = p.classes[md.cls];
-      const int acc = local & 1;
-      const uint32_t acc_phase = (local >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
+      const int acc = (PREC == P_FP32) ? 0 : (local & 1);
+      if (PREC == P_FP32) {
+        // merge chunks 1.. of this tile into S, then wait for the tile's end
+        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
+        const int nchunks = (nk + C::kChunkBlocks - 1) / C::kChunkBlocks;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+        bool ok = true;
+        for (int c = 1; c < nchunks; ++c) {
+          if (!mbar_wait(&tfull[0], merges & 1, p.err)) { ok = false; break; }
+          tc_fence_after();
+          for (int g = 0; g < kBN / 32; ++g) {
+            float sv[32], cv[32];
+            tmem_ld32(lane_base + g * 32, sv);
+            tmem_ld32(lane_base + kBN + g * 32, cv);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sv[j] += cv[j];
+            tmem_st32(lane_base + g * 32, sv);
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[0]);
+          ++merges;
+        }
+        if (!ok || !mbar_wait(&tfull[1], local & 1, p.err)) break;
+      } else {
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
+      }
       tc_fence_after();
       const int row = td.bi * kBM + lrow;
       // tcgen05.ld is warp-collective: chunk skips below depend on the warp's
@@ -332,7 +423,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      mbar_arrive(&tempty[PREC == P_FP32 ? 1 : acc]);
     }
   }
 
