@@ -137,6 +137,7 @@ struct muonh_ctx {
   int device = 0;
   int sm_count = 148;
   int32_t max_steps = 0;
+  bool pairs = false;        // 16-bit operands: CTA-pair GEMMs on 256 x 256 tiles
   int64_t n_et = 0;
   int64_t step_count = 0;
   int32_t last_launches = 0;
@@ -328,6 +329,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   ctx->eps = cfg->eps;
   ctx->device = dev;
   ctx->sm_count = prop.multiProcessorCount;
+  ctx->pairs = cfg->ns_precision != P_FP32;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ctx->last_stream = s;
 
@@ -438,6 +440,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       if ((st = encode_map(&m[TM_A_K128 + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
       if ((st = encode_map(&m[TM_C_K256 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN))) return st;
       if ((st = encode_map(&m[TM_B_K128 + part], cd.b[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
+      if ((st = encode_map(&m[TM_C_K128 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
     }
   }
 
@@ -493,19 +496,21 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       if (cx.c_pad != cy.c_pad) return cx.c_pad > cy.c_pad;
       return cx.r_pad > cy.r_pad;
     });
+    // Tile rows are 128 (single-CTA kernel, FP32 mode) or 256 (CTA pairs).
+    const int tm = ctx->pairs ? 2 * kBM : kBM;
     std::vector<TileDesc> gram, apply;
     for (int32_t i : order) {
       const ClassHost& ch = ctx->classes[ctx->mats[i].cls];
-      for (int bi = 0; bi < ch.r_pad / kBM; ++bi)
+      for (int bi = 0; bi < ch.r_pad / tm; ++bi)
         for (int bj = 0; bj < ch.r_pad / kBN; ++bj)
-          if (bj * kBN + kBN - 1 >= bi * kBM) gram.push_back(TileDesc{i, int16_t(bi), int16_t(bj)});
+          if (bj * kBN + kBN - 1 >= bi * tm) gram.push_back(TileDesc{i, int16_t(bi), int16_t(bj)});
     }
     std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
       return ctx->classes[ctx->mats[x].cls].r_pad > ctx->classes[ctx->mats[y].cls].r_pad;
     });
     for (int32_t i : order) {
       const ClassHost& ch = ctx->classes[ctx->mats[i].cls];
-      for (int bi = 0; bi < ch.r_pad / kBM; ++bi)
+      for (int bi = 0; bi < ch.r_pad / tm; ++bi)
         for (int bj = 0; bj < ch.c_pad / kBN; ++bj) apply.push_back(TileDesc{i, int16_t(bi), int16_t(bj)});
     }
     TileList gl, al;
@@ -575,14 +580,26 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
     np.src = k & 1;
     np.tiles = ctx->gram_lists[k].dev;
     np.ntiles = ctx->gram_lists[k].count;
-    const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
-    STEP_LAUNCH(MUONH_PHASE_NS_GRAM, launch_ns_gemm(M_GRAM, ctx->prec, np, ggrid, s), "ns_gram");
-    STEP_LAUNCH(MUONH_PHASE_NS_SQUARE, launch_ns_gemm(M_SQUARE, ctx->prec, np, ggrid, s), "ns_square");
-    np.tiles = ctx->apply_lists[k].dev;
-    np.ntiles = ctx->apply_lists[k].count;
-    STEP_LAUNCH(MUONH_PHASE_NS_APPLY,
-                launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), s),
-                "ns_apply");
+    if (ctx->pairs) {
+      const int pairs_max = std::max(1, ctx->sm_count / 2);
+      const int gp = std::min(pairs_max, std::max(1, np.ntiles));
+      STEP_LAUNCH(MUONH_PHASE_NS_GRAM, launch_ns_gemm_pair(M_GRAM, ctx->prec, np, gp, s), "ns_gram");
+      STEP_LAUNCH(MUONH_PHASE_NS_SQUARE, launch_ns_gemm_pair(M_SQUARE, ctx->prec, np, gp, s), "ns_square");
+      np.tiles = ctx->apply_lists[k].dev;
+      np.ntiles = ctx->apply_lists[k].count;
+      STEP_LAUNCH(MUONH_PHASE_NS_APPLY,
+                  launch_ns_gemm_pair(M_APPLY, ctx->prec, np, std::min(pairs_max, std::max(1, np.ntiles)), s),
+                  "ns_apply");
+    } else {
+      const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
+      STEP_LAUNCH(MUONH_PHASE_NS_GRAM, launch_ns_gemm(M_GRAM, ctx->prec, np, ggrid, s), "ns_gram");
+      STEP_LAUNCH(MUONH_PHASE_NS_SQUARE, launch_ns_gemm(M_SQUARE, ctx->prec, np, ggrid, s), "ns_square");
+      np.tiles = ctx->apply_lists[k].dev;
+      np.ntiles = ctx->apply_lists[k].count;
+      STEP_LAUNCH(MUONH_PHASE_NS_APPLY,
+                  launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), s),
+                  "ns_apply");
+    }
   }
   STEP_LAUNCH(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, s), "update_dots");
   STEP_LAUNCH(MUONH_PHASE_FINALIZE_UPDATE, launch_finalize_update(p, s), "finalize_update");

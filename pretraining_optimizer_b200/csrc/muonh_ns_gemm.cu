@@ -433,6 +433,240 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
   if (warp == 1) tmem_dealloc(tmem_base, 512);
 }
 
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (fp16 / bf16 operands): a cluster of two CTAs on two SMs
+// computes a 256 x 256 tile with tcgen05.mma.cta_group::2.  Each CTA loads
+// its own 128 rows of the A operand and its own 128-column half of the B
+// operand (no multicast), so a pair moves a third less operand data per
+// FLOP than two single-CTA 128 x 256 tiles.  The leader CTA (rank 0) issues
+// the MMAs; both CTAs' TMA loads complete on the leader's stage barrier, and
+// the leader's commits arrive on the matching barriers of both CTAs.  Each
+// CTA drains its own TMEM (its 128 rows) in the epilogue.
+template <int PREC>
+struct PairCfg {
+  static constexpr int kStages = 6;
+  static constexpr int kABytes = 128 * kBK * 2;                 // 16 KB: this CTA's 128 rows
+  static constexpr int kBBytes = 128 * kBK * 2;                 // 16 KB: this CTA's half of N
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kSmem = kBarOffset + 256 + 1024;
+};
+constexpr int kPairM = 256;
+
+template <int MODE, int PREC>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    ns_gemm_pair_kernel(const __grid_constant__ NsParams p) {
+  using C = PairCfg<PREC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();          // 0 = leader
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);                        // leader: one expect_tx arrival per phase
+      mbar_init(&empty[s], 1);                       // one multicast commit per phase
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 128);                // both CTAs' epilogue threads
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                    // barriers initialised in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_parity[C::kStages];
+      bool issued[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) issued[s] = false;
+      bool ok = true;
+      for (int t = pair; t < p.ntiles && ok; t += npairs) {
+        const TileDesc td = p.tiles[t];
+        const MatDev& md = p.mats[td.mat];
+        const ClassDev& cd = p.classes[md.cls];
+        const int z = md.z;
+        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
+        const int arow = td.bi * kPairM + static_cast<int>(rank) * 128;   // this CTA's A rows
+        const int bcol = td.bj * kBN + static_cast<int>(rank) * 128;      // this CTA's B half
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) { ok = false; break; }
+          if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
+          const uint32_t bar = map_shared_rank(&full[stage], 0);
+          uint8_t* sa = smem + stage * C::kStageBytes;
+          uint8_t* sb = sa + C::kABytes;
+          const int k0 = kb * kBK;
+          if (MODE == M_GRAM) {
+            tma_load_3d_pair(sa, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, arow, z);
+            tma_load_3d_pair(sb, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, bcol, z);
+          } else if (MODE == M_SQUARE) {
+            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_A_K128, bar, k0, arow, z);
+            tma_load_3d_pair(sb, p.tmaps + cd.tm_base + TM_C_K128, bar, k0, bcol, z);
+          } else {
+            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_B_K128, bar, k0, arow, z);
+            const CUtensorMap* xm = p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, 0);
+            tma_load_3d_pair(sb, xm, bar, bcol, k0, z);
+            tma_load_3d_pair(sb + 64 * kBK * 2, xm, bar, bcol + 64, k0, z);
+          }
+          issued[stage] = true;
+          issued_parity[stage] = phase;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int s = 0; s < C::kStages; ++s)
+          if (issued[s]) {
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&full[s], issued_parity[s]) && globaltimer() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdesc = idesc_f16(kPairM, kBN, PREC == P_BF16 ? 1 : 0, MODE == M_APPLY ? 1 : 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int t = pair; t < p.ntiles && ok; t += npairs, ++local) {
+        const TileDesc td = p.tiles[t];
+        const MatDev& md = p.mats[td.mat];
+        const ClassDev& cd = p.classes[md.cls];
+        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kBN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t adesc = sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bdesc = (MODE == M_APPLY) ? sdesc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
+                                                     : sdesc_sw128(sb + k * 32, 16, 1024);
+            umma_f16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc]);
+      }
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int lrow = quarter * 32 + lane;
+    const uint32_t tempty_leader[2] = {map_shared_rank(&tempty[0], 0), map_shared_rank(&tempty[1], 0)};
+    int local = 0;
+    for (int t = pair; t < p.ntiles; t += npairs, ++local) {
+      const TileDesc td = p.tiles[t];
+      const MatDev& md = p.mats[td.mat];
+      const ClassDev& cd = p.classes[md.cls];
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
+      tc_fence_after();
+      const int row = td.bi * kPairM + static_cast<int>(rank) * 128 + lrow;
+      const int warp_row0 = row - lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
+      if (MODE == M_GRAM) {
+        const float sa = exp2f(static_cast<float>(md.ea - 2 * md.ex));
+        const float sc = md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
+        const float diag = md.b * exp2f(static_cast<float>(md.ec));
+        const int64_t mo = md.z * cd.a_stride * 2;
+        void* ahi = static_cast<uint8_t*>(cd.a[0]) + mo;
+        void* chi = static_cast<uint8_t*>(cd.c[0]) + mo;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int col0 = td.bj * kBN + ch * 32;
+          if (col0 + 31 < warp_row0) continue;
+          float v[32], w[32];
+          tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            w[j] = sc * v[j];
+            v[j] *= sa;
+          }
+          const int dj = row - col0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j == dj) w[j] += diag;
+          store_symmetric<PREC>(ahi, nullptr, cd.r_pad, row, col0, v);
+          store_symmetric<PREC>(chi, nullptr, cd.r_pad, row, col0, w);
+        }
+      } else if (MODE == M_SQUARE) {
+        const float sb = exp2f(static_cast<float>(md.eb - md.ea - md.ec));
+        const float diag = md.a * exp2f(static_cast<float>(md.eb));
+        void* bhi = static_cast<uint8_t*>(cd.b[0]) + md.z * cd.a_stride * 2;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int col0 = td.bj * kBN + ch * 32;
+          if (col0 + 31 < warp_row0) continue;
+          float v[32];
+          tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= sb;
+          const int dj = row - col0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j == dj) v[j] += diag;
+          store_symmetric<PREC>(bhi, nullptr, cd.r_pad, row, col0, v);
+        }
+      } else {
+        const float ks = exp2f(static_cast<float>(-md.eb));
+        void* yhi = static_cast<uint8_t*>(cd.x[p.src ^ 1][0]) + md.z * cd.x_stride * 2;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          const int col0 = td.bj * kBN + ch * 32;
+          float v[32];
+          tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= ks;
+          store_row32<PREC>(yhi, nullptr, static_cast<int64_t>(row) * cd.c_pad + col0, v);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();              // the leader's MMAs into both CTAs' TMEM have drained
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
+}
+
 }  // namespace
 
 template <int MODE, int PREC>
@@ -441,8 +675,19 @@ static cudaError_t set_attr() {
                               Cfg<PREC>::kSmem);
 }
 
+template <int MODE, int PREC>
+static cudaError_t set_pair_attr() {
+  return cudaFuncSetAttribute(ns_gemm_pair_kernel<MODE, PREC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              PairCfg<PREC>::kSmem);
+}
+
 cudaError_t ns_gemm_set_attributes() {
   cudaError_t e;
+#define MUONH_SET_PAIR(MD, PR) \
+  if ((e = set_pair_attr<MD, PR>()) != cudaSuccess) return e;
+  MUONH_SET_PAIR(M_GRAM, P_FP16) MUONH_SET_PAIR(M_SQUARE, P_FP16) MUONH_SET_PAIR(M_APPLY, P_FP16)
+  MUONH_SET_PAIR(M_GRAM, P_BF16) MUONH_SET_PAIR(M_SQUARE, P_BF16) MUONH_SET_PAIR(M_APPLY, P_BF16)
+#undef MUONH_SET_PAIR
 #define MUONH_SET(MD, PR) \
   if ((e = set_attr<MD, PR>()) != cudaSuccess) return e;
   MUONH_SET(M_GRAM, P_FP16) MUONH_SET(M_SQUARE, P_FP16) MUONH_SET(M_APPLY, P_FP16)
@@ -454,6 +699,20 @@ cudaError_t ns_gemm_set_attributes() {
 
 size_t ns_gemm_smem_bytes(int prec) {
   return prec == P_FP32 ? Cfg<P_FP32>::kSmem : Cfg<P_FP16>::kSmem;
+}
+
+cudaError_t launch_ns_gemm_pair(int mode, int prec, const NsParams& p, int pairs, cudaStream_t s) {
+  if (p.ntiles <= 0) return cudaSuccess;
+  const size_t smem = PairCfg<P_FP16>::kSmem;
+#define MUONH_LAUNCH_PAIR(MD, PR)                                                \
+  if (mode == MD && prec == PR) {                                                \
+    ns_gemm_pair_kernel<MD, PR><<<2 * pairs, kGemmThreads, smem, s>>>(p);       \
+    return cudaGetLastError();                                                   \
+  }
+  MUONH_LAUNCH_PAIR(M_GRAM, P_FP16) MUONH_LAUNCH_PAIR(M_SQUARE, P_FP16) MUONH_LAUNCH_PAIR(M_APPLY, P_FP16)
+  MUONH_LAUNCH_PAIR(M_GRAM, P_BF16) MUONH_LAUNCH_PAIR(M_SQUARE, P_BF16) MUONH_LAUNCH_PAIR(M_APPLY, P_BF16)
+#undef MUONH_LAUNCH_PAIR
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_ns_gemm(int mode, int prec, const NsParams& p, int grid, cudaStream_t s) {
