@@ -226,16 +226,17 @@ void release(muonh_ctx* ctx) {
 }
 
 muonh_status encode_map(CUtensorMap* out, void* base, int prec16_is_bf16, int64_t inner, int64_t rows,
-                        int64_t count, int box_rows) {
+                        int64_t count, int box_rows, int box_inner = 64,
+                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(count)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner * 2), static_cast<cuuint64_t>(inner * rows * 2)};
-  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(out, prec16_is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-                  base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return MUONH_OK;
@@ -435,12 +436,26 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           return st;
         if ((st = encode_map(&m[tm_x(TM_X_MN, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBK)))
           return st;
+        if (part == 0 && (st = encode_map(&m[TM_X_ST + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count, kBM, 32,
+                                          CU_TENSOR_MAP_SWIZZLE_64B)))
+          return st;
       }
       muonh_status st;
       if ((st = encode_map(&m[TM_A_K128 + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
       if ((st = encode_map(&m[TM_C_K256 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN))) return st;
       if ((st = encode_map(&m[TM_B_K128 + part], cd.b[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
       if ((st = encode_map(&m[TM_C_K128 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
+      if ((st = encode_map(&m[TM_A_MN + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBK))) return st;
+      if ((st = encode_map(&m[TM_C_MN + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBK))) return st;
+      if ((st = encode_map(&m[TM_B_MN + part], cd.b[part], bf, cd.r_pad, cd.r_pad, cd.count, kBK))) return st;
+      if (part == 0) {
+        if ((st = encode_map(&m[TM_A_ST], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+          return st;
+        if ((st = encode_map(&m[TM_C_ST], cd.c[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+          return st;
+        if ((st = encode_map(&m[TM_B_ST], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+          return st;
+      }
     }
   }
 
@@ -503,7 +518,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       const ClassHost& ch = ctx->classes[ctx->mats[i].cls];
       for (int bi = 0; bi < ch.r_pad / tm; ++bi)
         for (int bj = 0; bj < ch.r_pad / kBN; ++bj)
-          if (bj * kBN + kBN - 1 >= bi * tm) gram.push_back(TileDesc{i, int16_t(bi), int16_t(bj)});
+          if (bj * kBN + kBN - 1 >= bi * tm) gram.push_back(TileDesc{i, int16_t(bi), int16_t(bj), ch.c_pad / kBK, ch.r_pad / kBK});
     }
     std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
       return ctx->classes[ctx->mats[x].cls].r_pad > ctx->classes[ctx->mats[y].cls].r_pad;
@@ -511,7 +526,8 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
     for (int32_t i : order) {
       const ClassHost& ch = ctx->classes[ctx->mats[i].cls];
       for (int bi = 0; bi < ch.r_pad / tm; ++bi)
-        for (int bj = 0; bj < ch.c_pad / kBN; ++bj) apply.push_back(TileDesc{i, int16_t(bi), int16_t(bj)});
+        for (int bj = 0; bj < ch.c_pad / kBN; ++bj)
+          apply.push_back(TileDesc{i, int16_t(bi), int16_t(bj), ch.r_pad / kBK, ch.r_pad / kBK});
     }
     TileList gl, al;
     gl.count = static_cast<int32_t>(gram.size());

@@ -36,7 +36,14 @@ enum TmSlot {
   TM_C_K256 = 14,  // C = b I + c A, 256-row box (+part)
   TM_B_K128 = 16,  // B' = a I + A C, 128-row box (+part)
   TM_C_K128 = 18,  // C, 128-row box (+part): B operand half of a CTA pair
-  TM_PER_CLASS = 20
+  TM_A_MN = 20,    // A, 64 x 64 box: a below-diagonal block read through its stored transpose
+  TM_C_MN = 22,    // C, 64 x 64 box
+  TM_B_MN = 24,    // B', 64 x 64 box
+  TM_X_ST = 26,    // X[buf] store box 32 x 128 (64-byte swizzle)   (+buf)
+  TM_A_ST = 28,    // A store box
+  TM_C_ST = 29,    // C store box
+  TM_B_ST = 30,    // B' store box
+  TM_PER_CLASS = 32
 };
 __host__ __device__ inline int tm_x(int base, int buf, int part) { return base + buf + 2 * part; }
 
@@ -86,6 +93,8 @@ struct MatScal {             // device-resident per-matrix scalars
 struct TileDesc {
   int32_t mat;
   int16_t bi, bj;
+  int32_t nk;                // k-blocks of 64 along K: GRAM (c_pad/64) or APPLY (r_pad/64)
+  int32_t nk_sq;             // SQUARE k-blocks (r_pad/64) for GRAM-list tiles
 };
 
 struct NsParams {
@@ -178,6 +187,24 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// TMA store of a shared-memory box into a tiled tensor (bulk-group completion).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Make generic-proxy shared-memory writes visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

@@ -443,6 +443,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 // the MMAs; both CTAs' TMA loads complete on the leader's stage barrier, and
 // the leader's commits arrive on the matching barriers of both CTAs.  Each
 // CTA drains its own TMEM (its 128 rows) in the epilogue.
+//
+// Symmetric results (A, C, B') are stored as whole 256 x 256 tiles of the
+// upper block triangle only.  A consumer that needs a block below the
+// diagonal loads the stored transposed block and hands it to the MMA as an
+// MN-major operand, so no epilogue writes a mirrored copy.
 template <int PREC>
 struct PairCfg {
   static constexpr int kStages = 6;
@@ -450,8 +455,55 @@ struct PairCfg {
   static constexpr int kBBytes = 128 * kBK * 2;                 // 16 KB: this CTA's half of N
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = kStages * kStageBytes;
-  static constexpr int kSmem = kBarOffset + 256 + 1024;
+  // SQUARE epilogue: per-warp 32 x 32 16-bit staging block for the mirrored
+  // copy of B' (rows padded to 80 bytes: conflict-free 16-byte stores and
+  // 2-byte column reads)
+  static constexpr int kMirrorStride = 80;
+  static constexpr int kMirrorOffset = kBarOffset + 256;
+  static constexpr int kMirrorBytes = 4 * 32 * kMirrorStride;
+  // Epilogue output staging: two 128-row x 32-column 16-bit boxes written
+  // to global memory by TMA stores (64-byte swizzle)
+  static constexpr int kStoreBox = 128 * 32 * 2;
+  static constexpr int kStoreOffset = (kMirrorOffset + kMirrorBytes + 1023) / 1024 * 1024;
+  static constexpr int kSmem = kStoreOffset + 2 * kStoreBox + 1024;
 };
+
+// Epilogue row `r` (0..127) of a 128 x 32 16-bit box, 16-byte piece q,
+// in the 64-byte swizzle pattern of the TMA store box.
+__device__ __forceinline__ uint32_t store_box_offset(int r, int q) {
+  return static_cast<uint32_t>(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+}
+
+// Double-buffered TMA-store staging shared by the 128 epilogue threads.
+struct StoreStager {
+  uint8_t* base;
+  int count;   // boxes issued so far by this CTA
+  __device__ __forceinline__ void put(const CUtensorMap* map, int lrow, const uint4 (&packed)[4], int x, int y,
+                                      int z) {
+    uint8_t* buf = base + (count & 1) * (128 * 32 * 2);
+    if (count >= 2) {
+      if (threadIdx.x == 64) bulk_wait_read<1>();   // the box issued two stores ago has been read
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + store_box_offset(lrow, q)) = packed[q];
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (threadIdx.x == 64) {
+      tma_store_3d(map, buf, x, y, z);
+      bulk_commit();
+    }
+    ++count;
+  }
+};
+
+template <int PREC>
+__device__ __forceinline__ void pack32(const float (&v)[32], uint4 (&packed)[4]) {
+  using T = typename Store16<PREC>::T;
+  T* h = reinterpret_cast<T*>(packed);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) h[j] = Store16<PREC>::cvt(v[j]);
+}
 constexpr int kPairM = 256;
 
 template <int MODE, int PREC>
@@ -506,9 +558,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const MatDev& md = p.mats[td.mat];
         const ClassDev& cd = p.classes[md.cls];
         const int z = md.z;
-        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
-        const int arow = td.bi * kPairM + static_cast<int>(rank) * 128;   // this CTA's A rows
-        const int bcol = td.bj * kBN + static_cast<int>(rank) * 128;      // this CTA's B half
+        const int nk = (MODE == M_SQUARE) ? td.nk_sq : td.nk;
+        const int abase = td.bi * kPairM, bbase = td.bj * kBN;                // tile origin
+        const int arow = abase + static_cast<int>(rank) * 128;              // this CTA's A rows
+        const int bcol = bbase + static_cast<int>(rank) * 128;              // this CTA's B half
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
@@ -516,17 +569,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           const int k0 = kb * kBK;
+          constexpr int kHalf = 64 * kBK * 2;   // one 64-wide MN-major chunk
           if (MODE == M_GRAM) {
             tma_load_3d_pair(sa, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, arow, z);
             tma_load_3d_pair(sb, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, bcol, z);
-          } else if (MODE == M_SQUARE) {
-            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_A_K128, bar, k0, arow, z);
-            tma_load_3d_pair(sb, p.tmaps + cd.tm_base + TM_C_K128, bar, k0, bcol, z);
           } else {
-            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_B_K128, bar, k0, arow, z);
-            const CUtensorMap* xm = p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, 0);
-            tma_load_3d_pair(sb, xm, bar, bcol, k0, z);
-            tma_load_3d_pair(sb + 64 * kBK * 2, xm, bar, bcol + 64, k0, z);
+            // A operand: rows of the symmetric A (SQUARE: upper blocks only,
+            // lower blocks through their stored transpose) or of B' (APPLY:
+            // stored with its mirror, always K-major)
+            if (MODE == M_APPLY || k0 >= abase) {
+              tma_load_3d_pair(sa, p.tmaps + cd.tm_base + (MODE == M_SQUARE ? TM_A_K128 : TM_B_K128), bar, k0,
+                               arow, z);
+            } else {
+              tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_A_MN, bar, arow, k0, z);
+              tma_load_3d_pair(sa + kHalf, p.tmaps + cd.tm_base + TM_A_MN, bar, arow + 64, k0, z);
+            }
+            if (MODE == M_SQUARE && k0 >= bbase) {
+              tma_load_3d_pair(sb, p.tmaps + cd.tm_base + TM_C_K128, bar, k0, bcol, z);
+            } else {
+              const CUtensorMap* bm = (MODE == M_SQUARE) ? p.tmaps + cd.tm_base + TM_C_MN
+                                                         : p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, 0);
+              tma_load_3d_pair(sb, bm, bar, bcol, k0, z);
+              tma_load_3d_pair(sb + kHalf, bm, bar, bcol + 64, k0, z);
+            }
           }
           issued[stage] = true;
           issued_parity[stage] = phase;
@@ -546,38 +611,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t kIdesc = idesc_f16(kPairM, kBN, PREC == P_BF16 ? 1 : 0, MODE == M_APPLY ? 1 : 0);
+      constexpr uint32_t kIdescKK = idesc_f16(kPairM, kBN, PREC == P_BF16 ? 1 : 0, 0);
+      constexpr uint32_t kAMn = 1u << 15;   // A operand MN-major
+      constexpr uint32_t kBMn = 1u << 16;   // B operand MN-major
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int local = 0;
+      TileDesc td = pair < p.ntiles ? p.tiles[pair] : TileDesc{};
       for (int t = pair; t < p.ntiles && ok; t += npairs, ++local) {
-        const TileDesc td = p.tiles[t];
-        const MatDev& md = p.mats[td.mat];
-        const ClassDev& cd = p.classes[md.cls];
-        const int nk = (MODE == M_GRAM ? cd.c_pad : cd.r_pad) / kBK;
+        const TileDesc next = (t + npairs < p.ntiles) ? p.tiles[t + npairs] : td;   // prefetch
+        const int nk = (MODE == M_SQUARE) ? td.nk_sq : td.nk;
+        const int abase = td.bi * kPairM, bbase = td.bj * kBN;
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
         for (int kb = 0; kb < nk; ++kb) {
+          const int k0 = kb * kBK;
+          const bool a_mn = (MODE == M_SQUARE) && k0 < abase;
+          const bool b_mn = (MODE == M_APPLY) || (MODE == M_SQUARE && k0 < bbase);
+          const uint32_t idesc = kIdescKK | (a_mn ? kAMn : 0u) | (b_mn ? kBMn : 0u);
           if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t sb = sa + C::kABytes;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t adesc = sdesc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t bdesc = (MODE == M_APPLY) ? sdesc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
-                                                     : sdesc_sw128(sb + k * 32, 16, 1024);
-            umma_f16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | k) != 0 ? 1u : 0u);
+            const uint64_t adesc = a_mn ? sdesc_sw128(sa + k * 16 * 128, 64 * kBK * 2, 1024)
+                                        : sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bdesc = b_mn ? sdesc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
+                                        : sdesc_sw128(sb + k * 32, 16, 1024);
+            umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit_pair(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         umma_commit_pair(&tfull[acc]);
+        td = next;
       }
       umma_commit(drain);
       const uint64_t t0 = globaltimer();
@@ -590,6 +663,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int quarter = warp & 3;
     const int lrow = quarter * 32 + lane;
     const uint32_t tempty_leader[2] = {map_shared_rank(&tempty[0], 0), map_shared_rank(&tempty[1], 0)};
+    StoreStager stager{smem + C::kStoreOffset, 0};
     int local = 0;
     for (int t = pair; t < p.ntiles; t += npairs, ++local) {
       const TileDesc td = p.tiles[t];
@@ -599,21 +673,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
       tc_fence_after();
-      const int row = td.bi * kPairM + static_cast<int>(rank) * 128 + lrow;
-      const int warp_row0 = row - lane;
+      const int row0 = td.bi * kPairM + static_cast<int>(rank) * 128;   // this CTA's first row
+      const int row = row0 + lrow;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       if (MODE == M_GRAM) {
         const float sa = exp2f(static_cast<float>(md.ea - 2 * md.ex));
         const float sc = md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
         const float diag = md.b * exp2f(static_cast<float>(md.ec));
-        const int64_t mo = md.z * cd.a_stride * 2;
-        void* ahi = static_cast<uint8_t*>(cd.a[0]) + mo;
-        void* chi = static_cast<uint8_t*>(cd.c[0]) + mo;
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
-          if (col0 + 31 < warp_row0) continue;
           float v[32], w[32];
           tmem_ld32(taddr + ch * 32, v);
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive_cluster(tempty_leader[acc]);   // accumulator drained
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             w[j] = sc * v[j];
@@ -623,41 +697,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (j == dj) w[j] += diag;
-          store_symmetric<PREC>(ahi, nullptr, cd.r_pad, row, col0, v);
-          store_symmetric<PREC>(chi, nullptr, cd.r_pad, row, col0, w);
+          uint4 pv[4], pw[4];
+          pack32<PREC>(v, pv);
+          pack32<PREC>(w, pw);
+          stager.put(p.tmaps + cd.tm_base + TM_A_ST, lrow, pv, col0, row0, md.z);
+          stager.put(p.tmaps + cd.tm_base + TM_C_ST, lrow, pw, col0, row0, md.z);
         }
       } else if (MODE == M_SQUARE) {
         const float sb = exp2f(static_cast<float>(md.eb - md.ea - md.ec));
         const float diag = md.a * exp2f(static_cast<float>(md.eb));
-        void* bhi = static_cast<uint8_t*>(cd.b[0]) + md.z * cd.a_stride * 2;
+        using T16 = typename Store16<PREC>::T;
+        T16* bhi = reinterpret_cast<T16*>(static_cast<uint8_t*>(cd.b[0]) + md.z * cd.a_stride * 2);
+        uint8_t* mirror_buf = smem + C::kMirrorOffset + quarter * 32 * C::kMirrorStride;
+        const bool mirror = td.bj > td.bi;   // off-diagonal block: also store B'[col][row]
+        const int warp_row0 = row - lane;
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
-          if (col0 + 31 < warp_row0) continue;
           float v[32];
           tmem_ld32(taddr + ch * 32, v);
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive_cluster(tempty_leader[acc]);
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] *= sb;
           const int dj = row - col0;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (j == dj) v[j] += diag;
-          store_symmetric<PREC>(bhi, nullptr, cd.r_pad, row, col0, v);
+          uint4 packed[4];
+          pack32<PREC>(v, packed);
+          stager.put(p.tmaps + cd.tm_base + TM_B_ST, lrow, packed, col0, row0, md.z);
+          if (mirror) {
+            // transpose the warp's 32 x 32 block through shared memory
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(mirror_buf + lane * C::kMirrorStride + q * 16) = packed[q];
+            __syncwarp();
+            uint4 colv[4];
+            T16* cv = reinterpret_cast<T16*>(colv);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              cv[i] = *reinterpret_cast<const T16*>(mirror_buf + i * C::kMirrorStride + lane * 2);
+            uint4* mdst = reinterpret_cast<uint4*>(bhi + static_cast<int64_t>(col0 + lane) * cd.r_pad + warp_row0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) mdst[q] = colv[q];
+            __syncwarp();
+          }
         }
       } else {
         const float ks = exp2f(static_cast<float>(-md.eb));
-        void* yhi = static_cast<uint8_t*>(cd.x[p.src ^ 1][0]) + md.z * cd.x_stride * 2;
+        const CUtensorMap* ymap = p.tmaps + cd.tm_base + TM_X_ST + (p.src ^ 1);
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
           float v[32];
           tmem_ld32(taddr + ch * 32, v);
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive_cluster(tempty_leader[acc]);
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] *= ks;
-          store_row32<PREC>(yhi, nullptr, static_cast<int64_t>(row) * cd.c_pad + col0, v);
+          uint4 packed[4];
+          pack32<PREC>(v, packed);
+          stager.put(ymap, lrow, packed, col0, row0, md.z);
         }
       }
-      tc_fence_before();
-      mbar_arrive_cluster(tempty_leader[acc]);
     }
+    if (threadIdx.x == 64) bulk_wait_all();   // every TMA store has completed
   }
 
   tc_fence_before();
