@@ -143,7 +143,8 @@ muonh_status muonh_get_update(muonh_ctx* ctx, int32_t i, float* dst, int64_t ld,
 /* Host copy of the n radii R. */
 muonh_status muonh_get_radius(const muonh_ctx* ctx, float* host_R);
 
-/* Checkpointing of the library-held state (R[], ||W_t||^2[], step count).
+/* Checkpointing of the library-held state (R[], ||W_t||^2[], the scale the
+ * next step writes the Newton-Schulz input with, and the step count).
  * W and M are caller-owned and saved by the caller.  With buf == NULL,
  * *len receives the size needed.  Export synchronises the last stream. */
 muonh_status muonh_export_state(muonh_ctx* ctx, void* buf, size_t* len);

@@ -594,6 +594,8 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
     np.tmaps = ctx->d_tmaps;
     np.err = ctx->d_err;
     np.src = k & 1;
+    np.iter = k;
+    np.scal = ctx->d_scal;
     np.tiles = ctx->gram_lists[k].dev;
     np.ntiles = ctx->gram_lists[k].count;
     if (ctx->pairs) {
@@ -660,7 +662,7 @@ muonh_status muonh_get_radius(const muonh_ctx* ctx, float* host_R) {
 muonh_status muonh_export_state(muonh_ctx* ctx, void* buf, size_t* len) {
   g_last_error.clear();
   if (!ctx || !len) return fail(MUONH_ERR_INVALID_ARG, "ctx or len is NULL");
-  const size_t need = 16 + static_cast<size_t>(ctx->n) * (sizeof(float) + sizeof(double));
+  const size_t need = 16 + static_cast<size_t>(ctx->n) * (2 * sizeof(float) + sizeof(double));
   if (!buf) {
     *len = need;
     return MUONH_OK;
@@ -677,7 +679,8 @@ muonh_status muonh_export_state(muonh_ctx* ctx, void* buf, size_t* len) {
   for (int32_t i = 0; i < ctx->n; ++i) {
     std::memcpy(o, &scal[i].R, sizeof(float));
     std::memcpy(o + sizeof(float), &scal[i].wnorm2, sizeof(double));
-    o += sizeof(float) + sizeof(double);
+    std::memcpy(o + sizeof(float) + sizeof(double), &scal[i].sigma, sizeof(float));
+    o += 2 * sizeof(float) + sizeof(double);
   }
   *len = need;
   return MUONH_OK;
@@ -686,7 +689,7 @@ muonh_status muonh_export_state(muonh_ctx* ctx, void* buf, size_t* len) {
 muonh_status muonh_import_state(muonh_ctx* ctx, const void* buf, size_t len) {
   g_last_error.clear();
   if (!ctx || !buf) return fail(MUONH_ERR_INVALID_ARG, "ctx or buf is NULL");
-  const size_t need = 16 + static_cast<size_t>(ctx->n) * (sizeof(float) + sizeof(double));
+  const size_t need = 16 + static_cast<size_t>(ctx->n) * (2 * sizeof(float) + sizeof(double));
   if (len != need) return fail(MUONH_ERR_INVALID_ARG, "state of %zu bytes, %zu expected", len, need);
   const uint8_t* in = static_cast<const uint8_t*>(buf);
   uint32_t hdr[2];
@@ -702,7 +705,8 @@ muonh_status muonh_import_state(muonh_ctx* ctx, const void* buf, size_t len) {
   for (int32_t i = 0; i < ctx->n; ++i) {
     std::memcpy(&scal[i].R, in, sizeof(float));
     std::memcpy(&scal[i].wnorm2, in + sizeof(float), sizeof(double));
-    in += sizeof(float) + sizeof(double);
+    std::memcpy(&scal[i].sigma, in + sizeof(float) + sizeof(double), sizeof(float));
+    in += 2 * sizeof(float) + sizeof(double);
   }
   CUDA_TRY(cudaMemcpy(ctx->d_scal, scal.data(), ctx->n * sizeof(MatScal), cudaMemcpyHostToDevice));
   ctx->step_count = steps;

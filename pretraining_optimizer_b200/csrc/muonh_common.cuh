@@ -82,7 +82,10 @@ struct MatStep {             // per step, copied from the host
 
 struct MatScal {             // device-resident per-matrix scalars
   float R;
-  float xscale;              // 2^ex / (||X|| + eps)
+  float xscale;              // 2^ex / (||X|| + eps): scale of the rewrite pass
+  float sigma;               // scale the momentum kernel applies when it writes X (0: it does not)
+  float kappa;               // first-iteration correction: stored X times kappa = 2^ex X / (||X|| + eps)
+  int32_t rewrite;           // 1: write_x rewrites X at the ideal scale this step
   float kw, ko;              // projection: W <- kw W + ko O_stored
   int32_t mode;              // 0 step, 1 re-project only, 2 keep W
   uint32_t flags;
@@ -101,6 +104,8 @@ struct NsParams {
   const TileDesc* tiles;
   int32_t ntiles;
   int32_t src;               // X buffer read by this phase
+  int32_t iter;              // Newton-Schulz iteration of this launch (0: apply kappa)
+  const MatScal* scal;
   const MatDev* mats;
   const ClassDev* classes;
   const CUtensorMap* tmaps;

@@ -55,16 +55,35 @@ __device__ __forceinline__ float4 load4(const float* base, const MatDev& md, int
   return v;
 }
 
-__device__ __forceinline__ void store4(float* base, const MatDev& md, int64_t row, int64_t col, float4 v) {
-  if (row >= md.rows) return;
-  float* dst = base + row * md.ld + col;
+// Tile-relative variants: base points at the tile's first element, (r, c)
+// are tile coordinates, rows_left/cols_left bound the matrix.
+__device__ __forceinline__ float4 load4_rel(const float* base, const MatDev& md, int r, int c, int64_t rows_left,
+                                            int64_t cols_left) {
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (r >= rows_left) return v;
+  const float* src = base + r * md.ld + c;
   if (md.vec) {
-    if (col < md.cols) *reinterpret_cast<float4*>(dst) = v;
+    if (c < cols_left) v = *reinterpret_cast<const float4*>(src);
   } else {
-    if (col + 0 < md.cols) dst[0] = v.x;
-    if (col + 1 < md.cols) dst[1] = v.y;
-    if (col + 2 < md.cols) dst[2] = v.z;
-    if (col + 3 < md.cols) dst[3] = v.w;
+    if (c + 0 < cols_left) v.x = src[0];
+    if (c + 1 < cols_left) v.y = src[1];
+    if (c + 2 < cols_left) v.z = src[2];
+    if (c + 3 < cols_left) v.w = src[3];
+  }
+  return v;
+}
+
+__device__ __forceinline__ void store4_rel(float* base, const MatDev& md, int r, int c, int64_t rows_left,
+                                           int64_t cols_left, float4 v) {
+  if (r >= rows_left) return;
+  float* dst = base + r * md.ld + c;
+  if (md.vec) {
+    if (c < cols_left) *reinterpret_cast<float4*>(dst) = v;
+  } else {
+    if (c + 0 < cols_left) dst[0] = v.x;
+    if (c + 1 < cols_left) dst[1] = v.y;
+    if (c + 2 < cols_left) dst[2] = v.z;
+    if (c + 3 < cols_left) dst[3] = v.w;
   }
 }
 
@@ -185,6 +204,42 @@ __device__ __forceinline__ float4 o_at(const XView& xv, const MatDev& md, const 
   return make_float4(tile[r][c], tile[r][c + 1], tile[r][c + 2], tile[r][c + 3]);
 }
 
+// X[off .. off+3] = scale * (x, y, z, w) in the 16-bit storage (off multiple of 4).
+__device__ __forceinline__ void put4(const XView& xv, int64_t off, float4 x, float scale, int prec) {
+  if (prec == P_FP16) {
+    __half2 h01 = __floats2half2_rn(x.x * scale, x.y * scale);
+    __half2 h23 = __floats2half2_rn(x.z * scale, x.w * scale);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&h01);
+    u.y = *reinterpret_cast<uint32_t*>(&h23);
+    *reinterpret_cast<uint2*>(static_cast<__half*>(xv.hi) + off) = u;
+  } else {
+    put16(xv.hi, xv.lo, off + 0, x.x * scale, prec);
+    put16(xv.hi, xv.lo, off + 1, x.y * scale, prec);
+    put16(xv.hi, xv.lo, off + 2, x.z * scale, prec);
+    put16(xv.hi, xv.lo, off + 3, x.w * scale, prec);
+  }
+}
+
+// X[c0 + q][r0 + p] = tile[p][q] for a tall matrix's 64 x 64 tile.
+__device__ __forceinline__ void store_x_tile_t(const XView& xv, const TileCoord& tc, int prec,
+                                               float (*tile)[kEwTile + 1]) {
+  const int q = threadIdx.x / 4, p0 = (threadIdx.x % 4) * 16;
+  const int64_t off = (tc.c0 + q) * xv.ld + tc.r0 + p0;
+  if (prec == P_FP16) {
+    uint4 u[2];
+    __half* h = reinterpret_cast<__half*>(u);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) h[i] = __float2half_rn(tile[p0 + i][q]);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(xv.hi) + off);
+    dst[0] = u[0];
+    dst[1] = u[1];
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) put16(xv.hi, xv.lo, off + i, tile[p0 + i][q], prec);
+  }
+}
+
 // ------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kEwThreads) init_norm_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
@@ -201,44 +256,102 @@ __global__ void __launch_bounds__(kEwThreads) init_norm_kernel(const EwParams p)
   }
 }
 
-// M <- beta M + G; X = G + beta M (Nesterov) or M; partial ||X||^2.
-__global__ void __launch_bounds__(kEwThreads) momentum_norm_kernel(const EwParams p) {
-  __shared__ float red[kEwThreads / 32];
-  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
-    const TileCoord tc = tile_coord(p, e);
-    const MatDev& md = p.mats[tc.mi];
-    const float* g = p.step[tc.mi].g;
-    const float beta = md.beta;
-    constexpr int J = kPasses;
-    float4 gv[J], mv[J];
-    // issue every load of the tile before the first store
+// Loads and stores of one thread's 4 consecutive elements at tile coordinates
+// (r, c); FULL tiles (whole tile inside the matrix, vector path) skip every
+// bounds check and use 32-bit offsets from the tile origin.
+template <bool FULL>
+__device__ __forceinline__ float4 tile_ld(const float* base, const MatDev& md, int r, int c, int64_t rows_left,
+                                          int64_t cols_left) {
+  if (FULL) return *reinterpret_cast<const float4*>(base + (r * static_cast<int>(md.ld) + c));
+  return load4_rel(base, md, r, c, rows_left, cols_left);
+}
+template <bool FULL>
+__device__ __forceinline__ void tile_st(float* base, const MatDev& md, int r, int c, int64_t rows_left,
+                                        int64_t cols_left, float4 v) {
+  if (FULL) {
+    *reinterpret_cast<float4*>(base + (r * static_cast<int>(md.ld) + c)) = v;
+    return;
+  }
+  store4_rel(base, md, r, c, rows_left, cols_left, v);
+}
+
+__device__ __forceinline__ bool tile_is_full(const MatDev& md, const TileCoord& tc) {
+  return md.vec && tc.r0 + md.et_th <= md.rows && tc.c0 + md.et_tw <= md.cols;
+}
+
+template <bool FULL>
+__device__ __forceinline__ float momentum_tile(const EwParams& p, const MatDev& md, const TileCoord& tc,
+                                               const float* g, float sigma, const XView& xv,
+                                               float (*tile)[kEwTile + 1]) {
+  const float beta = md.beta;
+  const float* gb = g + tc.r0 * md.ld + tc.c0;
+  float* mb = md.m + tc.r0 * md.ld + tc.c0;
+  const int64_t rows_left = md.rows - tc.r0, cols_left = md.cols - tc.c0;
+  float acc = 0.f;
+  // two passes at a time: both loads of each pass issued before its store
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int64_t row = tc.r0 + tc.rin + tc.rstep * j, col = tc.c0 + tc.cin;
-      gv[j] = load4(g, md, row, col);
-      mv[j] = load4(md.m, md, row, col);
+  for (int j0 = 0; j0 < kPasses; j0 += 2) {
+    float4 gv[2], mv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = tc.rin + tc.rstep * (j0 + u);
+      gv[u] = tile_ld<FULL>(gb, md, r, tc.cin, rows_left, cols_left);
+      mv[u] = tile_ld<FULL>(mb, md, r, tc.cin, rows_left, cols_left);
     }
-    float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int64_t row = tc.r0 + tc.rin + tc.rstep * j, col = tc.c0 + tc.cin;
-      float4 m = mv[j];
-      m.x = fmaf(beta, m.x, gv[j].x);
-      m.y = fmaf(beta, m.y, gv[j].y);
-      m.z = fmaf(beta, m.z, gv[j].z);
-      m.w = fmaf(beta, m.w, gv[j].w);
-      store4(md.m, md, row, col, m);
+    for (int u = 0; u < 2; ++u) {
+      const int r = tc.rin + tc.rstep * (j0 + u);
+      float4 m = mv[u];
+      m.x = fmaf(beta, m.x, gv[u].x);
+      m.y = fmaf(beta, m.y, gv[u].y);
+      m.z = fmaf(beta, m.z, gv[u].z);
+      m.w = fmaf(beta, m.w, gv[u].w);
+      tile_st<FULL>(mb, md, r, tc.cin, rows_left, cols_left, m);
       float4 x = m;
       if (md.nesterov) {
-        x.x = fmaf(beta, m.x, gv[j].x);
-        x.y = fmaf(beta, m.y, gv[j].y);
-        x.z = fmaf(beta, m.z, gv[j].z);
-        x.w = fmaf(beta, m.w, gv[j].w);
+        x.x = fmaf(beta, m.x, gv[u].x);
+        x.y = fmaf(beta, m.y, gv[u].y);
+        x.z = fmaf(beta, m.z, gv[u].z);
+        x.w = fmaf(beta, m.w, gv[u].w);
       }
       acc = fmaf(x.x, x.x, acc);
       acc = fmaf(x.y, x.y, acc);
       acc = fmaf(x.z, x.z, acc);
       acc = fmaf(x.w, x.w, acc);
+      if (sigma > 0.f) {
+        if (!md.transposed) {
+          const int64_t col = tc.c0 + tc.cin;
+          if (FULL || col < xv.ld) put4(xv, (tc.r0 + r) * xv.ld + col, x, sigma, p.prec);
+        } else {
+          tile[r][tc.cin + 0] = x.x * sigma;
+          tile[r][tc.cin + 1] = x.y * sigma;
+          tile[r][tc.cin + 2] = x.z * sigma;
+          tile[r][tc.cin + 3] = x.w * sigma;
+        }
+      }
+    }
+  }
+  return acc;
+}
+
+// M <- beta M + G; X = G + beta M (Nesterov) or M; partial ||X||^2.  When
+// sigma > 0 it also writes the 16-bit Newton-Schulz input sigma * X (wide
+// orientation; tall matrices through a transposed shared-memory tile).
+__global__ void __launch_bounds__(kEwThreads, 5) momentum_norm_kernel(const EwParams p) {
+  __shared__ float red[kEwThreads / 32];
+  __shared__ float tile[kEwTile][kEwTile + 1];
+  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+    const TileCoord tc = tile_coord(p, e);
+    const MatDev& md = p.mats[tc.mi];
+    const float* g = p.step[tc.mi].g;
+    const float sigma = p.scal[tc.mi].sigma;
+    const XView xv = x_view(p, md, 0);
+    if (sigma > 0.f && md.transposed) __syncthreads();   // previous tile's readers are done with `tile`
+    const float acc = tile_is_full(md, tc) ? momentum_tile<true>(p, md, tc, g, sigma, xv, tile)
+                                           : momentum_tile<false>(p, md, tc, g, sigma, xv, tile);
+    if (sigma > 0.f && md.transposed) {
+      __syncthreads();
+      store_x_tile_t(xv, tc, p.prec, tile);
     }
     const float s = block_sum(acc, red);
     if (threadIdx.x == 0) p.part[e] = s;
@@ -246,9 +359,18 @@ __global__ void __launch_bounds__(kEwThreads) momentum_norm_kernel(const EwParam
 }
 
 // X_stored = xscale * X into NS buffer 0 (wide orientation, transposed for tall W).
-__global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
+__global__ void __launch_bounds__(kEwThreads, 6) write_x_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+    const int mi = p.et_mat[e];
+    if (!p.scal[mi].rewrite) {
+      // the momentum kernel already wrote this matrix's X: jump past its tiles
+      const MatDev& ms = p.mats[mi];
+      const int64_t end = ms.et_begin + static_cast<int64_t>(ms.et_rows) * ms.et_cols;
+      const int64_t skip = (end - e + gridDim.x - 1) / gridDim.x - 1;
+      e += skip * gridDim.x;
+      continue;
+    }
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     const float* g = p.step[tc.mi].g;
@@ -326,7 +448,7 @@ __global__ void __launch_bounds__(kEwThreads) write_x_kernel(const EwParams p) {
 }
 
 // Partial ||O||^2 and <W, O> (O at its stored scale).
-__global__ void __launch_bounds__(kEwThreads) update_dots_kernel(const EwParams p) {
+__global__ void __launch_bounds__(kEwThreads, 8) update_dots_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   __shared__ float red[kEwThreads / 32];
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
@@ -356,8 +478,44 @@ __global__ void __launch_bounds__(kEwThreads) update_dots_kernel(const EwParams 
   }
 }
 
+template <bool FULL>
+__device__ __forceinline__ float project_tile(const EwParams& p, const MatDev& md, const TileCoord& tc, int mode,
+                                              float kw, float ko, const XView& xv, float (*tile)[kEwTile + 1]) {
+  float* wb = md.w + tc.r0 * md.ld + tc.c0;
+  const int64_t rows_left = md.rows - tc.r0, cols_left = md.cols - tc.c0;
+  float acc = 0.f;
+#pragma unroll
+  for (int j0 = 0; j0 < kPasses; j0 += 2) {
+    float4 wv[2], ov[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = tc.rin + tc.rstep * (j0 + u);
+      wv[u] = tile_ld<FULL>(wb, md, r, tc.cin, rows_left, cols_left);
+      if (mode != 0)
+        ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      else if (FULL && !md.transposed)
+        ov[u] = x4(xv, (tc.r0 + r) * xv.ld + tc.c0 + tc.cin, p.prec);
+      else
+        ov[u] = o_at(xv, md, tc, r, tc.cin, p.prec, tile);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = tc.rin + tc.rstep * (j0 + u);
+      float4 w = wv[u];
+      const float4 o = ov[u];
+      w.x = fmaf(ko, o.x, kw * w.x);
+      w.y = fmaf(ko, o.y, kw * w.y);
+      w.z = fmaf(ko, o.z, kw * w.z);
+      w.w = fmaf(ko, o.w, kw * w.w);
+      tile_st<FULL>(wb, md, r, tc.cin, rows_left, cols_left, w);
+      acc = fmaf(w.x, w.x, fmaf(w.y, w.y, fmaf(w.z, w.z, fmaf(w.w, w.w, acc))));
+    }
+  }
+  return acc;
+}
+
 // W <- kw W + ko O (Eq. (1) with both normalisations folded into kw, ko).
-__global__ void __launch_bounds__(kEwThreads) project_kernel(const EwParams p) {
+__global__ void __launch_bounds__(kEwThreads, 6) project_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   __shared__ float red[kEwThreads / 32];
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
@@ -376,26 +534,8 @@ __global__ void __launch_bounds__(kEwThreads) project_kernel(const EwParams p) {
       load_o_tile_t(xv, tc, p.prec, tile);
       __syncthreads();
     }
-    float4 wv[kPasses], ov[kPasses];
-#pragma unroll
-    for (int j = 0; j < kPasses; ++j) {
-      const int r = tc.rin + tc.rstep * j;
-      wv[j] = load4(md.w, md, tc.r0 + r, tc.c0 + tc.cin);
-      ov[j] = mode == 0 ? o_at(xv, md, tc, r, tc.cin, p.prec, tile) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float acc = 0.f;
-#pragma unroll
-    for (int j = 0; j < kPasses; ++j) {
-      const int r = tc.rin + tc.rstep * j;
-      float4 w = wv[j];
-      const float4 o = ov[j];
-      w.x = fmaf(ko, o.x, kw * w.x);
-      w.y = fmaf(ko, o.y, kw * w.y);
-      w.z = fmaf(ko, o.z, kw * w.z);
-      w.w = fmaf(ko, o.w, kw * w.w);
-      store4(md.w, md, tc.r0 + r, tc.c0 + tc.cin, w);
-      acc = fmaf(w.x, w.x, fmaf(w.y, w.y, fmaf(w.z, w.z, fmaf(w.w, w.w, acc))));
-    }
+    const float acc = tile_is_full(md, tc) ? project_tile<true>(p, md, tc, mode, kw, ko, xv, tile)
+                                           : project_tile<false>(p, md, tc, mode, kw, ko, xv, tile);
     const float s = block_sum(acc, red);
     if (threadIdx.x == 0) p.part[e] = s;
   }
@@ -461,15 +601,34 @@ __global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwPara
     sc.mode = 0;
     const double xn = sqrt(s);
     sc.stats.input_norm = static_cast<float>(xn);
+    // The momentum kernel wrote X at scale sigma (chosen from the previous
+    // step's norm).  |X_ij| <= ||X||_F, so its largest stored entry is at
+    // most sigma ||X||; keep it when that lies in [2^(ex-6), 60000] and
+    // correct the scale exactly in the first GEMM epilogues (kappa);
+    // otherwise rewrite X at the ideal scale 2^ex / (||X|| + eps).
+    const double sigma = sc.sigma;
+    const double peak = sigma * xn;
+    sc.kappa = 1.f;
+    sc.rewrite = 1;
     if (!isfinite(s)) {
       sc.flags |= MUONH_FLAG_NONFINITE_INPUT;
       sc.xscale = 0.f;
     } else if (s == 0.0) {
       sc.flags |= MUONH_FLAG_ZERO_UPDATE;
       sc.xscale = 0.f;
+      if (sigma > 0.0) {   // X was written as zeros already
+        sc.rewrite = 0;
+        sc.kappa = 0.f;
+      }
     } else {
       sc.xscale = static_cast<float>(ldexp(1.0, md.ex) / (xn + static_cast<double>(p.eps)));
+      if (sigma > 0.0 && md.ns_steps > 0 && peak <= 60000.0 && peak >= ldexp(1.0, md.ex - 6)) {
+        sc.rewrite = 0;
+        sc.kappa = static_cast<float>(ldexp(1.0, md.ex) / (sigma * (xn + static_cast<double>(p.eps))));
+      }
     }
+    // scale for the next step's momentum kernel (not in FP32 mode: hi/lo X)
+    sc.sigma = (p.prec != P_FP32 && isfinite(s) && s > 0.0) ? static_cast<float>(ldexp(1.0, md.ex - 2) / xn) : 0.f;
   }
 }
 

@@ -360,10 +360,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
       // first row only, so a warp never splits around it.
       const int warp_row0 = row - lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
+      const float kap = (p.iter == 0) ? p.scal[td.mat].kappa : 1.f;
       if (MODE == M_GRAM) {
         // acc = 2^(2ex) A;  A_s = 2^ea A;  C_s = 2^ec (b I + c A)
-        const float sa = exp2f(static_cast<float>(md.ea - 2 * md.ex));
-        const float sc = md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
+        const float sa = kap * kap * exp2f(static_cast<float>(md.ea - 2 * md.ex));
+        const float sc = kap * kap * md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
         const float diag = md.b * exp2f(static_cast<float>(md.ec));
         const int64_t mo = md.z * cd.a_stride * 2;
         void* ahi = static_cast<uint8_t*>(cd.a[0]) + mo;
@@ -409,7 +410,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
         }
       } else {
         // acc = 2^(eb+ex) B' Y;  Y'_s = 2^ex B' Y
-        const float ks = exp2f(static_cast<float>(-md.eb));
+        const float ks = kap * exp2f(static_cast<float>(-md.eb));
         const int64_t xo = md.z * cd.x_stride * 2;
         void* yhi = static_cast<uint8_t*>(cd.x[p.src ^ 1][0]) + xo;
         void* ylo = cd.x[p.src ^ 1][1] ? static_cast<uint8_t*>(cd.x[p.src ^ 1][1]) + xo : nullptr;
@@ -676,9 +677,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int row0 = td.bi * kPairM + static_cast<int>(rank) * 128;   // this CTA's first row
       const int row = row0 + lrow;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
+      // iteration 0 reads X at the momentum kernel's scale: kappa corrects it
+      const float kap = (p.iter == 0) ? p.scal[td.mat].kappa : 1.f;
       if (MODE == M_GRAM) {
-        const float sa = exp2f(static_cast<float>(md.ea - 2 * md.ex));
-        const float sc = md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
+        const float sa = kap * kap * exp2f(static_cast<float>(md.ea - 2 * md.ex));
+        const float sc = kap * kap * md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
         const float diag = md.b * exp2f(static_cast<float>(md.ec));
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
@@ -746,7 +749,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-        const float ks = exp2f(static_cast<float>(-md.eb));
+        const float ks = kap * exp2f(static_cast<float>(-md.eb));
         const CUtensorMap* ymap = p.tmaps + cd.tm_base + TM_X_ST + (p.src ^ 1);
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
