@@ -153,6 +153,28 @@ def committed_traffic(kernel_file, workload, prec):
     return d[key]["dram_bytes_per_launch"]
 
 
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (device timings are reported as
+    the slowest rank's).  NCCL reduces on the rank's GPU, gloo on the CPU."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    if dist.get_backend() == "nccl":
+        dev = torch.device("cuda", torch.cuda.current_device())
+    else:
+        dev = torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, steps: int, max_ms: float) -> float:
+    """Steps per second of the whole job: every rank ran `steps` steps of its
+    own replica within the slowest rank's `max_ms`."""
+    return world * steps / (max_ms / 1000.0)
+
+
 # ------------------------------------------------------------------ oracle arm
 def oracle_sample_rate(shapes, wl, sample_idx, steps=1):
     """Time the oracle (as it stands, fp64) on a sample of the set for `steps`
@@ -269,12 +291,9 @@ def run_ours(args):
     ms = t_start.elapsed_time(t_end)
     phases = opt.phase_times()
     opt.device_status()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1000.0)
+    value = whole_job_rate(world, args.steps, ms)
 
     # ---------------- end to end through the public API, host buffers
     e2e = None
@@ -299,13 +318,9 @@ def run_ours(args):
             stream.synchronize()                  # the caller reads the step's stats
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world)
         h2d = sum(4 * a * b for a, b in shapes)
-        e2e = {"value": world * e2e_steps / (e_ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(world, e2e_steps, e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": 24 * n, "steps": e2e_steps}
         del host
 

@@ -108,12 +108,15 @@ def hyperball_update(W, O, lr, R, dtype=np.float64):
 
 
 def muonh_step(W, M, G, lr, R, beta=0.95, nesterov=True, ns_steps=5,
-               coeffs=QUINTIC, eps=1e-7, dtype=np.float64):
+               coeffs=QUINTIC, eps=1e-7, dtype=np.float64, ns_dtype=None):
     """One MuonH step for one matrix: momentum, Newton-Schulz, Eq. (1).
 
     Returns (W_{t+1}, M_t, O, stats) where stats also carries
     input_norm = ||X||_F.  A non-finite X leaves W unchanged (M follows the
-    plain arithmetic) and sets FLAG_NONFINITE_INPUT."""
+    plain arithmetic) and sets FLAG_NONFINITE_INPUT.  `ns_dtype` (default:
+    `dtype`) sets the precision of the Newton-Schulz products alone, so a
+    large matrix can run its O(r^2 c) matmuls in fp32 while every norm and
+    the projection stay in `dtype`."""
     M_new, X = momentum_update(M, G, beta, nesterov, dtype)
     x_norm = float(np.linalg.norm(X))
     if not np.isfinite(x_norm):
@@ -122,7 +125,7 @@ def muonh_step(W, M, G, lr, R, beta=0.95, nesterov=True, ns_steps=5,
         return W.copy(), M_new, None, dict(
             elr=0.0, pre_norm=w_norm, post_norm=w_norm, update_norm=0.0,
             input_norm=x_norm, flags=FLAG_NONFINITE_INPUT)
-    O = newton_schulz(X, ns_steps, coeffs, eps, dtype)
+    O = newton_schulz(X, ns_steps, coeffs, eps, ns_dtype or dtype).astype(dtype)
     W_new, st = hyperball_update(W, O, lr, R, dtype)
     if x_norm == 0.0:
         st["flags"] |= FLAG_ZERO_UPDATE

@@ -1,0 +1,39 @@
+"""The oracle pins must catch plausible mistakes: each case below plants one
+in a copy of the oracle (on the CPU, never in the CUDA path) and expects the
+pin tests to fail against it."""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "dropped A^2 term": ("B = b * A + c * (A @ A)", "B = b * A"),
+    "wrong sign of B Y": ("Y = a * Y + B @ Y", "Y = a * Y - B @ Y"),
+    "scaled Gram": ("A = Y @ Y.T", "A = 1.0001 * (Y @ Y.T)"),
+    "||W|| used for R": ("displacement = (lr * R / o_norm) * O", "displacement = (lr * w_norm / o_norm) * O"),
+    "projection onto ||W||": ("W_new = (R / wt_norm) * W_tilde", "W_new = (R / w_norm) * W_tilde"),
+    "lerp momentum": ("M_new = beta * M + G", "M_new = beta * M + (1 - beta) * G"),
+    "stale Nesterov term": ("X = G + beta * M_new if nesterov", "X = G + beta * M if nesterov"),
+    "max-norm input scaling": ("Y = Y / (np.linalg.norm(Y) + eps)", "Y = Y / (np.abs(Y).max() + eps)"),
+    "ELR over R": ("elr = float(np.linalg.norm(displacement)) / w_norm",
+                   "elr = float(np.linalg.norm(displacement)) / R"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTATIONS[name]
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d, ignore=shutil.ignore_patterns("__pycache__"))
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), tmp_path / "pytest.ini")
+    src = tmp_path / "oracle" / "muonh.py"
+    text = src.read_text()
+    assert old in text, "the oracle changed: update this mutation"
+    src.write_text(text.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "tests/test_oracle.py", "-m", "not gpu",
+                        "-p", "no:cacheprovider"], cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, f"pins did not catch: {name}"
