@@ -455,6 +455,9 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           return st;
         if ((st = encode_map(&m[TM_B_ST], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
+        if ((st = encode_map(&m[TM_B_MIR], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B)))
+          return st;
       }
     }
   }

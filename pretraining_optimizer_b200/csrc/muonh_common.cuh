@@ -43,6 +43,7 @@ enum TmSlot {
   TM_A_ST = 28,    // A store box
   TM_C_ST = 29,    // C store box
   TM_B_ST = 30,    // B' store box
+  TM_B_MIR = 31,   // B' mirrored-store box 64 x 32 (128-byte swizzle)
   TM_PER_CLASS = 32
 };
 __host__ __device__ inline int tm_x(int base, int buf, int part) { return base + buf + 2 * part; }

@@ -475,26 +475,52 @@ __device__ __forceinline__ uint32_t store_box_offset(int r, int q) {
   return static_cast<uint32_t>(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
 }
 
-// Double-buffered TMA-store staging shared by the 128 epilogue threads.
+// Double-buffered TMA-store staging shared by the 128 epilogue threads; each
+// 8 KB buffer holds either one 128-row x 32-column box of a tile (64-byte
+// swizzle) or the transposed 32-row x 128-column block of a mirrored store
+// (two 64-column halves, 128-byte swizzle).
 struct StoreStager {
   uint8_t* base;
-  int count;   // boxes issued so far by this CTA
-  __device__ __forceinline__ void put(const CUtensorMap* map, int lrow, const uint4 (&packed)[4], int x, int y,
-                                      int z) {
+  int count;   // buffers handed out so far by this CTA
+  __device__ __forceinline__ uint8_t* acquire() {
     uint8_t* buf = base + (count & 1) * (128 * 32 * 2);
     if (count >= 2) {
-      if (threadIdx.x == 64) bulk_wait_read<1>();   // the box issued two stores ago has been read
+      if (threadIdx.x == 64) bulk_wait_read<1>();   // the buffer's previous stores have been read
       asm volatile("bar.sync 1, 128;" ::: "memory");
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + store_box_offset(lrow, q)) = packed[q];
+    return buf;
+  }
+  __device__ __forceinline__ void issue(const CUtensorMap* map, const uint8_t* buf, int x, int y, int z,
+                                        bool mirror_halves) {
     fence_proxy_async_smem();
     asm volatile("bar.sync 1, 128;" ::: "memory");
     if (threadIdx.x == 64) {
       tma_store_3d(map, buf, x, y, z);
+      if (mirror_halves) tma_store_3d(map, buf + 64 * 32 * 2, x + 64, y, z);
       bulk_commit();
     }
     ++count;
+  }
+  __device__ __forceinline__ void put(const CUtensorMap* map, int lrow, const uint4 (&packed)[4], int x, int y,
+                                      int z) {
+    uint8_t* buf = acquire();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + store_box_offset(lrow, q)) = packed[q];
+    issue(map, buf, x, y, z, false);
+  }
+  // Mirrored store: warp `quarter` supplies, in lane j, row j of its
+  // transposed 32 x 32 block (32 values = columns quarter*32 .. +31 of the
+  // mirrored 32 x 128 block).  Stored at (x = first row of the CTA, y = col0).
+  __device__ __forceinline__ void put_mirror(const CUtensorMap* map, int quarter, int lane, const uint4 (&colv)[4],
+                                             int x, int y, int z) {
+    uint8_t* buf = acquire();
+    uint8_t* half = buf + (quarter >> 1) * (64 * 32 * 2);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c16 = (quarter & 1) * 4 + k;
+      *reinterpret_cast<uint4*>(half + lane * 128 + ((c16 ^ (lane & 7)) << 4)) = colv[k];
+    }
+    issue(map, buf, x, y, z, true);
   }
 };
 
@@ -710,10 +736,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const float sb = exp2f(static_cast<float>(md.eb - md.ea - md.ec));
         const float diag = md.a * exp2f(static_cast<float>(md.eb));
         using T16 = typename Store16<PREC>::T;
-        T16* bhi = reinterpret_cast<T16*>(static_cast<uint8_t*>(cd.b[0]) + md.z * cd.a_stride * 2);
         uint8_t* mirror_buf = smem + C::kMirrorOffset + quarter * 32 * C::kMirrorStride;
         const bool mirror = td.bj > td.bi;   // off-diagonal block: also store B'[col][row]
-        const int warp_row0 = row - lane;
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
           float v[32];
@@ -742,10 +766,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               cv[i] = *reinterpret_cast<const T16*>(mirror_buf + i * C::kMirrorStride + lane * 2);
-            uint4* mdst = reinterpret_cast<uint4*>(bhi + static_cast<int64_t>(col0 + lane) * cd.r_pad + warp_row0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) mdst[q] = colv[q];
             __syncwarp();
+            stager.put_mirror(p.tmaps + cd.tm_base + TM_B_MIR, quarter, lane, colv, row0, col0, md.z);
           }
         }
       } else {
