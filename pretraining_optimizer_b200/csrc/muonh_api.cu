@@ -155,6 +155,10 @@ struct muonh_ctx {
   int32_t* d_et_mat = nullptr;
   float* d_part = nullptr;
   double* d_part64 = nullptr;
+  float* d_part_ns = nullptr;      // fused last-APPLY partials
+  CUtensorMap* d_wmaps = nullptr;  // per matrix fp32 W tiles (fused matrices)
+  int64_t n_ns_slots = 0;
+  bool any_unfused = true;
   CUtensorMap* d_tmaps = nullptr;
   int* d_err = nullptr;
 
@@ -192,6 +196,7 @@ struct muonh_ctx {
     p.n_et = n_et;
     p.part = d_part;
     p.part64 = d_part64;
+    p.part_ns = d_part_ns;
     p.n = n;
     p.eps = eps;
     p.prec = prec;
@@ -239,6 +244,23 @@ muonh_status encode_map(CUtensorMap* out, void* base, int prec16_is_bf16, int64_
                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return MUONH_OK;
+}
+
+// 2-D fp32 map over a caller's W (rows x cols, row stride ld elements):
+// wide W: 32 x 128 boxes (128-byte swizzle); tall W: 128 x 32 boxes.
+muonh_status encode_w_map(CUtensorMap* out, const MatDev& md) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(md.cols), static_cast<cuuint64_t>(md.rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(md.ld * 4)};
+  const cuuint32_t box[2] = {md.transposed ? 128u : 32u, md.transposed ? 32u : 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, md.w, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  md.transposed ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled (W) failed (%d)", static_cast<int>(r));
   return MUONH_OK;
 }
 
@@ -393,6 +415,22 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   }
   ctx->n_et = n_et;
 
+  // ---- fused ||O||^2, <W, O> in the last APPLY (CTA pairs, vector path,
+  // matrices whose last iteration is the last launch): 2 slots per pair tile
+  for (int32_t i = 0; i < n; ++i) {
+    MatDev& md = ctx->mats[i];
+    const ClassHost& ch = ctx->classes[md.cls];
+    md.fused_dots = (ctx->pairs && md.vec && md.ns_steps > 0 && md.ns_steps == ctx->max_steps) ? 1 : 0;
+    md.ns_tiles_bj = ch.c_pad / kBN;
+    if (md.fused_dots) {
+      md.ns_slots = 2 * (ch.r_pad / (2 * kBM)) * md.ns_tiles_bj;
+      md.ns_slot_base = ctx->n_ns_slots;
+      ctx->n_ns_slots += md.ns_slots;
+    }
+  }
+  ctx->any_unfused = false;
+  for (int32_t i = 0; i < n; ++i) ctx->any_unfused |= !ctx->mats[i].fused_dots;
+
   // ---- workspace
   const int parts = ctx->prec == P_FP32 ? 2 : 1;
   for (ClassHost& ch : ctx->classes) {
@@ -472,6 +510,9 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_et_mat), n_et * sizeof(int32_t)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part), 2 * n_et * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part64), n_et * sizeof(double)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part_ns),
+                std::max<int64_t>(1, 2 * ctx->n_ns_slots) * sizeof(float)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_wmaps), n * sizeof(CUtensorMap)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), sizeof(int)) != cudaSuccess)
     return fail(MUONH_ERR_OOM, "allocation of the device tables failed");
 
@@ -487,6 +528,14 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
     scal[i] = MatScal{};
     scal[i].R = mats[i].radius > 0.f ? mats[i].radius : 0.f;
   }
+  std::vector<CUtensorMap> wmaps(n);
+  std::memset(wmaps.data(), 0, n * sizeof(CUtensorMap));
+  for (int32_t i = 0; i < n; ++i)
+    if (ctx->mats[i].fused_dots) {
+      muonh_status st = encode_w_map(&wmaps[i], ctx->mats[i]);
+      if (st != MUONH_OK) return st;
+    }
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_wmaps, wmaps.data(), n * sizeof(CUtensorMap), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_mats, ctx->mats.data(), n * sizeof(MatDev), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_classes, cdev.data(), cdev.size() * sizeof(ClassDev), cudaMemcpyHostToDevice, s));
@@ -599,6 +648,8 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
     np.src = k & 1;
     np.iter = k;
     np.scal = ctx->d_scal;
+    np.wmaps = ctx->d_wmaps;
+    np.part_ns = ctx->d_part_ns;
     np.tiles = ctx->gram_lists[k].dev;
     np.ntiles = ctx->gram_lists[k].count;
     if (ctx->pairs) {
@@ -608,8 +659,9 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
       STEP_LAUNCH(MUONH_PHASE_NS_SQUARE, launch_ns_gemm_pair(M_SQUARE, ctx->prec, np, gp, s), "ns_square");
       np.tiles = ctx->apply_lists[k].dev;
       np.ntiles = ctx->apply_lists[k].count;
+      const int amode = (k == ctx->max_steps - 1) ? M_APPLY_LAST : M_APPLY;
       STEP_LAUNCH(MUONH_PHASE_NS_APPLY,
-                  launch_ns_gemm_pair(M_APPLY, ctx->prec, np, std::min(pairs_max, std::max(1, np.ntiles)), s),
+                  launch_ns_gemm_pair(amode, ctx->prec, np, std::min(pairs_max, std::max(1, np.ntiles)), s),
                   "ns_apply");
     } else {
       const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
@@ -622,7 +674,7 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
                   "ns_apply");
     }
   }
-  STEP_LAUNCH(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, s), "update_dots");
+  if (ctx->any_unfused) STEP_LAUNCH(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, s), "update_dots");
   STEP_LAUNCH(MUONH_PHASE_FINALIZE_UPDATE, launch_finalize_update(p, s), "finalize_update");
   STEP_LAUNCH(MUONH_PHASE_PROJECT, launch_project(p, grid, s), "project");
   STEP_LAUNCH(MUONH_PHASE_FINALIZE_STEP, launch_finalize_step(p, s), "finalize_step");

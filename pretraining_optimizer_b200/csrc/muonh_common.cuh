@@ -24,7 +24,7 @@ constexpr int kGemmThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2-5 epilog
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
 
 enum Prec { P_FP16 = 0, P_BF16 = 1, P_FP32 = 2 };
-enum Mode { M_GRAM = 0, M_SQUARE = 1, M_APPLY = 2 };
+enum Mode { M_GRAM = 0, M_SQUARE = 1, M_APPLY = 2, M_APPLY_LAST = 3 };   // LAST: also ||O||^2, <W, O>
 
 // Tensor-map slots of one shape class.  "hi" buffers hold the 16-bit
 // operand (fp16/bf16), "lo" buffers the fp16 residual in FP32 mode.
@@ -64,6 +64,10 @@ struct MatDev {
   int32_t et_rows, et_cols;  // elementwise tile grid
   int32_t et_th, et_tw;      // elementwise tile shape: 64 x 64 for tall W, <= 8 x 512 rows otherwise
   int64_t et_begin;          // first elementwise tile
+  int32_t fused_dots;        // ||O||^2, <W, O> come from the last APPLY (else from update_dots)
+  int32_t ns_tiles_bj;       // APPLY pair tiles per tile row (c_pad / 256)
+  int64_t ns_slot_base;      // first (||O||^2, <W, O>) slot: 2 per pair tile (one per CTA)
+  int32_t ns_slots;
 };
 
 struct ClassDev {
@@ -107,6 +111,8 @@ struct NsParams {
   int32_t src;               // X buffer read by this phase
   int32_t iter;              // Newton-Schulz iteration of this launch (0: apply kappa)
   const MatScal* scal;
+  const CUtensorMap* wmaps;  // per matrix: fp32 W tiles for the last APPLY's <W, O>
+  float* part_ns;            // per (pair tile, CTA): ||O||^2 and <W, O> at the stored scale
   const MatDev* mats;
   const ClassDev* classes;
   const CUtensorMap* tmaps;
@@ -122,6 +128,7 @@ struct EwParams {
   int64_t n_et;
   float* part;               // per-tile partials
   double* part64;
+  const float* part_ns;      // partials of the fused last APPLY (MatDev::fused_dots)
   int32_t n;
   float eps;
   int32_t prec;
@@ -211,6 +218,14 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // Make generic-proxy shared-memory writes visible to the async (TMA) proxy.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

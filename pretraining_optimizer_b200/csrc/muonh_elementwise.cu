@@ -454,6 +454,7 @@ __global__ void __launch_bounds__(kEwThreads, 8) update_dots_kernel(const EwPara
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
+    if (md.fused_dots) continue;   // the last APPLY produced this matrix's partials
     const XView xv = x_view(p, md, md.ns_steps & 1);
     if (md.transposed) {
       __syncthreads();
@@ -636,9 +637,15 @@ __global__ void __launch_bounds__(kEwThreads) finalize_update_kernel(const EwPar
   __shared__ double red[kEwThreads / 32];
   const int mi = blockIdx.x;
   const MatDev& md = p.mats[mi];
-  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
-  const double soo = matrix_sum(p.part, md.et_begin, cnt, 2, 0, red);
-  const double swo = matrix_sum(p.part, md.et_begin, cnt, 2, 1, red);
+  double soo, swo;
+  if (md.fused_dots) {
+    soo = matrix_sum(p.part_ns, md.ns_slot_base, md.ns_slots, 2, 0, red);
+    swo = matrix_sum(p.part_ns, md.ns_slot_base, md.ns_slots, 2, 1, red);
+  } else {
+    const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
+    soo = matrix_sum(p.part, md.et_begin, cnt, 2, 0, red);
+    swo = matrix_sum(p.part, md.et_begin, cnt, 2, 1, red);
+  }
   if (threadIdx.x == 0) {
     MatScal& sc = p.scal[mi];
     const double unscale = ldexp(1.0, -md.ex);

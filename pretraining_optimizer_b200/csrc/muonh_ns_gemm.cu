@@ -449,9 +449,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 // upper block triangle only.  A consumer that needs a block below the
 // diagonal loads the stored transposed block and hands it to the MMA as an
 // MN-major operand, so no epilogue writes a mirrored copy.
-template <int PREC>
+template <int PREC, int MODE>
 struct PairCfg {
-  static constexpr int kStages = 6;
+  // the last APPLY gives one pipeline stage to the fp32 W staging buffers
+  static constexpr bool kLast = MODE == M_APPLY_LAST;
+  static constexpr int kStages = kLast ? 5 : 6;
   static constexpr int kABytes = 128 * kBK * 2;                 // 16 KB: this CTA's 128 rows
   static constexpr int kBBytes = 128 * kBK * 2;                 // 16 KB: this CTA's half of N
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -466,7 +468,11 @@ struct PairCfg {
   // to global memory by TMA stores (64-byte swizzle)
   static constexpr int kStoreBox = 128 * 32 * 2;
   static constexpr int kStoreOffset = (kMirrorOffset + kMirrorBytes + 1023) / 1024 * 1024;
-  static constexpr int kSmem = kStoreOffset + 2 * kStoreBox + 1024;
+  // Last APPLY: two fp32 W boxes (128 rows x 32 columns, or 32 x 128 for
+  // a tall W) loaded by TMA for the <W, O> partials
+  static constexpr int kWBox = 128 * 32 * 4;
+  static constexpr int kWOffset = kStoreOffset + 2 * kStoreBox;
+  static constexpr int kSmem = kWOffset + (kLast ? 2 * kWBox : 0) + 1024;
 };
 
 // Epilogue row `r` (0..127) of a 128 x 32 16-bit box, 16-byte piece q,
@@ -536,7 +542,8 @@ constexpr int kPairM = 256;
 template <int MODE, int PREC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     ns_gemm_pair_kernel(const __grid_constant__ NsParams p) {
-  using C = PairCfg<PREC>;
+  using C = PairCfg<PREC, MODE>;
+  constexpr bool kApply = MODE == M_APPLY || MODE == M_APPLY_LAST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -544,7 +551,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* wfull = drain + 1;                       // last APPLY: W boxes landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + 2);
+  float* red = reinterpret_cast<float*>(tmem_slot + 4);   // 8 floats
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -562,6 +571,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[a], 2 * 128);                // both CTAs' epilogue threads
     }
     mbar_init(drain, 1);
+    mbar_init(&wfull[0], 1);
+    mbar_init(&wfull[1], 1);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
@@ -604,7 +615,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             // A operand: rows of the symmetric A (SQUARE: upper blocks only,
             // lower blocks through their stored transpose) or of B' (APPLY:
             // stored with its mirror, always K-major)
-            if (MODE == M_APPLY || k0 >= abase) {
+            if (kApply || k0 >= abase) {
               tma_load_3d_pair(sa, p.tmaps + cd.tm_base + (MODE == M_SQUARE ? TM_A_K128 : TM_B_K128), bar, k0,
                                arow, z);
             } else {
@@ -658,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         for (int kb = 0; kb < nk; ++kb) {
           const int k0 = kb * kBK;
           const bool a_mn = (MODE == M_SQUARE) && k0 < abase;
-          const bool b_mn = (MODE == M_APPLY) || (MODE == M_SQUARE && k0 < bbase);
+          const bool b_mn = kApply || (MODE == M_SQUARE && k0 < bbase);
           const uint32_t idesc = kIdescKK | (a_mn ? kAMn : 0u) | (b_mn ? kBMn : 0u);
           if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
           tc_fence_after();
@@ -691,6 +702,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int lrow = quarter * 32 + lane;
     const uint32_t tempty_leader[2] = {map_shared_rank(&tempty[0], 0), map_shared_rank(&tempty[1], 0)};
     StoreStager stager{smem + C::kStoreOffset, 0};
+    uint32_t wphase[2] = {0u, 0u};   // last APPLY: phases of the two W buffers
+    int w_pending[2] = {0, 0};       // thread 64: W loads issued and not yet consumed
+    bool werr = false;
+    // thread 64 loads the W box of chunk `chk` into buffer b
+    auto w_issue = [&](const TileDesc& td, const MatDev& md, int row0, int b, int chk) {
+      const int c0 = td.bj * kBN + chk * 32;
+      mbar_expect_tx(&wfull[b], C::kWBox);
+      uint8_t* dst = smem + C::kWOffset + b * C::kWBox;
+      if (!md.transposed)
+        tma_load_2d(dst, p.wmaps + td.mat, &wfull[b], c0, row0);
+      else
+        tma_load_2d(dst, p.wmaps + td.mat, &wfull[b], row0, c0);
+      ++w_pending[b];
+    };
     int local = 0;
     for (int t = pair; t < p.ntiles; t += npairs, ++local) {
       const TileDesc td = p.tiles[t];
@@ -698,6 +723,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const ClassDev& cd = p.classes[md.cls];
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
+      if (C::kLast && threadIdx.x == 64 && md.fused_dots && p.iter == md.ns_steps - 1) {
+        const int r0 = td.bi * kPairM + static_cast<int>(rank) * 128;
+        w_issue(td, md, r0, 0, 0);   // W of chunks 0 and 1 while the tile's MMAs run
+        w_issue(td, md, r0, 1, 1);
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
       tc_fence_after();
       const int row0 = td.bi * kPairM + static_cast<int>(rank) * 128;   // this CTA's first row
@@ -773,6 +803,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       } else {
         const float ks = kap * exp2f(static_cast<float>(-md.eb));
         const CUtensorMap* ymap = p.tmaps + cd.tm_base + TM_X_ST + (p.src ^ 1);
+        // Last APPLY: Y' is the update O; accumulate ||O||^2 and <W, O> over
+        // the stored values, W staged per 32-column chunk by TMA (wide W: box
+        // of W[row0.., col0..]; tall W: box of W[col0.., row0..]).
+        const bool dots = C::kLast && md.fused_dots && p.iter == md.ns_steps - 1;
+        float oo = 0.f, wo = 0.f;
         for (int ch = 0; ch < kBN / 32; ++ch) {
           const int col0 = td.bj * kBN + ch * 32;
           float v[32];
@@ -786,10 +821,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           uint4 packed[4];
           pack32<PREC>(v, packed);
           stager.put(ymap, lrow, packed, col0, row0, md.z);
+          if (C::kLast && dots) {
+            const int b = ch & 1;
+            if (!mbar_wait(&wfull[b], wphase[b], p.err)) { werr = true; break; }
+            wphase[b] ^= 1u;
+            if (threadIdx.x == 64) --w_pending[b];
+            const uint8_t* wb = smem + C::kWOffset + b * C::kWBox;
+            using T16 = typename Store16<PREC>::T;
+            const T16* h = reinterpret_cast<const T16*>(packed);
+            if (!md.transposed) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 w4 = *reinterpret_cast<const float4*>(wb + lrow * 128 + ((q ^ (lrow & 7)) << 4));
+                const float o0 = Store16<PREC>::back(h[4 * q]), o1 = Store16<PREC>::back(h[4 * q + 1]);
+                const float o2 = Store16<PREC>::back(h[4 * q + 2]), o3 = Store16<PREC>::back(h[4 * q + 3]);
+                oo = fmaf(o0, o0, fmaf(o1, o1, fmaf(o2, o2, fmaf(o3, o3, oo))));
+                wo = fmaf(w4.x, o0, fmaf(w4.y, o1, fmaf(w4.z, o2, fmaf(w4.w, o3, wo))));
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float w = *reinterpret_cast<const float*>(wb + j * 512 + lrow * 4);
+                const float o = Store16<PREC>::back(h[j]);
+                oo = fmaf(o, o, oo);
+                wo = fmaf(w, o, wo);
+              }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // every thread is done with W buffer b
+            if (threadIdx.x == 64 && ch + 2 < kBN / 32) w_issue(td, md, row0, b, ch + 2);
+          }
+        }
+        if (werr) break;
+        if (C::kLast && dots) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            oo += __shfl_xor_sync(0xffffffffu, oo, o);
+            wo += __shfl_xor_sync(0xffffffffu, wo, o);
+          }
+          if (lane == 0) {
+            red[2 * quarter] = oo;
+            red[2 * quarter + 1] = wo;
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (threadIdx.x == 64) {
+            const int64_t slot =
+                md.ns_slot_base + (static_cast<int64_t>(td.bi) * md.ns_tiles_bj + td.bj) * 2 + rank;
+            p.part_ns[2 * slot] = ((red[0] + red[2]) + red[4]) + red[6];
+            p.part_ns[2 * slot + 1] = ((red[1] + red[3]) + red[5]) + red[7];
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
         }
       }
     }
-    if (threadIdx.x == 64) bulk_wait_all();   // every TMA store has completed
+    if (threadIdx.x == 64) {
+      bulk_wait_all();   // every TMA store has completed
+      // on a give-up path, let issued W loads land before the CTA exits
+      for (int b = 0; b < 2; ++b)
+        for (; w_pending[b] > 0; --w_pending[b]) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&wfull[b], wphase[b]) && globaltimer() - t0 < kWaitLimitNs) {
+          }
+          wphase[b] ^= 1u;
+        }
+    }
   }
 
   tc_fence_before();
@@ -810,7 +904,7 @@ static cudaError_t set_attr() {
 template <int MODE, int PREC>
 static cudaError_t set_pair_attr() {
   return cudaFuncSetAttribute(ns_gemm_pair_kernel<MODE, PREC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              PairCfg<PREC>::kSmem);
+                              PairCfg<PREC, MODE>::kSmem);
 }
 
 cudaError_t ns_gemm_set_attributes() {
@@ -818,7 +912,9 @@ cudaError_t ns_gemm_set_attributes() {
 #define MUONH_SET_PAIR(MD, PR) \
   if ((e = set_pair_attr<MD, PR>()) != cudaSuccess) return e;
   MUONH_SET_PAIR(M_GRAM, P_FP16) MUONH_SET_PAIR(M_SQUARE, P_FP16) MUONH_SET_PAIR(M_APPLY, P_FP16)
+  MUONH_SET_PAIR(M_APPLY_LAST, P_FP16)
   MUONH_SET_PAIR(M_GRAM, P_BF16) MUONH_SET_PAIR(M_SQUARE, P_BF16) MUONH_SET_PAIR(M_APPLY, P_BF16)
+  MUONH_SET_PAIR(M_APPLY_LAST, P_BF16)
 #undef MUONH_SET_PAIR
 #define MUONH_SET(MD, PR) \
   if ((e = set_attr<MD, PR>()) != cudaSuccess) return e;
@@ -835,14 +931,15 @@ size_t ns_gemm_smem_bytes(int prec) {
 
 cudaError_t launch_ns_gemm_pair(int mode, int prec, const NsParams& p, int pairs, cudaStream_t s) {
   if (p.ntiles <= 0) return cudaSuccess;
-  const size_t smem = PairCfg<P_FP16>::kSmem;
-#define MUONH_LAUNCH_PAIR(MD, PR)                                                \
-  if (mode == MD && prec == PR) {                                                \
-    ns_gemm_pair_kernel<MD, PR><<<2 * pairs, kGemmThreads, smem, s>>>(p);       \
-    return cudaGetLastError();                                                   \
+#define MUONH_LAUNCH_PAIR(MD, PR)                                                              \
+  if (mode == MD && prec == PR) {                                                              \
+    ns_gemm_pair_kernel<MD, PR><<<2 * pairs, kGemmThreads, PairCfg<PR, MD>::kSmem, s>>>(p);   \
+    return cudaGetLastError();                                                                 \
   }
   MUONH_LAUNCH_PAIR(M_GRAM, P_FP16) MUONH_LAUNCH_PAIR(M_SQUARE, P_FP16) MUONH_LAUNCH_PAIR(M_APPLY, P_FP16)
+  MUONH_LAUNCH_PAIR(M_APPLY_LAST, P_FP16)
   MUONH_LAUNCH_PAIR(M_GRAM, P_BF16) MUONH_LAUNCH_PAIR(M_SQUARE, P_BF16) MUONH_LAUNCH_PAIR(M_APPLY, P_BF16)
+  MUONH_LAUNCH_PAIR(M_APPLY_LAST, P_BF16)
 #undef MUONH_LAUNCH_PAIR
   return cudaErrorInvalidValue;
 }
