@@ -56,6 +56,7 @@ def parse():
     ap.add_argument("--ns-precision", default="fp16", choices=["fp16", "bf16", "fp32"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-aux", action="store_true")
     return ap.parse_args()
 
 
@@ -234,6 +235,58 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ our arm
+def time_launches(fn, stream, warmup=3, reps=10):
+    """Average device time (ms) of fn() over `reps` launches after `warmup`."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_aux(dev, stream, hbm_peak, matrix_params):
+    """The two auxiliary kernels of the recipe on the 1.7B model's own sizes,
+    each timed alone (burst HBM peak): the AdamW step over the parameters
+    outside the matrix set, and the average of six bf16 checkpoints of the
+    whole model.  Inputs far exceed L2."""
+    import torch
+    import synth
+    from pretraining_optimizer_b200 import adamw_step, average
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    group = synth.qwen3_adamw_group(2048)
+    p = [torch.randn(n, generator=gen, device=dev) * 0.02 for _, n in group]
+    m = [torch.zeros_like(x) for x in p]
+    v = [torch.zeros_like(x) for x in p]
+    g = [torch.randn(x.shape, generator=gen, device=dev) * 1e-3 for x in p]
+    n_adam = sum(n for _, n in group)
+    adam_ms = time_launches(lambda: adamw_step(p, m, v, g, 1, 1e-3, 0.9, 0.95, 1e-8, 0.1), stream)
+    adam_gbps = 28 * n_adam / (adam_ms / 1000.0) / 1e9          # read p, m, v, g; write p, m, v
+    del p, m, v, g
+    total = n_adam + matrix_params
+    ckpts = [torch.randn(total, generator=gen, device=dev, dtype=torch.bfloat16) for _ in range(6)]
+    out = torch.empty(total, device=dev, dtype=torch.bfloat16)
+    avg_ms = time_launches(lambda: average(ckpts, out=out), stream, reps=5)
+    avg_gbps = 14 * total / (avg_ms / 1000.0) / 1e9             # read 6 x 2 B, write 2 B
+    del ckpts, out
+    torch.cuda.empty_cache()
+    return {
+        "adamw_step": {"elements": n_adam, "tensors": len(group), "launches": -(-len(group) // 32),
+                       "ms": adam_ms, "gbps": adam_gbps, "frac": adam_gbps / hbm_peak,
+                       "bytes_per_elem": 28},
+        "average": {"elements": total, "checkpoints": 6, "dtype": "bf16 -> bf16", "ms": avg_ms,
+                    "gbps": avg_gbps, "frac": avg_gbps / hbm_peak, "bytes_per_elem": 14},
+        "peak": "hbm_gbs (burst copy)",
+    }
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -353,6 +406,11 @@ def run_ours(args):
         "hbm_peak_gbps": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
     }
 
+    # ---------------- auxiliary kernels (rank 0 of a single-GPU run; not part of the step)
+    aux = None
+    if rank == 0 and world == 1 and not args.no_aux and args.workload == "qwen3_1.7b":
+        aux = measure_aux(dev, stream, peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), elems)
+
     # ---------------- CPU baseline: the oracle on layer 0, rank 0, N = 1
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -374,7 +432,8 @@ def run_ours(args):
                            "l2": "inputs larger than L2 (no flush)",
                            "parallelism": f"{world} independent replica(s)"},
                 "roofline": roofline, "summary": summary, "kernels": kernels, "clocks": clocks,
-                "gpu_launches": launches_per_step * args.steps, "e2e": e2e, "cpu_baseline": cpu}
+                "gpu_launches": launches_per_step * args.steps, "e2e": e2e, "cpu_baseline": cpu,
+                "aux_kernels": aux}
         print(json.dumps(line), flush=True)
     opt.close()
     if world > 1:

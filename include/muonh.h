@@ -70,6 +70,14 @@ enum {
   MUONH_FLAG_TIMEOUT = 16u           /* a device wait gave up during this step   */
 };
 
+/* Update rule of a matrix (report Sec. 3.3 and 3.3.1).
+ *   HYPERBALL     Eq. (1): MuonH, W <- R (W - lr R u^)/||.||, lr = the ELR.
+ *   DECOUPLED_WD  Eq. (3): ordinary Muon, W <- (1 - wd lr) W - lr u.
+ *   ELR_ALIGNED   Eq. (5): ordinary Muon with eta = lr ||W||/||u|| (lr = the
+ *                 prescribed ELR), W <- (1 - wd eta) W - eta u, no projection.
+ * For the ordinary rules u = update_scale * O, O the Newton-Schulz output. */
+enum { MUONH_RULE_HYPERBALL = 0, MUONH_RULE_DECOUPLED_WD = 1, MUONH_RULE_ELR_ALIGNED = 2 };
+
 /* One wrapped matrix.  w and m are caller-owned fp32 device buffers of
  * rows x cols elements, row-major with row stride ld (elements, ld >= cols),
  * 16-byte aligned base.  Rows are moved with 16-byte vector accesses when
@@ -92,6 +100,9 @@ typedef struct {
   float ns_a;
   float ns_b;
   float ns_c;
+  int32_t update_rule;    /* MUONH_RULE_*; 0 = MuonH                        */
+  float weight_decay;     /* lambda of Eq. (3)/(5); ignored by MuonH         */
+  float update_scale;     /* u = update_scale * O for the ordinary rules     */
 } muonh_matrix_desc;
 
 typedef struct {
@@ -204,6 +215,62 @@ muonh_status muonh_phase_times(muonh_ctx* ctx, float* ms_out, int64_t* launches_
  * ordered and safe.  Enqueued on `stream`. */
 muonh_status muonh_momentum_norm_noalloc(float* m, const float* g, int64_t rows, int64_t cols, int64_t ld,
                                          float beta, int32_t nesterov, double* x_norm, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Auxiliary operations of the same training recipe.  Stateless: no context,
+ * no allocation; enqueued on `stream`.
+ * ------------------------------------------------------------------------- */
+
+#define MUONH_DTYPE_F32 0
+#define MUONH_DTYPE_BF16 1
+#define MUONH_AVERAGE_MAX_INPUTS 16
+#define MUONH_ADAMW_MAX_TENSORS 32   /* per launch; longer lists take several */
+
+/* Checkpoint parameter averaging (Puro-2B report, Sec. 3.4: the released
+ * model is the equal average of six checkpoints; parameters only).
+ *   out[j] = (in[0][j] + in[1][j] + ... + in[k-1][j]) / k
+ * summed in fp32 in that order, rounded once to out_dtype.
+ *   out     device buffer of `count` elements of out_dtype; may alias in[0]
+ *           (each element is read before it is written, by the same thread).
+ *   in      HOST array of k device pointers, each `count` elements of in_dtype.
+ *   dtypes  MUONH_DTYPE_F32 or MUONH_DTYPE_BF16.
+ *   k       1..MUONH_AVERAGE_MAX_INPUTS.
+ * Every pointer must be 16-byte aligned (MUONH_ERR_ALIGNMENT otherwise).
+ * count == 0 checks k and the dtypes only (the buffers may be NULL) and
+ * enqueues nothing. */
+muonh_status muonh_average(void* out, int32_t out_dtype, const void* const* in, int32_t in_dtype, int32_t k,
+                           int64_t count, void* stream);
+
+/* One flat fp32 tensor of the AdamW group: parameters p, first and second
+ * moments m and v (updated in place), gradient g (read), `count` elements
+ * each.  Pointers need 4-byte alignment; a tensor whose four pointers are
+ * all 16-byte aligned takes the vector path. */
+typedef struct {
+  float* p;
+  float* m;
+  float* v;
+  const float* g;
+  int64_t count;
+} muonh_adamw_tensor;
+
+typedef struct {
+  float lr;
+  float beta1;          /* Puro-2B report App. E: 0.9  */
+  float beta2;          /*                        0.95 */
+  float eps;
+  float weight_decay;   /* Table 8: 0.1 for the AdamW group */
+} muonh_adamw_config;
+
+/* AdamW step for the parameter group outside MuonH (Puro-2B report, Table 8:
+ * embeddings, normalisation layers, LM head).  With `step` = t >= 1 (1-based,
+ * the caller's count of steps taken including this one), per element:
+ *   p <- p (1 - lr wd);   m <- b1 m + (1 - b1) g;   v <- b2 v + (1 - b2) g^2
+ *   p <- p - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * in fp32 (the bias corrections are formed in double, then rounded).
+ * `tensors` is a HOST array of n descriptors; all of them are updated by
+ * ceil(n / MUONH_ADAMW_MAX_TENSORS) launches.  Tensors must not overlap. */
+muonh_status muonh_adamw_step(const muonh_adamw_tensor* tensors, int32_t n, const muonh_adamw_config* cfg,
+                              int64_t step, void* stream);
 
 void muonh_destroy(muonh_ctx* ctx);
 

@@ -16,6 +16,7 @@ and the geometric-sum form of the momentum buffer.
 """
 from .muonh import (  # noqa: F401
     QUINTIC, FLAG_NONFINITE_INPUT, FLAG_ZERO_UPDATE, FLAG_NONFINITE_UPDATE,
-    FLAG_DEGENERATE, momentum_update, newton_schulz, hyperball_update,
+    FLAG_DEGENERATE, RULE_HYPERBALL, RULE_DECOUPLED_WD, RULE_ELR_ALIGNED,
+    momentum_update, newton_schulz, hyperball_update, muon_update,
     radius, muonh_step, run_steps,
 )

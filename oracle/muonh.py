@@ -25,6 +25,10 @@ import numpy as np
 
 QUINTIC = (3.4445, -4.7750, 2.0315)
 
+RULE_HYPERBALL = 0          # Eq. (1): MuonH
+RULE_DECOUPLED_WD = 1       # Eq. (3): ordinary Muon with decoupled weight decay
+RULE_ELR_ALIGNED = 2        # Eq. (5): ordinary Muon, scalar LR set online to a prescribed ELR
+
 FLAG_NONFINITE_INPUT = 1    # the Newton-Schulz input X has a NaN/Inf entry
 FLAG_ZERO_UPDATE = 2        # ||X||_F == 0 or ||O||_F == 0: no displacement
 FLAG_NONFINITE_UPDATE = 4   # X finite but the orthogonalised O is not
@@ -107,9 +111,40 @@ def hyperball_update(W, O, lr, R, dtype=np.float64):
                        update_norm=o_norm, flags=flags)
 
 
+def muon_update(W, O, lr, weight_decay=0.0, update_scale=1.0, rule=RULE_DECOUPLED_WD,
+                dtype=np.float64):
+    """Ordinary Muon on one matrix, with the update u = update_scale * O.
+
+    Eq. (3) (report Sec. 3.3.1): W_{t+1} = (1 - lambda eta) W_t - eta u_t with
+    eta = lr; its effective LR, Eq. (4), is eta ||u||_F / ||W_t||_F.
+    Eq. (5): the scalar LR is set online, eta = rho ||W_t||_F / ||u_t||_F with
+    rho = lr the prescribed effective LR, so Eq. (4) gives exactly rho; W is
+    not projected.  A zero update leaves W unchanged.
+    Returns (W_{t+1}, stats) with the fields of hyperball_update plus eta."""
+    W = np.asarray(W, dtype=dtype)
+    O = np.asarray(O, dtype=dtype)
+    u = update_scale * O
+    w_norm = float(np.linalg.norm(W))
+    u_norm = float(np.linalg.norm(u))
+    o_norm = float(np.linalg.norm(O))
+    if not np.isfinite(u_norm):
+        return W.copy(), dict(elr=0.0, pre_norm=w_norm, post_norm=w_norm, update_norm=o_norm,
+                              flags=FLAG_NONFINITE_UPDATE, eta=0.0)
+    if u_norm == 0.0:
+        return W.copy(), dict(elr=0.0, pre_norm=w_norm, post_norm=w_norm, update_norm=o_norm,
+                              flags=FLAG_ZERO_UPDATE, eta=0.0)
+    eta = lr if rule == RULE_DECOUPLED_WD else lr * w_norm / u_norm
+    W_new = (1.0 - weight_decay * eta) * W - eta * u
+    return W_new, dict(elr=eta * u_norm / w_norm, pre_norm=w_norm,
+                       post_norm=float(np.linalg.norm(W_new)), update_norm=o_norm, flags=0,
+                       eta=eta)
+
+
 def muonh_step(W, M, G, lr, R, beta=0.95, nesterov=True, ns_steps=5,
-               coeffs=QUINTIC, eps=1e-7, dtype=np.float64, ns_dtype=None):
-    """One MuonH step for one matrix: momentum, Newton-Schulz, Eq. (1).
+               coeffs=QUINTIC, eps=1e-7, dtype=np.float64, ns_dtype=None,
+               rule=RULE_HYPERBALL, weight_decay=0.0, update_scale=1.0):
+    """One step for one matrix: momentum, Newton-Schulz, then Eq. (1)
+    (rule RULE_HYPERBALL, MuonH) or ordinary Muon by Eq. (3) / Eq. (5).
 
     Returns (W_{t+1}, M_t, O, stats) where stats also carries
     input_norm = ||X||_F.  A non-finite X leaves W unchanged (M follows the
@@ -126,7 +161,10 @@ def muonh_step(W, M, G, lr, R, beta=0.95, nesterov=True, ns_steps=5,
             elr=0.0, pre_norm=w_norm, post_norm=w_norm, update_norm=0.0,
             input_norm=x_norm, flags=FLAG_NONFINITE_INPUT)
     O = newton_schulz(X, ns_steps, coeffs, eps, ns_dtype or dtype).astype(dtype)
-    W_new, st = hyperball_update(W, O, lr, R, dtype)
+    if rule == RULE_HYPERBALL:
+        W_new, st = hyperball_update(W, O, lr, R, dtype)
+    else:
+        W_new, st = muon_update(W, O, lr, weight_decay, update_scale, rule, dtype)
     if x_norm == 0.0:
         st["flags"] |= FLAG_ZERO_UPDATE
     st["input_norm"] = x_norm

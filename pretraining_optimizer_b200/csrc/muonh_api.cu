@@ -333,6 +333,9 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
     if (!std::isfinite(d.beta) || !std::isfinite(d.ns_a) || !std::isfinite(d.ns_b) || !std::isfinite(d.ns_c) ||
         !std::isfinite(d.radius))
       return fail(MUONH_ERR_INVALID_ARG, "matrix %d: beta, coefficients and radius must be finite", i);
+    if (d.update_rule < 0 || d.update_rule > 2 || !std::isfinite(d.weight_decay) || !std::isfinite(d.update_scale) ||
+        (d.update_rule != 0 && !(d.update_scale > 0.f)))
+      return fail(MUONH_ERR_INVALID_ARG, "matrix %d: update_rule in 0..2, finite weight_decay, update_scale > 0", i);
     if (round_up(std::min(d.rows, d.cols), kPad) > kMaxRPad)
       return fail(MUONH_ERR_UNSUPPORTED, "matrix %d: min(rows, cols) above %lld", i, (long long)kMaxRPad);
   }
@@ -387,6 +390,9 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
     md.a = d.ns_a;
     md.b = d.ns_b;
     md.c_coef = d.ns_c;
+    md.rule = d.update_rule;
+    md.wd = d.weight_decay;
+    md.uscale = d.update_rule == 0 ? 1.f : d.update_scale;
     scale_exponents(d.ns_a, d.ns_b, d.ns_c, d.ns_steps, ctx->prec, &md.ex, &md.ea, &md.ec, &md.eb);
     if (md.transposed) {
       md.et_th = md.et_tw = kEwTile;

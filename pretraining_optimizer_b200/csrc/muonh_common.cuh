@@ -61,6 +61,8 @@ struct MatDev {
   int32_t ns_steps;
   float a, b, c_coef;
   int32_t ex, ea, ec, eb;    // power-of-two scales of stored X, A, C, B'
+  int32_t rule;              // MUONH_RULE_*
+  float wd, uscale;          // ordinary-Muon weight decay and update scale
   int32_t et_rows, et_cols;  // elementwise tile grid
   int32_t et_th, et_tw;      // elementwise tile shape: 64 x 64 for tall W, <= 8 x 512 rows otherwise
   int64_t et_begin;          // first elementwise tile

@@ -666,13 +666,23 @@ __global__ void __launch_bounds__(kEwThreads) finalize_update_kernel(const EwPar
       sc.mode = 2;
     } else if (oo == 0.0) {
       sc.flags |= MUONH_FLAG_ZERO_UPDATE;
-      if (wn > 0.0) {
+      if (md.rule != MUONH_RULE_HYPERBALL) {
+        sc.mode = 2;   // ordinary Muon: no update, W kept
+      } else if (wn > 0.0) {
         sc.mode = 1;
         sc.kw = static_cast<float>(R / wn);
       } else {
         sc.flags |= MUONH_FLAG_DEGENERATE;
         sc.mode = 2;
       }
+    } else if (md.rule != MUONH_RULE_HYPERBALL) {
+      // Eq. (3): eta = lr; Eq. (5): eta = lr ||W|| / ||u||; W <- (1 - wd eta) W - eta u, u = s O
+      const double un = static_cast<double>(md.uscale) * on;
+      const double eta = (md.rule == MUONH_RULE_DECOUPLED_WD) ? lr : lr * wn / un;
+      sc.mode = 0;
+      sc.kw = static_cast<float>(1.0 - static_cast<double>(md.wd) * eta);
+      sc.ko = static_cast<float>(-eta * static_cast<double>(md.uscale) * unscale);
+      elr = wn > 0.0 ? eta * un / wn : 0.0;
     } else {
       const double alpha = lr * R / on;
       const double wt2 = wn2 - 2.0 * alpha * wo + alpha * alpha * oo;

@@ -13,6 +13,8 @@ from ctypes import POINTER, Structure, c_char_p, c_float, c_int32, c_int64, c_si
 QUINTIC = (3.4445, -4.7750, 2.0315)
 NS_FP16, NS_BF16, NS_FP32 = 0, 1, 2
 _PREC = {"fp16": NS_FP16, "bf16": NS_BF16, "fp32": NS_FP32}
+RULE_HYPERBALL, RULE_DECOUPLED_WD, RULE_ELR_ALIGNED = 0, 1, 2
+_RULE = {"hyperball": RULE_HYPERBALL, "decoupled_wd": RULE_DECOUPLED_WD, "elr_aligned": RULE_ELR_ALIGNED}
 FLAG_NONFINITE_INPUT = 1
 FLAG_ZERO_UPDATE = 2
 FLAG_NONFINITE_UPDATE = 4
@@ -22,9 +24,12 @@ FLAG_TIMEOUT = 16
 EXPORTED_SYMBOLS = (
     "muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
     "muonh_export_state", "muonh_import_state", "muonh_device_status", "muonh_last_launch_count",
-    "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc", "muonh_destroy",
-    "muonh_status_string", "muonh_last_error",
+    "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc", "muonh_average",
+    "muonh_adamw_step", "muonh_destroy", "muonh_status_string", "muonh_last_error",
 )
+DTYPE_F32, DTYPE_BF16 = 0, 1
+AVERAGE_MAX_INPUTS = 16
+ADAMW_MAX_TENSORS = 32
 PHASES = ("momentum_norm", "finalize_input", "write_x", "ns_gram", "ns_square", "ns_apply",
           "update_dots", "finalize_update", "project", "finalize_step")
 
@@ -32,7 +37,8 @@ PHASES = ("momentum_norm", "finalize_input", "write_x", "ns_gram", "ns_square", 
 class MatrixDesc(Structure):
     _fields_ = [("w", c_void_p), ("m", c_void_p), ("rows", c_int64), ("cols", c_int64),
                 ("ld", c_int64), ("radius", c_float), ("beta", c_float), ("nesterov", c_int32),
-                ("ns_steps", c_int32), ("ns_a", c_float), ("ns_b", c_float), ("ns_c", c_float)]
+                ("ns_steps", c_int32), ("ns_a", c_float), ("ns_b", c_float), ("ns_c", c_float),
+                ("update_rule", c_int32), ("weight_decay", c_float), ("update_scale", c_float)]
 
 
 class Config(Structure):
@@ -42,6 +48,15 @@ class Config(Structure):
 class Stats(Structure):
     _fields_ = [("elr", c_float), ("pre_norm", c_float), ("post_norm", c_float),
                 ("update_norm", c_float), ("input_norm", c_float), ("flags", c_uint32)]
+
+
+class AdamWTensor(Structure):
+    _fields_ = [("p", c_void_p), ("m", c_void_p), ("v", c_void_p), ("g", c_void_p), ("count", c_int64)]
+
+
+class AdamWConfig(Structure):
+    _fields_ = [("lr", c_float), ("beta1", c_float), ("beta2", c_float), ("eps", c_float),
+                ("weight_decay", c_float)]
 
 
 class MuonHError(RuntimeError):
@@ -80,6 +95,8 @@ def library() -> ctypes.CDLL:
     lib.muonh_phase_times.argtypes = [c_void_p, POINTER(c_float), POINTER(c_int64)]
     lib.muonh_momentum_norm_noalloc.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_float,
                                                 c_int32, c_void_p, c_void_p]
+    lib.muonh_average.argtypes = [c_void_p, c_int32, POINTER(c_void_p), c_int32, c_int32, c_int64, c_void_p]
+    lib.muonh_adamw_step.argtypes = [POINTER(AdamWTensor), c_int32, POINTER(AdamWConfig), c_int64, c_void_p]
     lib.muonh_destroy.argtypes = [c_void_p]
     lib.muonh_destroy.restype = None
     lib.muonh_status_string.argtypes = [c_int32]
@@ -88,7 +105,8 @@ def library() -> ctypes.CDLL:
     lib.muonh_last_error.restype = c_char_p
     for name in ("muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
                  "muonh_export_state", "muonh_import_state", "muonh_device_status",
-                 "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc"):
+                 "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc",
+                 "muonh_average", "muonh_adamw_step"):
         getattr(lib, name).restype = c_int32
     _LIB = lib
     return lib
@@ -133,6 +151,60 @@ def momentum_norm_noalloc(m, g, beta=0.95, nesterov=True, x_norm=None, stream=No
     return x_norm
 
 
+def _flat_view(t, what: str, dtypes):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype not in dtypes or not t.is_contiguous():
+        raise TypeError(f"{what} must be a contiguous CUDA tensor of dtype {', '.join(map(str, dtypes))}")
+    return t.data_ptr(), t.numel()
+
+
+def average(checkpoints, out=None, stream=None):
+    """Equal average of k <= 16 same-shape fp32 or bf16 CUDA tensors,
+    (c_0 + ... + c_{k-1}) / k summed in fp32.  `out` (default: a new tensor
+    of the inputs' dtype) may be fp32 or bf16 and may be checkpoints[0]."""
+    import torch
+    dtypes = (torch.float32, torch.bfloat16)
+    checkpoints = list(checkpoints)
+    if not 1 <= len(checkpoints) <= AVERAGE_MAX_INPUTS:
+        raise ValueError(f"between 1 and {AVERAGE_MAX_INPUTS} checkpoints")
+    ptrs, count = [], None
+    for i, c in enumerate(checkpoints):
+        ptr, n = _flat_view(c, f"checkpoints[{i}]", dtypes)
+        if c.dtype != checkpoints[0].dtype or c.shape != checkpoints[0].shape or c.device != checkpoints[0].device:
+            raise ValueError("checkpoints must share dtype, shape and device")
+        ptrs.append(ptr)
+        count = n
+    if out is None:
+        out = torch.empty_like(checkpoints[0])
+    optr, on = _flat_view(out, "out", dtypes)
+    if on != count:
+        raise ValueError("out must have as many elements as each checkpoint")
+    code = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
+    arr = (c_void_p * len(ptrs))(*ptrs)
+    _check(library().muonh_average(optr, code[out.dtype], arr, code[checkpoints[0].dtype], len(ptrs), count,
+                                   _stream_handle(stream)))
+    return out
+
+
+def adamw_step(params, exp_avgs, exp_avg_sqs, grads, step, lr, beta1=0.9, beta2=0.95, eps=1e-8,
+               weight_decay=0.1, stream=None):
+    """One AdamW step (1-based `step`) over lists of fp32 CUDA tensors,
+    updated in place: params, first moments, second moments; grads read."""
+    import torch
+    lists = (list(params), list(exp_avgs), list(exp_avg_sqs), list(grads))
+    n = len(lists[0])
+    if any(len(x) != n for x in lists):
+        raise ValueError("params, exp_avgs, exp_avg_sqs and grads must have equal lengths")
+    ts = (AdamWTensor * max(n, 1))()
+    for i in range(n):
+        views = [_flat_view(x[i], f"tensor {i}", (torch.float32,)) for x in lists]
+        if len({v[1] for v in views}) != 1:
+            raise ValueError(f"tensor {i}: p, m, v and g differ in size")
+        ts[i] = AdamWTensor(views[0][0], views[1][0], views[2][0], views[3][0], views[0][1])
+    cfg = AdamWConfig(lr, beta1, beta2, eps, weight_decay)
+    _check(library().muonh_adamw_step(ts, n, ctypes.byref(cfg), int(step), _stream_handle(stream)))
+
+
 class MuonH:
     """MuonH over a list of fp32 CUDA weight matrices (updated in place).
 
@@ -140,7 +212,8 @@ class MuonH:
     (the caller applies the hyperball multiplier and the schedule)."""
 
     def __init__(self, weights, momenta=None, *, beta=0.95, nesterov=True, ns_steps=5,
-                 ns_coeffs=QUINTIC, eps=1e-7, ns_precision="fp16", radii=None, stream=None):
+                 ns_coeffs=QUINTIC, eps=1e-7, ns_precision="fp16", radii=None, stream=None,
+                 update_rule="hyperball", weight_decay=0.0, update_scale=1.0):
         import torch
         self._lib = library()
         self.weights = list(weights)
@@ -162,7 +235,12 @@ class MuonH:
             a, b, c = ns_coeffs if not isinstance(ns_coeffs[0], (tuple, list)) else ns_coeffs[i]
             steps = ns_steps if isinstance(ns_steps, int) else ns_steps[i]
             bt = beta if isinstance(beta, (int, float)) else beta[i]
-            descs[i] = MatrixDesc(wp, mp, rows, cols, ld, R, bt, int(bool(nesterov)), steps, a, b, c)
+            rule = update_rule if isinstance(update_rule, (str, int)) else update_rule[i]
+            rule = _RULE[rule] if isinstance(rule, str) else int(rule)
+            wd = weight_decay if isinstance(weight_decay, (int, float)) else weight_decay[i]
+            us = update_scale if isinstance(update_scale, (int, float)) else update_scale[i]
+            descs[i] = MatrixDesc(wp, mp, rows, cols, ld, R, bt, int(bool(nesterov)), steps, a, b, c,
+                                  rule, wd, us)
             self.shapes.append((rows, cols, ld))
         cfg = Config(prec, eps)
         ctx = c_void_p()

@@ -75,6 +75,24 @@ def qwen3_1p7b() -> list[MatrixSpec]:
     return qwen3_matrix_set(2048, 6144)
 
 
+QWEN3_VOCAB = 151936
+
+
+def qwen3_adamw_group(d_model: int, layers: int = 28, vocab: int = QWEN3_VOCAB,
+                      d_head: int = 128) -> list[tuple[str, int]]:
+    """The parameters outside the matrix set, which AdamW trains: the input
+    embedding and the (untied) LM head, vocab x d_model each; per layer the
+    two RMSNorm weights (d_model) and the q/k norms (d_head); the final norm.
+    For Qwen3-1.7B with untied head: 622,453,760 elements, which with the
+    matrix set makes the ~2.03e9 parameters of the model."""
+    out = [("embed_tokens", vocab * d_model), ("lm_head", vocab * d_model)]
+    for layer in range(layers):
+        out += [(f"layers.{layer}.input_layernorm", d_model), (f"layers.{layer}.post_attention_layernorm", d_model),
+                (f"layers.{layer}.q_norm", d_head), (f"layers.{layer}.k_norm", d_head)]
+    out.append(("norm", d_model))
+    return out
+
+
 def single_256x512() -> list[MatrixSpec]:
     return [MatrixSpec("w", 256, 512)]
 

@@ -18,7 +18,8 @@ def rel_fro(a, b):
 
 
 def run_gpu(W0, grad_fn, lrs, *, prec="fp16", ns_steps=5, coeffs=oracle.QUINTIC, beta=0.95,
-            nesterov=True, eps=1e-7, keep_updates=(), radii=None, strides=None):
+            nesterov=True, eps=1e-7, keep_updates=(), radii=None, strides=None, rule="hyperball",
+            weight_decay=0.0, update_scale=1.0):
     """Run len(lrs) steps through the C-ABI; returns W, M (numpy fp32), per-step stats,
     and {step: [O_i]} for the steps listed in keep_updates."""
     import torch
@@ -36,7 +37,8 @@ def run_gpu(W0, grad_fn, lrs, *, prec="fp16", ns_steps=5, coeffs=oracle.QUINTIC,
     W = [place(w, i) for i, w in enumerate(W0)]
     M = [place(np.zeros_like(w), i) for i, w in enumerate(W0)]
     opt = MuonH(W, M, beta=beta, nesterov=nesterov, ns_steps=ns_steps, ns_coeffs=coeffs, eps=eps,
-                ns_precision=prec, radii=radii)
+                ns_precision=prec, radii=radii, update_rule=rule, weight_decay=weight_decay,
+                update_scale=update_scale)
     stats, updates = [], {}
     for t, lr in enumerate(lrs):
         G = [place(grad_fn(t, i), i) for i in range(len(W0))]
@@ -53,7 +55,10 @@ def run_gpu(W0, grad_fn, lrs, *, prec="fp16", ns_steps=5, coeffs=oracle.QUINTIC,
 
 
 def run_oracle(W0, grad_fn, lrs, *, ns_steps=5, coeffs=oracle.QUINTIC, beta=0.95, nesterov=True,
-               eps=1e-7, keep_updates=(), R_list=None):
+               eps=1e-7, keep_updates=(), R_list=None, rule="hyperball", weight_decay=0.0,
+               update_scale=1.0):
+    rule_id = {"hyperball": oracle.RULE_HYPERBALL, "decoupled_wd": oracle.RULE_DECOUPLED_WD,
+               "elr_aligned": oracle.RULE_ELR_ALIGNED}[rule]
     W = [np.asarray(w, dtype=np.float64) for w in W0]
     M = [np.zeros_like(w) for w in W]
     R = list(R_list) if R_list is not None else [oracle.radius(w) for w in W]
@@ -63,7 +68,8 @@ def run_oracle(W0, grad_fn, lrs, *, ns_steps=5, coeffs=oracle.QUINTIC, beta=0.95
         for i in range(len(W)):
             lri = lr[i] if isinstance(lr, (list, tuple)) else lr
             W[i], M[i], O, st = oracle.muonh_step(W[i], M[i], grad_fn(t, i), lri, R[i], beta, nesterov,
-                                                  ns_steps, coeffs, eps)
+                                                  ns_steps, coeffs, eps, rule=rule_id,
+                                                  weight_decay=weight_decay, update_scale=update_scale)
             st_t.append(st)
             O_t.append(O)
         stats.append(st_t)

@@ -28,10 +28,11 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_struct_layouts_match_the_header():
-    assert ctypes.sizeof(B.MatrixDesc) == 72
+    assert ctypes.sizeof(B.MatrixDesc) == 80
     assert ctypes.sizeof(B.Config) == 8
     assert ctypes.sizeof(B.Stats) == 24
     assert B.MatrixDesc.radius.offset == 40 and B.MatrixDesc.ns_c.offset == 64
+    assert B.MatrixDesc.update_rule.offset == 68 and B.MatrixDesc.update_scale.offset == 76
 
 
 def test_status_strings_and_argument_checks_without_a_gpu():

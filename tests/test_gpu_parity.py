@@ -173,3 +173,31 @@ def test_checkpoint_resume_is_bitwise():
     torch.cuda.synchronize()
     assert np.array_equal(w_ck.cpu().numpy(), straight)
     opt.close()
+
+
+@pytest.mark.parametrize("prec,ns_tol,w_tol", [("fp16", FP16_NS_TOL, 2e-4), ("fp32", FP32_NS_TOL, 2e-6)])
+@pytest.mark.parametrize("rule", ["decoupled_wd", "elr_aligned"])
+def test_ordinary_muon_rules(rule, prec, ns_tol, w_tol):
+    """Eq. (3) (eta = lr) and Eq. (5) (eta = lr ||W||/||u||) through the same
+    kernels: a wide and a tall matrix, 5 steps, weight decay 0.1, u = 0.2 O."""
+    shapes = [(256, 512), (640, 384)]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    lrs = [0.02, 0.015, 0.01, 0.01, 0.005]
+    kw = dict(rule=rule, weight_decay=0.1, update_scale=0.2)
+    g = run_gpu(W0, grad, lrs, prec=prec, keep_updates=(4,), **kw)
+    o = run_oracle(W0, grad, lrs, keep_updates=(4,), **kw)
+    for i in range(len(shapes)):
+        assert rel_fro(g["O"][4][i], o["O"][4][i]) <= ns_tol
+        for t, lr in enumerate(lrs):
+            gs, os_ = g["stats"][t][i], o["stats"][t][i]
+            assert gs["flags"] == 0
+            assert abs(gs["pre_norm"] - os_["pre_norm"]) <= NORM_TOL * os_["pre_norm"], (t, i)
+            assert abs(gs["post_norm"] - os_["post_norm"]) <= w_tol * os_["post_norm"], (t, i)
+            if rule == "elr_aligned":
+                assert abs(gs["elr"] - lr) <= NORM_TOL * lr, (t, i, gs["elr"])     # Eq. (4) = rho
+            else:
+                assert abs(gs["elr"] - os_["elr"]) <= ns_tol * os_["elr"], (t, i)
+        # no projection: the norm moves, unlike MuonH
+        assert abs(g["stats"][4][i]["post_norm"] - o["R"][i]) > 1e-3 * o["R"][i]
+        assert np.linalg.norm(g["W"][i] - o["W"][i]) / np.linalg.norm(o["W"][i]) <= w_tol, i

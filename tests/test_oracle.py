@@ -169,3 +169,29 @@ def test_multi_step_norm_stays_on_sphere():
         assert abs(np.linalg.norm(out["W"][i]) - out["R"][i]) <= 1e-12 * out["R"][i]
         for st in out["stats"]:
             assert abs(st[i]["elr"] - 0.01) < 1e-12
+
+
+def test_ordinary_muon_rules_hand_solved():
+    """Eq. (3) and Eq. (5) of Sec. 3.3.1 on hand-solved cases."""
+    rows = _golden_rows("muon_rules_two_element.txt")
+    assert len(rows) == 3
+    for (rule, lr, lam, s), (n0, n1, elr, eta) in rows:
+        W_new, st = oracle.muon_update(np.array([[3.0, 4.0]]), np.array([[0.0, 2.0]]), lr, lam, s, int(rule))
+        assert np.allclose(W_new, [[n0, n1]], rtol=0, atol=1e-14)
+        assert abs(st["elr"] - elr) < 1e-15 and abs(st["eta"] - eta) < 1e-15
+
+
+def test_elr_aligned_rule_hits_the_prescribed_elr():
+    """Eq. (5): the induced effective LR (Eq. (4)) equals rho for any update
+    scale, and the step direction is the Eq. (3) direction at that eta."""
+    rng = np.random.default_rng(9)
+    for scale in (1.0, 0.2, 37.0):
+        W = 0.02 * rng.standard_normal((24, 60))
+        G = 1e-3 * rng.standard_normal((24, 60))
+        W1, _, O, st = oracle.muonh_step(W, np.zeros_like(W), G, 0.015, 0.0, rule=oracle.RULE_ELR_ALIGNED,
+                                         weight_decay=0.1, update_scale=scale)
+        assert abs(st["elr"] - 0.015) < 1e-14
+        W3, st3 = oracle.muon_update(W, O, st["eta"], 0.1, scale, oracle.RULE_DECOUPLED_WD)
+        assert np.allclose(W1, W3, rtol=0, atol=1e-15)
+        # no projection: the norm drifts from ||W_0||
+        assert abs(np.linalg.norm(W1) - np.linalg.norm(W)) > 1e-6

@@ -21,6 +21,8 @@ MUTATIONS = {
     "max-norm input scaling": ("Y = Y / (np.linalg.norm(Y) + eps)", "Y = Y / (np.abs(Y).max() + eps)"),
     "ELR over R": ("elr = float(np.linalg.norm(displacement)) / w_norm",
                    "elr = float(np.linalg.norm(displacement)) / R"),
+    "Eq. (5) without the update scale": ("else lr * w_norm / u_norm", "else lr * w_norm / o_norm"),
+    "Eq. (3) without weight decay": ("W_new = (1.0 - weight_decay * eta) * W - eta * u", "W_new = W - eta * u"),
 }
 
 
