@@ -384,9 +384,11 @@ def run_ours(args):
     for name, (tms, cnt) in phases.items():
         if cnt == 0:
             continue
-        entry = {"ms_per_launch": tms / cnt, "launches": cnt, "share": tms / sum(v[0] for v in phases.values())}
+        # a phase may take more than one launch a step (wide and tall tiles)
+        entry = {"ms_per_step": tms / args.steps, "launches_per_step": cnt / args.steps,
+                 "ms_per_launch": tms / cnt, "share": tms / sum(v[0] for v in phases.values())}
         if name in KERNEL_BYTES:
-            entry["gbps"] = KERNEL_BYTES[name] * elems / (tms / cnt / 1000.0) / 1e9
+            entry["gbps"] = KERNEL_BYTES[name] * elems / (tms / args.steps / 1000.0) / 1e9
         kernels[name] = entry
     apply_ms, apply_n = phases["ns_apply"]
     ap_flops = apply_flops(shapes)

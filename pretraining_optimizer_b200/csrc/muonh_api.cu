@@ -159,6 +159,11 @@ struct muonh_ctx {
   CUtensorMap* d_wmaps = nullptr;  // per matrix fp32 W tiles (fused matrices)
   int64_t n_ns_slots = 0;
   bool any_unfused = true;
+  bool any_warp_tiled = false;     // matrices handled by the warp-tiled momentum/project kernels
+  bool any_wt[2] = {false, false}; // ... among them wide (0) and tall (1) ones
+  bool any_general = true;         // matrices handled by the general ones
+  int ew_warp_grid[4] = {148, 148, 148, 148};   // blocks of the warp-tiled kernels (one wave each)
+  float* d_part8 = nullptr;
   CUtensorMap* d_tmaps = nullptr;
   int* d_err = nullptr;
 
@@ -196,6 +201,7 @@ struct muonh_ctx {
     p.n_et = n_et;
     p.part = d_part;
     p.part64 = d_part64;
+    p.part8 = d_part8;
     p.part_ns = d_part_ns;
     p.n = n;
     p.eps = eps;
@@ -355,6 +361,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   ctx->eps = cfg->eps;
   ctx->device = dev;
   ctx->sm_count = prop.multiProcessorCount;
+  for (int k = 0; k < 4; ++k) ctx->ew_warp_grid[k] = ctx->sm_count * ew_warp_blocks_per_sm(k);
   ctx->pairs = cfg->ns_precision != P_FP32;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ctx->last_stream = s;
@@ -384,6 +391,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
     md.c = static_cast<int32_t>(std::max(d.rows, d.cols));
     md.transposed = d.rows > d.cols ? 1 : 0;
     md.vec = (d.cols % 4 == 0 && d.ld % 4 == 0) ? 1 : 0;
+    md.warp_tiled = (md.vec && ctx->prec != P_FP32) ? 1 : 0;
     md.beta = d.beta;
     md.nesterov = d.nesterov ? 1 : 0;
     md.ns_steps = d.ns_steps;
@@ -429,13 +437,20 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
     md.fused_dots = (ctx->pairs && md.vec && md.ns_steps > 0 && md.ns_steps == ctx->max_steps) ? 1 : 0;
     md.ns_tiles_bj = ch.c_pad / kBN;
     if (md.fused_dots) {
-      md.ns_slots = 2 * (ch.r_pad / (2 * kBM)) * md.ns_tiles_bj;
+      md.ns_slots = 8 * (ch.r_pad / (2 * kBM)) * md.ns_tiles_bj;   // per pair tile: 2 CTAs x 4 epilogue warps
       md.ns_slot_base = ctx->n_ns_slots;
       ctx->n_ns_slots += md.ns_slots;
     }
   }
   ctx->any_unfused = false;
-  for (int32_t i = 0; i < n; ++i) ctx->any_unfused |= !ctx->mats[i].fused_dots;
+  ctx->any_warp_tiled = false;
+  ctx->any_general = false;
+  for (int32_t i = 0; i < n; ++i) {
+    ctx->any_unfused |= !ctx->mats[i].fused_dots;
+    ctx->any_warp_tiled |= ctx->mats[i].warp_tiled != 0;
+    if (ctx->mats[i].warp_tiled) ctx->any_wt[ctx->mats[i].transposed ? 1 : 0] = true;
+    ctx->any_general |= ctx->mats[i].warp_tiled == 0;
+  }
 
   // ---- workspace
   const int parts = ctx->prec == P_FP32 ? 2 : 1;
@@ -454,12 +469,13 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", xb);
         CUDA_TRY(cudaMemsetAsync(cd.x[buf][part], 0, xb, s));
       }
-      if (dev_alloc(ctx, &cd.a[part], ab) != cudaSuccess || dev_alloc(ctx, &cd.c[part], ab) != cudaSuccess ||
-          dev_alloc(ctx, &cd.b[part], ab) != cudaSuccess)
+      // C = b I + c A is a separate operand of the FP32-mode kernel only
+      if (dev_alloc(ctx, &cd.a[part], ab) != cudaSuccess || dev_alloc(ctx, &cd.b[part], ab) != cudaSuccess ||
+          (!ctx->pairs && dev_alloc(ctx, &cd.c[part], ab) != cudaSuccess))
         return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", ab);
       CUDA_TRY(cudaMemsetAsync(cd.a[part], 0, ab, s));
-      CUDA_TRY(cudaMemsetAsync(cd.c[part], 0, ab, s));
       CUDA_TRY(cudaMemsetAsync(cd.b[part], 0, ab, s));
+      if (!ctx->pairs) CUDA_TRY(cudaMemsetAsync(cd.c[part], 0, ab, s));
     }
   }
 
@@ -480,27 +496,24 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           return st;
         if ((st = encode_map(&m[tm_x(TM_X_MN, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBK)))
           return st;
-        if (part == 0 && (st = encode_map(&m[TM_X_ST + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count, kBM, 32,
+        if (part == 0 && (st = encode_map(&m[TM_X_ST + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count, 32, 32,
                                           CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
       }
       muonh_status st;
       if ((st = encode_map(&m[TM_A_K128 + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
-      if ((st = encode_map(&m[TM_C_K256 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN))) return st;
       if ((st = encode_map(&m[TM_B_K128 + part], cd.b[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
-      if ((st = encode_map(&m[TM_C_K128 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
-      if ((st = encode_map(&m[TM_A_MN + part], cd.a[part], bf, cd.r_pad, cd.r_pad, cd.count, kBK))) return st;
-      if ((st = encode_map(&m[TM_C_MN + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBK))) return st;
-      if ((st = encode_map(&m[TM_B_MN + part], cd.b[part], bf, cd.r_pad, cd.r_pad, cd.count, kBK))) return st;
-      if (part == 0) {
-        if ((st = encode_map(&m[TM_A_ST], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+      if (!ctx->pairs &&
+          (st = encode_map(&m[TM_C_K256 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN)))
+        return st;
+      if (part == 0 && ctx->pairs) {
+        // epilogue store boxes: 32 rows x 32 columns, one per epilogue warp
+        if ((st = encode_map(&m[TM_A_ST], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
-        if ((st = encode_map(&m[TM_C_ST], cd.c[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+        if ((st = encode_map(&m[TM_B_ST], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
-        if ((st = encode_map(&m[TM_B_ST], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
-          return st;
-        if ((st = encode_map(&m[TM_B_MIR], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 64,
-                             CU_TENSOR_MAP_SWIZZLE_128B)))
+        // SQUARE epilogue: A chunks of 128 rows x 32 columns
+        if ((st = encode_map(&m[TM_A_EPI], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, 128, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
       }
     }
@@ -516,6 +529,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_et_mat), n_et * sizeof(int32_t)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part), 2 * n_et * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part64), n_et * sizeof(double)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part8), kStreamSlots * n_et * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part_ns),
                 std::max<int64_t>(1, 2 * ctx->n_ns_slots) * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_wmaps), n * sizeof(CUtensorMap)) != cudaSuccess ||
@@ -642,7 +656,11 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
   const EwParams p = ctx->ew(stats);
   const int grid = ctx->sm_count * 8;
   int launches = 0;
-  STEP_LAUNCH(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_norm(p, grid, s), "momentum_norm");
+  for (int tall = 0; tall < 2; ++tall)
+    if (ctx->any_wt[tall])
+      STEP_LAUNCH(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_warp(p, tall != 0, ctx->ew_warp_grid[tall], s),
+                  "momentum_warp");
+  if (ctx->any_general) STEP_LAUNCH(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_norm(p, grid, s), "momentum_norm");
   STEP_LAUNCH(MUONH_PHASE_FINALIZE_INPUT, launch_finalize_input(p, s), "finalize_input");
   STEP_LAUNCH(MUONH_PHASE_WRITE_X, launch_write_x(p, grid, s), "write_x");
   for (int32_t k = 0; k < ctx->max_steps; ++k) {
@@ -682,7 +700,11 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
   }
   if (ctx->any_unfused) STEP_LAUNCH(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, s), "update_dots");
   STEP_LAUNCH(MUONH_PHASE_FINALIZE_UPDATE, launch_finalize_update(p, s), "finalize_update");
-  STEP_LAUNCH(MUONH_PHASE_PROJECT, launch_project(p, grid, s), "project");
+  for (int tall = 0; tall < 2; ++tall)
+    if (ctx->any_wt[tall])
+      STEP_LAUNCH(MUONH_PHASE_PROJECT, launch_project_warp(p, tall != 0, ctx->ew_warp_grid[2 + tall], s),
+                  "project_warp");
+  if (ctx->any_general) STEP_LAUNCH(MUONH_PHASE_PROJECT, launch_project(p, grid, s), "project");
   STEP_LAUNCH(MUONH_PHASE_FINALIZE_STEP, launch_finalize_step(p, s), "finalize_step");
   ctx->last_launches = launches;
   ctx->last_stream = s;

@@ -27,24 +27,21 @@ enum Prec { P_FP16 = 0, P_BF16 = 1, P_FP32 = 2 };
 enum Mode { M_GRAM = 0, M_SQUARE = 1, M_APPLY = 2, M_APPLY_LAST = 3 };   // LAST: also ||O||^2, <W, O>
 
 // Tensor-map slots of one shape class.  "hi" buffers hold the 16-bit
-// operand (fp16/bf16), "lo" buffers the fp16 residual in FP32 mode.
+// operand (fp16/bf16), "lo" buffers the fp16 residual in FP32 mode.  The
+// CTA-pair kernels (16-bit operands) use the store boxes and TM_A_EPI; the
+// FP32-mode kernel stores directly and also reads C = b I + c A.
 enum TmSlot {
   TM_X_K128 = 0,   // X[buf] as K-major operand, 128-row box   (+buf, +2*part)
   TM_X_K256 = 4,   // X[buf] as K-major operand, 256-row box
   TM_X_MN = 8,     // X[buf] as MN-major operand, 64 x 64 box
   TM_A_K128 = 12,  // A, 128-row box (+part)
-  TM_C_K256 = 14,  // C = b I + c A, 256-row box (+part)
-  TM_B_K128 = 16,  // B' = a I + A C, 128-row box (+part)
-  TM_C_K128 = 18,  // C, 128-row box (+part): B operand half of a CTA pair
-  TM_A_MN = 20,    // A, 64 x 64 box: a below-diagonal block read through its stored transpose
-  TM_C_MN = 22,    // C, 64 x 64 box
-  TM_B_MN = 24,    // B', 64 x 64 box
-  TM_X_ST = 26,    // X[buf] store box 32 x 128 (64-byte swizzle)   (+buf)
-  TM_A_ST = 28,    // A store box
-  TM_C_ST = 29,    // C store box
-  TM_B_ST = 30,    // B' store box
-  TM_B_MIR = 31,   // B' mirrored-store box 64 x 32 (128-byte swizzle)
-  TM_PER_CLASS = 32
+  TM_C_K256 = 14,  // C = b I + c A, 256-row box (+part), FP32 mode only
+  TM_B_K128 = 16,  // B' = a I + b A + c A A, 128-row box (+part)
+  TM_X_ST = 18,    // X[buf] store box 32 x 32 (64-byte swizzle)   (+buf)
+  TM_A_ST = 20,    // A store box (direct and mirrored blocks)
+  TM_B_ST = 21,    // B' store box (direct and mirrored blocks)
+  TM_A_EPI = 22,   // A box of 128 rows x 32 columns staged by the SQUARE epilogue (64-byte swizzle)
+  TM_PER_CLASS = 23
 };
 __host__ __device__ inline int tm_x(int base, int buf, int part) { return base + buf + 2 * part; }
 
@@ -68,8 +65,9 @@ struct MatDev {
   int64_t et_begin;          // first elementwise tile
   int32_t fused_dots;        // ||O||^2, <W, O> come from the last APPLY (else from update_dots)
   int32_t ns_tiles_bj;       // APPLY pair tiles per tile row (c_pad / 256)
-  int64_t ns_slot_base;      // first (||O||^2, <W, O>) slot: 2 per pair tile (one per CTA)
+  int64_t ns_slot_base;      // first (||O||^2, <W, O>) slot: 8 per pair tile (CTA x epilogue warp)
   int32_t ns_slots;
+  int32_t warp_tiled;        // momentum/project run in the warp-tiled kernels (partials in part8)
 };
 
 struct ClassDev {
@@ -129,6 +127,7 @@ struct EwParams {
   const int32_t* et_mat;     // elementwise tile -> matrix
   int64_t n_et;
   float* part;               // per-tile partials
+  float* part8;              // warp-tiled kernels: one partial per (tile, warp), 8 per tile
   double* part64;
   const float* part_ns;      // partials of the fused last APPLY (MatDev::fused_dots)
   int32_t n;
@@ -410,5 +409,9 @@ cudaError_t launch_finalize_update(const EwParams& p, cudaStream_t s);
 cudaError_t launch_project(const EwParams& p, int grid, cudaStream_t s);
 cudaError_t launch_finalize_step(const EwParams& p, cudaStream_t s);
 cudaError_t launch_export_update(const EwParams& p, int mat, float* dst, int64_t ld, cudaStream_t s);
+int ew_warp_blocks_per_sm(int kind);
+cudaError_t launch_momentum_warp(const EwParams& p, bool tall, int grid, cudaStream_t s);
+cudaError_t launch_project_warp(const EwParams& p, bool tall, int grid, cudaStream_t s);
+constexpr int kStreamSlots = 8;      // partial slots per tile in EwParams::part8
 
 }  // namespace muonh

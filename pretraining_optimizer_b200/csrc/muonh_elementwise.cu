@@ -240,6 +240,13 @@ __device__ __forceinline__ void store_x_tile_t(const XView& xv, const TileCoord&
   }
 }
 
+// Index of this block's last tile of matrix md (the loop increment then
+// moves past the matrix): lets the general kernels skip warp-tiled matrices.
+__device__ __forceinline__ int64_t skip_matrix(const MatDev& md, int64_t e) {
+  const int64_t end = md.et_begin + static_cast<int64_t>(md.et_rows) * md.et_cols;
+  return e + ((end - e + gridDim.x - 1) / gridDim.x - 1) * gridDim.x;
+}
+
 // ------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kEwThreads) init_norm_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
@@ -343,6 +350,10 @@ __global__ void __launch_bounds__(kEwThreads, 5) momentum_norm_kernel(const EwPa
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
+    if (md.warp_tiled) {
+      e = skip_matrix(md, e);
+      continue;
+    }
     const float* g = p.step[tc.mi].g;
     const float sigma = p.scal[tc.mi].sigma;
     const XView xv = x_view(p, md, 0);
@@ -522,6 +533,10 @@ __global__ void __launch_bounds__(kEwThreads, 6) project_kernel(const EwParams p
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
+    if (md.warp_tiled) {
+      e = skip_matrix(md, e);
+      continue;
+    }
     const MatScal& sc = p.scal[tc.mi];
     const int mode = sc.mode;
     if (mode == 2) {
@@ -577,6 +592,14 @@ __device__ double matrix_sum(const T* part, int64_t begin, int64_t count, int st
   return block_sum(s, red);
 }
 
+// Sum of a matrix's per-tile partials of the momentum or project phase: 8
+// slots per tile from the warp-tiled kernels, one from the general ones.
+__device__ double tile_partials(const EwParams& p, const MatDev& md, double* red) {
+  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
+  if (md.warp_tiled) return matrix_sum(p.part8, md.et_begin * kStreamSlots, cnt * kStreamSlots, 1, 0, red);
+  return matrix_sum(p.part, md.et_begin, cnt, 1, 0, red);
+}
+
 __global__ void __launch_bounds__(kEwThreads) finalize_init_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
   const int mi = blockIdx.x;
@@ -594,8 +617,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwPara
   __shared__ double red[kEwThreads / 32];
   const int mi = blockIdx.x;
   const MatDev& md = p.mats[mi];
-  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
-  const double s = matrix_sum(p.part, md.et_begin, cnt, 1, 0, red);
+  const double s = tile_partials(p, md, red);
   if (threadIdx.x == 0) {
     MatScal& sc = p.scal[mi];
     sc.flags = 0u;
@@ -707,8 +729,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_step_kernel(const EwParam
   __shared__ double red[kEwThreads / 32];
   const int mi = blockIdx.x;
   const MatDev& md = p.mats[mi];
-  const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
-  const double s = matrix_sum(p.part, md.et_begin, cnt, 1, 0, red);
+  const double s = tile_partials(p, md, red);
   if (threadIdx.x == 0) {
     MatScal& sc = p.scal[mi];
     if (sc.mode != 2) sc.wnorm2 = s;

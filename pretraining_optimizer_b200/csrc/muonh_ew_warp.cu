@@ -1,0 +1,336 @@
+// Warp-tiled variants of the two large HBM-bound kernels of the step (sm_100a):
+//   momentum:  M <- beta M + G, X = G + beta M (Nesterov) or M, partials of
+//              ||X||^2, and the 16-bit Newton-Schulz input sigma X;
+//   project:   W <- kw W + ko O (Eq. (1) of the Puro-2B report, Sec. 3.3, with
+//              both normalisations folded into kw and ko), partials of ||W||^2.
+//
+// A block walks elementwise tiles (4096 elements of W) in a grid-stride loop;
+// each of its 8 warps owns a fixed eighth of every tile and never waits for
+// the others: no shared memory, no block barrier.  A lane issues all of its
+// loads for a tile (8 x 16 bytes on wide tiles, 16 x 8 bytes on tall ones)
+// before the first use, so a resident warp keeps 4 KB in flight.  Tall
+// matrices, whose X is the transpose, are tiled 64 x 64: warp w takes rows
+// 8w..8w+7 with two adjacent columns per lane, so a lane holds 8 consecutive
+// entries of two X rows and writes (or, in project, reads) each as one
+// 16-byte access.
+//
+// Every warp writes its partial sum of a tile to a fixed slot (8 per tile);
+// the finalize kernels add the slots of a matrix in a fixed order in fp64, so
+// results are bitwise reproducible.  Matrices whose rows are not 16-byte
+// vectors, and the FP32 Newton-Schulz mode (hi/lo operands), take the
+// general kernels instead (MatDev::warp_tiled == 0).
+#include "muonh_common.cuh"
+
+namespace muonh {
+namespace {
+
+constexpr int kWarps = kStreamSlots;          // 8 warps, one partial slot each
+constexpr int kWarpThreads = 32 * kWarps;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float4 unpack4(uint2 u, int prec) {
+  if (prec == P_BF16) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+  }
+  const __half2 a = *reinterpret_cast<const __half2*>(&u.x);
+  const __half2 b = *reinterpret_cast<const __half2*>(&u.y);
+  return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+}
+
+// Two fp32 values to a packed pair of 16-bit values (round to nearest even).
+__device__ __forceinline__ uint32_t pack2(float a, float b, int prec) {
+  if (prec == P_BF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint16_t* x_base(const EwParams& p, const MatDev& md, int buf) {
+  const ClassDev& cd = p.classes[md.cls];
+  return static_cast<uint16_t*>(cd.x[buf][0]) + md.z * cd.x_stride;
+}
+
+struct Tile {
+  int64_t r0, c0;
+  int nr, nc;        // valid rows / columns of the tile inside the matrix
+};
+
+__device__ __forceinline__ Tile tile_of(const MatDev& md, int64_t e) {
+  Tile t;
+  const uint32_t local = static_cast<uint32_t>(e - md.et_begin);
+  const uint32_t tr = local / static_cast<uint32_t>(md.et_cols);
+  t.r0 = static_cast<int64_t>(tr) * md.et_th;
+  t.c0 = static_cast<int64_t>(local - tr * static_cast<uint32_t>(md.et_cols)) * md.et_tw;
+  t.nr = static_cast<int>(md.rows - t.r0 < md.et_th ? md.rows - t.r0 : md.et_th);
+  t.nc = static_cast<int>(md.cols - t.c0 < md.et_tw ? md.cols - t.c0 : md.et_tw);
+  return t;
+}
+
+// Next tile of this block that belongs to a warp-tiled matrix of the
+// kernel's kind (wide or tall), or n_et.
+template <bool TALL>
+__device__ __forceinline__ int64_t next_tile(const EwParams& p, int64_t e) {
+  while (e < p.n_et) {
+    const MatDev& md = p.mats[p.et_mat[e]];
+    if (md.warp_tiled && (md.transposed != 0) == TALL) return e;
+    const int64_t end = md.et_begin + static_cast<int64_t>(md.et_rows) * md.et_cols;
+    e += ((end - e + gridDim.x - 1) / gridDim.x) * gridDim.x;   // first tile of ours past this matrix
+  }
+  return e;
+}
+
+// Chunk j (0..3) of lane `lane` in warp w of a wide tile: 4 consecutive
+// columns of one row; the warp covers chunks 128w .. 128w + 127.
+__device__ __forceinline__ void wide_chunk(const MatDev& md, int w, int lane, int j, int& row, int& col) {
+  const int sh = __ffs(md.et_tw) - 3;          // log2(chunks per row) = log2(tw / 4)
+  const int q = lane + 32 * j + 128 * w;
+  row = q >> sh;
+  col = (q & ((1 << sh) - 1)) * 4;
+}
+
+// ---------------------------------------------------------------- momentum
+template <bool TALL>
+__global__ void __launch_bounds__(kWarpThreads) momentum_warp_kernel(const EwParams p) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t e = next_tile<TALL>(p, blockIdx.x); e < p.n_et; e = next_tile<TALL>(p, e + gridDim.x)) {
+    const int mi = p.et_mat[e];
+    const MatDev& md = p.mats[mi];
+    const Tile t = tile_of(md, e);
+    const float beta = md.beta;
+    const int nesterov = md.nesterov;
+    const float sigma = p.scal[mi].sigma;
+    const float* gb = p.step[mi].g + t.r0 * md.ld + t.c0;
+    float* mb = md.m + t.r0 * md.ld + t.c0;
+    uint16_t* xg = x_base(p, md, 0);
+    const int64_t xld = p.classes[md.cls].c_pad;
+    float acc = 0.f;
+    if (!TALL) {
+      int row[4], col[4];
+      bool ok[4];
+      float4 gv[4], mv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        wide_chunk(md, w, lane, j, row[j], col[j]);
+        ok[j] = row[j] < t.nr && col[j] < t.nc;
+        if (ok[j]) {
+          gv[j] = *reinterpret_cast<const float4*>(gb + row[j] * md.ld + col[j]);
+          mv[j] = *reinterpret_cast<const float4*>(mb + row[j] * md.ld + col[j]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (!ok[j]) continue;
+        float4 m = mv[j];
+        const float4 g = gv[j];
+        m.x = fmaf(beta, m.x, g.x);
+        m.y = fmaf(beta, m.y, g.y);
+        m.z = fmaf(beta, m.z, g.z);
+        m.w = fmaf(beta, m.w, g.w);
+        *reinterpret_cast<float4*>(mb + row[j] * md.ld + col[j]) = m;
+        float4 x = m;
+        if (nesterov) {
+          x.x = fmaf(beta, m.x, g.x);
+          x.y = fmaf(beta, m.y, g.y);
+          x.z = fmaf(beta, m.z, g.z);
+          x.w = fmaf(beta, m.w, g.w);
+        }
+        acc = fmaf(x.x, x.x, acc);
+        acc = fmaf(x.y, x.y, acc);
+        acc = fmaf(x.z, x.z, acc);
+        acc = fmaf(x.w, x.w, acc);
+        if (sigma > 0.f) {
+          const uint2 u = make_uint2(pack2(x.x * sigma, x.y * sigma, p.prec), pack2(x.z * sigma, x.w * sigma, p.prec));
+          *reinterpret_cast<uint2*>(xg + (t.r0 + row[j]) * xld + t.c0 + col[j]) = u;
+        }
+      }
+    } else {
+      // tall 64 x 64: warp w takes rows 8w .. 8w+7; lane l covers columns
+      // c .. c+3 (c = 4 (l mod 16)) of the even rows (l < 16) or the odd rows
+      const int half = lane >> 4;
+      const int c = 4 * (lane & 15);
+      const bool cok = c < t.nc;   // nc is a multiple of 4
+      float4 gv[4], mv[4];
+#pragma unroll
+      for (int jr = 0; jr < 4; ++jr) {
+        const int r = 8 * w + 2 * jr + half;
+        if (cok && r < t.nr) {
+          gv[jr] = *reinterpret_cast<const float4*>(gb + r * md.ld + c);
+          mv[jr] = *reinterpret_cast<const float4*>(mb + r * md.ld + c);
+        }
+      }
+      float x[4][4];
+#pragma unroll
+      for (int jr = 0; jr < 4; ++jr) {
+        const int r = 8 * w + 2 * jr + half;
+        x[jr][0] = x[jr][1] = x[jr][2] = x[jr][3] = 0.f;   // rows past the matrix stay zero in X's padding
+        if (!cok || r >= t.nr) continue;
+        float4 m = mv[jr];
+        const float4 g = gv[jr];
+        m.x = fmaf(beta, m.x, g.x);
+        m.y = fmaf(beta, m.y, g.y);
+        m.z = fmaf(beta, m.z, g.z);
+        m.w = fmaf(beta, m.w, g.w);
+        *reinterpret_cast<float4*>(mb + r * md.ld + c) = m;
+        float4 xv = m;
+        if (nesterov) {
+          xv.x = fmaf(beta, m.x, g.x);
+          xv.y = fmaf(beta, m.y, g.y);
+          xv.z = fmaf(beta, m.z, g.z);
+          xv.w = fmaf(beta, m.w, g.w);
+        }
+        acc = fmaf(xv.x, xv.x, fmaf(xv.y, xv.y, fmaf(xv.z, xv.z, fmaf(xv.w, xv.w, acc))));
+        x[jr][0] = xv.x * sigma;
+        x[jr][1] = xv.y * sigma;
+        x[jr][2] = xv.z * sigma;
+        x[jr][3] = xv.w * sigma;
+      }
+      // X row c + k holds rows 8w .. 8w+7 of column k: the even-row lane
+      // writes columns c, c+1 and the odd-row lane (lane ^ 16) columns c+2,
+      // c+3, each taking the other's half of the rows by one exchange
+      float y[4][2];
+#pragma unroll
+      for (int jr = 0; jr < 4; ++jr)
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          y[jr][k] = __shfl_xor_sync(0xffffffffu, half ? x[jr][k] : x[jr][2 + k], 16);
+      if (sigma > 0.f && cok) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int kc = 2 * half + k;   // column of this X row inside the lane's four
+          uint32_t h[4];
+#pragma unroll
+          for (int jr = 0; jr < 4; ++jr) {   // rows 8w + 2jr (even) and 8w + 2jr + 1 (odd)
+            const float own = half ? x[jr][2 + k] : x[jr][k];
+            h[jr] = half ? pack2(y[jr][k], own, p.prec) : pack2(own, y[jr][k], p.prec);
+          }
+          *reinterpret_cast<uint4*>(xg + (t.c0 + c + kc) * xld + t.r0 + 8 * w) = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+      }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) p.part8[e * kWarps + w] = acc;
+  }
+}
+
+// ----------------------------------------------------------------- project
+template <bool TALL>
+__global__ void __launch_bounds__(kWarpThreads) project_warp_kernel(const EwParams p) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t e = next_tile<TALL>(p, blockIdx.x); e < p.n_et; e = next_tile<TALL>(p, e + gridDim.x)) {
+    const int mi = p.et_mat[e];
+    const MatDev& md = p.mats[mi];
+    const MatScal& sc = p.scal[mi];
+    const int mode = sc.mode;
+    float acc = 0.f;
+    if (mode != 2) {
+      const float kw = sc.kw, ko = sc.ko;
+      const Tile t = tile_of(md, e);
+      float* wb = md.w + t.r0 * md.ld + t.c0;
+      const uint16_t* xg = x_base(p, md, md.ns_steps & 1);
+      const int64_t xld = p.classes[md.cls].c_pad;
+      if (!TALL) {
+        int row[4], col[4];
+        bool ok[4];
+        float4 wv[4];
+        uint2 ov[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          wide_chunk(md, w, lane, j, row[j], col[j]);
+          ok[j] = row[j] < t.nr && col[j] < t.nc;
+          ov[j] = make_uint2(0u, 0u);
+          if (ok[j]) {
+            wv[j] = *reinterpret_cast<const float4*>(wb + row[j] * md.ld + col[j]);
+            if (mode == 0) ov[j] = *reinterpret_cast<const uint2*>(xg + (t.r0 + row[j]) * xld + t.c0 + col[j]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (!ok[j]) continue;
+          const float4 o = unpack4(ov[j], p.prec);
+          float4 v = wv[j];
+          v.x = fmaf(ko, o.x, kw * v.x);
+          v.y = fmaf(ko, o.y, kw * v.y);
+          v.z = fmaf(ko, o.z, kw * v.z);
+          v.w = fmaf(ko, o.w, kw * v.w);
+          *reinterpret_cast<float4*>(wb + row[j] * md.ld + col[j]) = v;
+          acc = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, acc))));
+        }
+      } else {
+        const int c = 2 * lane;
+        const bool cok = c < t.nc;
+        float2 wv[8];
+        uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
+        if (cok && mode == 0) {
+          // O(8w + i, c) = X[c0 + c][r0 + 8w + i]: 8 consecutive entries of two X rows
+          const uint16_t* src = xg + (t.c0 + c) * xld + t.r0 + 8 * w;
+          o0 = *reinterpret_cast<const uint4*>(src);
+          o1 = *reinterpret_cast<const uint4*>(src + xld);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 8 * w + i;
+          if (cok && r < t.nr) wv[i] = *reinterpret_cast<const float2*>(wb + r * md.ld + c);
+        }
+        const float4 a0 = unpack4(make_uint2(o0.x, o0.y), p.prec), a1 = unpack4(make_uint2(o0.z, o0.w), p.prec);
+        const float4 b0 = unpack4(make_uint2(o1.x, o1.y), p.prec), b1 = unpack4(make_uint2(o1.z, o1.w), p.prec);
+        const float oa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float ob[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 8 * w + i;
+          if (!cok || r >= t.nr) continue;
+          float2 v = wv[i];
+          v.x = fmaf(ko, oa[i], kw * v.x);
+          v.y = fmaf(ko, ob[i], kw * v.y);
+          *reinterpret_cast<float2*>(wb + r * md.ld + c) = v;
+          acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
+        }
+      }
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) p.part8[e * kWarps + w] = acc;
+  }
+}
+
+}  // namespace
+
+// Resident blocks per SM of a warp-tiled kernel: kind 0/1 momentum wide/tall,
+// 2/3 project wide/tall.
+int ew_warp_blocks_per_sm(int kind) {
+  int n = 0;
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (kind) {
+    case 0: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, momentum_warp_kernel<false>, kWarpThreads, 0); break;
+    case 1: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, momentum_warp_kernel<true>, kWarpThreads, 0); break;
+    case 2: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, project_warp_kernel<false>, kWarpThreads, 0); break;
+    case 3: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, project_warp_kernel<true>, kWarpThreads, 0); break;
+  }
+  return (e == cudaSuccess && n > 0) ? n : 1;
+}
+
+cudaError_t launch_momentum_warp(const EwParams& p, bool tall, int grid, cudaStream_t s) {
+  if (tall)
+    momentum_warp_kernel<true><<<grid, kWarpThreads, 0, s>>>(p);
+  else
+    momentum_warp_kernel<false><<<grid, kWarpThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_project_warp(const EwParams& p, bool tall, int grid, cudaStream_t s) {
+  if (tall)
+    project_warp_kernel<true><<<grid, kWarpThreads, 0, s>>>(p);
+  else
+    project_warp_kernel<false><<<grid, kWarpThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace muonh

@@ -4,14 +4,15 @@
 //   Y' = a Y + (b A + c A A) Y,   A = Y Y^T
 // (quintic iteration of the Muon update; the MuonH wrapper of the Puro-2B
 // report, Sec. 3.3, normalises its output), runs as three products with the
-// polynomial folded into the operands so that no epilogue reads memory:
-//   GRAM    A  = Y Y^T,  and  C = b I + c A      M = r, N = r, K = c   (symmetric)
-//   SQUARE  B' = A C + a I                       M = r, N = r, K = r   (symmetric)
-//   APPLY   Y' = B' Y                            M = r, N = c, K = r
+// polynomial folded into the products:
+//   GRAM    A  = Y Y^T  (and, FP32 mode, C = b I + c A)    M = r, N = r, K = c   (symmetric)
+//   SQUARE  B' = c A A + b A + a I  (FP32 mode: A C + a I)  M = r, N = r, K = r   (symmetric)
+//   APPLY   Y' = B' Y                                      M = r, N = c, K = r
 // Every launch covers the tiles of all matrices of the step (grouped), in a
-// persistent grid of one CTA per SM.  Symmetric products compute only the
-// 128 x 256 tiles that touch the upper triangle and write each element of
-// the upper triangle once directly and once mirrored.
+// persistent grid of one CTA per SM (one CTA pair per two SMs for 16-bit
+// operands).  Symmetric products compute only the tiles that touch the upper
+// triangle and store each off-diagonal block twice, directly and mirrored,
+// so that every consumer reads its operands K-major.
 //
 // Per CTA: warp 0 issues TMA loads into a ring of shared-memory stages,
 // warp 1 (one thread) issues tcgen05.mma into one of two TMEM accumulators
@@ -445,90 +446,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 // the leader's commits arrive on the matching barriers of both CTAs.  Each
 // CTA drains its own TMEM (its 128 rows) in the epilogue.
 //
-// Symmetric results (A, C, B') are stored as whole 256 x 256 tiles of the
-// upper block triangle only.  A consumer that needs a block below the
-// diagonal loads the stored transposed block and hands it to the MMA as an
-// MN-major operand, so no epilogue writes a mirrored copy.
+// Symmetric results (A, C, B') are computed on the 256 x 256 tiles of the
+// upper block triangle; the epilogue of an off-diagonal tile also writes its
+// transpose (a warp-level 32 x 32 transpose per store box), so SQUARE and
+// APPLY read A, C and B' as K-major operands.  (Reading a lower block
+// through its stored transpose as an MN-major operand instead ran SQUARE
+// about 30% slower on B200.)
 template <int PREC, int MODE>
 struct PairCfg {
-  // the last APPLY gives one pipeline stage to the fp32 W staging buffers
+  // the last APPLY gives staging space to the fp32 W boxes of its <W, O> partials
   static constexpr bool kLast = MODE == M_APPLY_LAST;
-  static constexpr int kStages = kLast ? 5 : 6;
+  static constexpr bool kSquare = MODE == M_SQUARE;
+  // SQUARE trades an operand stage for deeper staging of its epilogue A boxes
+  static constexpr int kStages = kSquare ? 4 : 5;
+  static constexpr int kWBufs = kSquare ? 4 : 2;
   static constexpr int kABytes = 128 * kBK * 2;                 // 16 KB: this CTA's 128 rows
   static constexpr int kBBytes = 128 * kBK * 2;                 // 16 KB: this CTA's half of N
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = kStages * kStageBytes;
-  // SQUARE epilogue: per-warp 32 x 32 16-bit staging block for the mirrored
-  // copy of B' (rows padded to 80 bytes: conflict-free 16-byte stores and
-  // 2-byte column reads)
+  // Epilogue warps: one per TMEM lane quarter
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  // per-epilogue-warp 32 x 32 16-bit scratch for the mirrored copies (rows
+  // padded to 80 bytes: conflict-free 16-byte stores and 2-byte column reads)
   static constexpr int kMirrorStride = 80;
   static constexpr int kMirrorOffset = kBarOffset + 256;
-  static constexpr int kMirrorBytes = 4 * 32 * kMirrorStride;
-  // Epilogue output staging: two 128-row x 32-column 16-bit boxes written
-  // to global memory by TMA stores (64-byte swizzle)
-  static constexpr int kStoreBox = 128 * 32 * 2;
+  static constexpr int kMirrorBytes = kEpiWarps * 32 * kMirrorStride;
+  // Epilogue output staging: each epilogue warp owns kWarpBufs boxes of
+  // 32 rows x 32 columns (16-bit, 64-byte swizzle) that it writes to global
+  // memory with its own TMA stores
+  static constexpr int kWarpBox = 32 * 32 * 2;
+  static constexpr int kWarpBufs = kLast ? 2 : 4;
   static constexpr int kStoreOffset = (kMirrorOffset + kMirrorBytes + 1023) / 1024 * 1024;
-  // Last APPLY: two fp32 W boxes (128 rows x 32 columns, or 32 x 128 for
-  // a tall W) loaded by TMA for the <W, O> partials
-  static constexpr int kWBox = 128 * 32 * 4;
-  static constexpr int kWOffset = kStoreOffset + 2 * kStoreBox;
-  static constexpr int kSmem = kWOffset + (kLast ? 2 * kWBox : 0) + 1024;
+  // Epilogue operand staging, kWBufs buffers filled kWBufs chunks ahead: the
+  // last APPLY's fp32 W boxes (128 rows x 32 columns, or 32 x 128 for a tall
+  // W) for the <W, O> partials; SQUARE's 16-bit A boxes (128 rows x 32
+  // columns, 64-byte swizzle) for its b A term
+  static constexpr int kWBox = kLast ? 128 * 32 * 4 : 128 * 32 * 2;
+  static constexpr int kWOffset = kStoreOffset + kEpiWarps * kWarpBufs * kWarpBox;
+  static constexpr int kSmem = kWOffset + ((kLast || kSquare) ? kWBufs * kWBox : 0) + 1024;
 };
 
-// Epilogue row `r` (0..127) of a 128 x 32 16-bit box, 16-byte piece q,
-// in the 64-byte swizzle pattern of the TMA store box.
+// Row `r` (0..31) of a 32 x 32 16-bit box, 16-byte piece q, in the 64-byte
+// swizzle pattern of the TMA store box.
 __device__ __forceinline__ uint32_t store_box_offset(int r, int q) {
   return static_cast<uint32_t>(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
 }
 
-// Double-buffered TMA-store staging shared by the 128 epilogue threads; each
-// 8 KB buffer holds either one 128-row x 32-column box of a tile (64-byte
-// swizzle) or the transposed 32-row x 128-column block of a mirrored store
-// (two 64-column halves, 128-byte swizzle).
-struct StoreStager {
+// TMA-store staging private to one epilogue warp: lane j supplies row j of
+// a 32 x 32 box; lane 0 issues the store.  A buffer is reused only after the
+// store issued from it kBufs puts earlier has read it, so the warps never
+// wait on one another.
+template <int kBufs>
+struct WarpStager {
   uint8_t* base;
-  int count;   // buffers handed out so far by this CTA
-  __device__ __forceinline__ uint8_t* acquire() {
-    uint8_t* buf = base + (count & 1) * (128 * 32 * 2);
-    if (count >= 2) {
-      if (threadIdx.x == 64) bulk_wait_read<1>();   // the buffer's previous stores have been read
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+  int count;   // boxes handed out so far
+  __device__ __forceinline__ void put(const CUtensorMap* map, int lane, const uint4 (&row)[4], int x, int y,
+                                      int z) {
+    uint8_t* buf = base + (count % kBufs) * (32 * 32 * 2);
+    if (count >= kBufs) {
+      if (lane == 0) bulk_wait_read<kBufs - 1>();
+      __syncwarp();
     }
-    return buf;
-  }
-  __device__ __forceinline__ void issue(const CUtensorMap* map, const uint8_t* buf, int x, int y, int z,
-                                        bool mirror_halves) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + store_box_offset(lane, q)) = row[q];
     fence_proxy_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (threadIdx.x == 64) {
+    __syncwarp();
+    if (lane == 0) {
       tma_store_3d(map, buf, x, y, z);
-      if (mirror_halves) tma_store_3d(map, buf + 64 * 32 * 2, x + 64, y, z);
       bulk_commit();
     }
     ++count;
   }
-  __device__ __forceinline__ void put(const CUtensorMap* map, int lrow, const uint4 (&packed)[4], int x, int y,
-                                      int z) {
-    uint8_t* buf = acquire();
-#pragma unroll
-    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + store_box_offset(lrow, q)) = packed[q];
-    issue(map, buf, x, y, z, false);
-  }
-  // Mirrored store: warp `quarter` supplies, in lane j, row j of its
-  // transposed 32 x 32 block (32 values = columns quarter*32 .. +31 of the
-  // mirrored 32 x 128 block).  Stored at (x = first row of the CTA, y = col0).
-  __device__ __forceinline__ void put_mirror(const CUtensorMap* map, int quarter, int lane, const uint4 (&colv)[4],
-                                             int x, int y, int z) {
-    uint8_t* buf = acquire();
-    uint8_t* half = buf + (quarter >> 1) * (64 * 32 * 2);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int c16 = (quarter & 1) * 4 + k;
-      *reinterpret_cast<uint4*>(half + lane * 128 + ((c16 ^ (lane & 7)) << 4)) = colv[k];
-    }
-    issue(map, buf, x, y, z, true);
-  }
 };
+
+// Transpose a warp's 32 x 32 block of 16-bit values through its padded
+// shared-memory scratch: lane j passes row j, receives column j.
+template <int PREC, int kStride>
+__device__ __forceinline__ void warp_transpose32(uint8_t* scratch, int lane, const uint4 (&row)[4], uint4 (&col)[4]) {
+  using T16 = typename Store16<PREC>::T;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(scratch + lane * kStride + q * 16) = row[q];
+  __syncwarp();
+  T16* cv = reinterpret_cast<T16*>(col);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) cv[i] = *reinterpret_cast<const T16*>(scratch + i * kStride + lane * 2);
+  __syncwarp();
+}
 
 template <int PREC>
 __device__ __forceinline__ void pack32(const float (&v)[32], uint4 (&packed)[4]) {
@@ -540,7 +544,7 @@ __device__ __forceinline__ void pack32(const float (&v)[32], uint4 (&packed)[4])
 constexpr int kPairM = 256;
 
 template <int MODE, int PREC>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>::kThreads, 1)
     ns_gemm_pair_kernel(const __grid_constant__ NsParams p) {
   using C = PairCfg<PREC, MODE>;
   constexpr bool kApply = MODE == M_APPLY || MODE == M_APPLY_LAST;
@@ -551,9 +555,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* wfull = drain + 1;                       // last APPLY: W boxes landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + 2);
-  float* red = reinterpret_cast<float*>(tmem_slot + 4);   // 8 floats
+  uint64_t* wfull = drain + 1;                       // last APPLY / SQUARE: staged boxes landed
+  uint64_t* wempty = wfull + 4;                      // ... and consumed by the 4 epilogue warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -568,11 +572,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * 128);                // both CTAs' epilogue threads
+      mbar_init(&tempty[a], 2 * 32 * C::kEpiWarps);  // both CTAs' epilogue threads
     }
     mbar_init(drain, 1);
-    mbar_init(&wfull[0], 1);
-    mbar_init(&wfull[1], 1);
+    for (int b = 0; b < C::kWBufs; ++b) {
+      mbar_init(&wfull[b], 1);
+      mbar_init(&wempty[b], C::kEpiWarps);
+    }
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
@@ -607,29 +613,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           const int k0 = kb * kBK;
-          constexpr int kHalf = 64 * kBK * 2;   // one 64-wide MN-major chunk
           if (MODE == M_GRAM) {
             tma_load_3d_pair(sa, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, arow, z);
             tma_load_3d_pair(sb, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, bcol, z);
+          } else if (MODE == M_SQUARE) {
+            // A A with A stored whole (GRAM writes every block and its mirror):
+            // both operands K-major; A is symmetric, so its rows serve as the
+            // N x K operand
+            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_A_K128, bar, k0, arow, z);
+            tma_load_3d_pair(sb, p.tmaps + cd.tm_base + TM_A_K128, bar, k0, bcol, z);
           } else {
-            // A operand: rows of the symmetric A (SQUARE: upper blocks only,
-            // lower blocks through their stored transpose) or of B' (APPLY:
-            // stored with its mirror, always K-major)
-            if (kApply || k0 >= abase) {
-              tma_load_3d_pair(sa, p.tmaps + cd.tm_base + (MODE == M_SQUARE ? TM_A_K128 : TM_B_K128), bar, k0,
-                               arow, z);
-            } else {
-              tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_A_MN, bar, arow, k0, z);
-              tma_load_3d_pair(sa + kHalf, p.tmaps + cd.tm_base + TM_A_MN, bar, arow + 64, k0, z);
-            }
-            if (MODE == M_SQUARE && k0 >= bbase) {
-              tma_load_3d_pair(sb, p.tmaps + cd.tm_base + TM_C_K128, bar, k0, bcol, z);
-            } else {
-              const CUtensorMap* bm = (MODE == M_SQUARE) ? p.tmaps + cd.tm_base + TM_C_MN
-                                                         : p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, 0);
-              tma_load_3d_pair(sb, bm, bar, bcol, k0, z);
-              tma_load_3d_pair(sb + kHalf, bm, bar, bcol + 64, k0, z);
-            }
+            // APPLY: rows of B' (stored with its mirror, K-major) times Y,
+            // read as an MN-major operand
+            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_B_K128, bar, k0, arow, z);
+            const CUtensorMap* bm = p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, 0);
+            tma_load_3d_pair(sb, bm, bar, bcol, k0, z);
+            tma_load_3d_pair(sb + 64 * kBK * 2, bm, bar, bcol + 64, k0, z);   // second 64-wide MN chunk
           }
           issued[stage] = true;
           issued_parity[stage] = phase;
@@ -649,9 +648,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t kIdescKK = idesc_f16(kPairM, kBN, PREC == P_BF16 ? 1 : 0, 0);
-      constexpr uint32_t kAMn = 1u << 15;   // A operand MN-major
-      constexpr uint32_t kBMn = 1u << 16;   // B operand MN-major
+      // A operand always K-major; B operand MN-major in APPLY (Y read as stored)
+      constexpr uint32_t kIdesc = idesc_f16(kPairM, kBN, PREC == P_BF16 ? 1 : 0, kApply ? 1 : 0);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -660,28 +658,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int t = pair; t < p.ntiles && ok; t += npairs, ++local) {
         const TileDesc next = (t + npairs < p.ntiles) ? p.tiles[t + npairs] : td;   // prefetch
         const int nk = (MODE == M_SQUARE) ? td.nk_sq : td.nk;
-        const int abase = td.bi * kPairM, bbase = td.bj * kBN;
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
         for (int kb = 0; kb < nk; ++kb) {
-          const int k0 = kb * kBK;
-          const bool a_mn = (MODE == M_SQUARE) && k0 < abase;
-          const bool b_mn = kApply || (MODE == M_SQUARE && k0 < bbase);
-          const uint32_t idesc = kIdescKK | (a_mn ? kAMn : 0u) | (b_mn ? kBMn : 0u);
           if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t sb = sa + C::kABytes;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t adesc = a_mn ? sdesc_sw128(sa + k * 16 * 128, 64 * kBK * 2, 1024)
-                                        : sdesc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t bdesc = b_mn ? sdesc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
-                                        : sdesc_sw128(sb + k * 32, 16, 1024);
-            umma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+            const uint64_t adesc = sdesc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bdesc = kApply ? sdesc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
+                                          : sdesc_sw128(sb + k * 32, 16, 1024);
+            umma_f16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit_pair(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -698,19 +690,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;             // TMEM lanes 32 quarter .. +31 (a warp reaches lanes of warp id mod 4)
+    const int epi = warp - 2;                 // 0 .. kEpiWarps-1
+    constexpr int kChStep = C::kEpiWarps / 4; // warps sharing a lane quarter split its chunks
+    const int ch0 = epi / 4;
     const int lrow = quarter * 32 + lane;
     const uint32_t tempty_leader[2] = {map_shared_rank(&tempty[0], 0), map_shared_rank(&tempty[1], 0)};
-    StoreStager stager{smem + C::kStoreOffset, 0};
-    uint32_t wphase[2] = {0u, 0u};   // last APPLY: phases of the two W buffers
-    int w_pending[2] = {0, 0};       // thread 64: W loads issued and not yet consumed
+    WarpStager<C::kWarpBufs> stager{smem + C::kStoreOffset + epi * C::kWarpBufs * C::kWarpBox, 0};
+    const int wrow0_off = quarter * 32;   // this warp's rows inside the CTA's 128
+    uint32_t wphase[C::kWBufs] = {};   // phases of the staging buffers
+    int w_pending[C::kWBufs] = {};     // thread 64: staged loads issued and not yet consumed
+    int w_issued[C::kWBufs] = {};      // thread 64: loads issued into each buffer so far
     bool werr = false;
-    // thread 64 loads the W box of chunk `chk` into buffer b
-    auto w_issue = [&](const TileDesc& td, const MatDev& md, int row0, int b, int chk) {
+    // thread 64 loads the epilogue operand of chunk `chk` into buffer b: the
+    // last APPLY's W box, or SQUARE's A box (rows row0.., chunk columns)
+    auto w_issue = [&](const TileDesc& td, const MatDev& md, const ClassDev& cd, int row0, int b, int chk) {
       const int c0 = td.bj * kBN + chk * 32;
+      // the buffer's previous contents must have been read by all epilogue warps
+      if (w_issued[b] > 0 && !mbar_wait(&wempty[b], static_cast<uint32_t>(w_issued[b] - 1) & 1u, p.err)) {
+        werr = true;
+        return;
+      }
+      ++w_issued[b];
       mbar_expect_tx(&wfull[b], C::kWBox);
       uint8_t* dst = smem + C::kWOffset + b * C::kWBox;
-      if (!md.transposed)
+      if (C::kSquare)
+        tma_load_3d(dst, p.tmaps + cd.tm_base + TM_A_EPI, &wfull[b], c0, row0, md.z);
+      else if (!md.transposed)
         tma_load_2d(dst, p.wmaps + td.mat, &wfull[b], c0, row0);
       else
         tma_load_2d(dst, p.wmaps + td.mat, &wfull[b], row0, c0);
@@ -723,10 +729,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const ClassDev& cd = p.classes[md.cls];
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      if (C::kLast && threadIdx.x == 64 && md.fused_dots && p.iter == md.ns_steps - 1) {
+      if (threadIdx.x == 64 && (C::kSquare || (C::kLast && md.fused_dots && p.iter == md.ns_steps - 1))) {
         const int r0 = td.bi * kPairM + static_cast<int>(rank) * 128;
-        w_issue(td, md, r0, 0, 0);   // W of chunks 0 and 1 while the tile's MMAs run
-        w_issue(td, md, r0, 1, 1);
+        for (int b = 0; b < C::kWBufs; ++b) w_issue(td, md, cd, r0, b, b);   // first chunks while the MMAs run
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
       tc_fence_after();
@@ -735,71 +740,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       // iteration 0 reads X at the momentum kernel's scale: kappa corrects it
       const float kap = (p.iter == 0) ? p.scal[td.mat].kappa : 1.f;
+      uint8_t* mirror_buf = smem + C::kMirrorOffset + epi * 32 * C::kMirrorStride;
+      const bool mirror = td.bj > td.bi;   // off-diagonal block: also store its transpose
       if (MODE == M_GRAM) {
         const float sa = kap * kap * exp2f(static_cast<float>(md.ea - 2 * md.ex));
-        const float sc = kap * kap * md.c_coef * exp2f(static_cast<float>(md.ec - 2 * md.ex));
-        const float diag = md.b * exp2f(static_cast<float>(md.ec));
-        for (int ch = 0; ch < kBN / 32; ++ch) {
+        for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
           const int col0 = td.bj * kBN + ch * 32;
-          float v[32], w[32];
+          float v[32];
           tmem_ld32(taddr + ch * 32, v);
-          if (ch == kBN / 32 - 1) {
+          if (ch + kChStep >= kBN / 32) {   // this warp's last chunk of the tile
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader[acc]);   // accumulator drained
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            w[j] = sc * v[j];
-            v[j] *= sa;
-          }
-          const int dj = row - col0;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j == dj) w[j] += diag;
-          uint4 pv[4], pw[4];
+          for (int j = 0; j < 32; ++j) v[j] *= sa;
+          uint4 pv[4];
           pack32<PREC>(v, pv);
-          pack32<PREC>(w, pw);
-          stager.put(p.tmaps + cd.tm_base + TM_A_ST, lrow, pv, col0, row0, md.z);
-          stager.put(p.tmaps + cd.tm_base + TM_C_ST, lrow, pw, col0, row0, md.z);
+          stager.put(p.tmaps + cd.tm_base + TM_A_ST, lane, pv, col0, row0 + wrow0_off, md.z);
+          if (mirror) {
+            // A is symmetric: A[col][row] = A[row][col]
+            uint4 cv[4];
+            warp_transpose32<PREC, C::kMirrorStride>(mirror_buf, lane, pv, cv);
+            stager.put(p.tmaps + cd.tm_base + TM_A_ST, lane, cv, row0 + wrow0_off, col0, md.z);
+          }
         }
       } else if (MODE == M_SQUARE) {
-        const float sb = exp2f(static_cast<float>(md.eb - md.ea - md.ec));
+        // stored B' = 2^eb (c A A + b A + a I), from the product of the stored
+        // A (2^ea A) with itself and the staged 2^ea A of this chunk
+        const float s2 = md.c_coef * exp2f(static_cast<float>(md.eb - 2 * md.ea));
+        const float s1 = md.b * exp2f(static_cast<float>(md.eb - md.ea));
         const float diag = md.a * exp2f(static_cast<float>(md.eb));
         using T16 = typename Store16<PREC>::T;
-        uint8_t* mirror_buf = smem + C::kMirrorOffset + quarter * 32 * C::kMirrorStride;
-        const bool mirror = td.bj > td.bi;   // off-diagonal block: also store B'[col][row]
-        for (int ch = 0; ch < kBN / 32; ++ch) {
+        for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
           const int col0 = td.bj * kBN + ch * 32;
           float v[32];
           tmem_ld32(taddr + ch * 32, v);
-          if (ch == kBN / 32 - 1) {
+          if (ch + kChStep >= kBN / 32) {   // this warp's last chunk of the tile
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader[acc]);
           }
+          const int b = ch % C::kWBufs;
+          if (!mbar_wait(&wfull[b], wphase[b], p.err)) { werr = true; break; }
+          wphase[b] ^= 1u;
+          if (threadIdx.x == 64) --w_pending[b];
+          {
+            // row lrow of the staged 128 x 32 box (64-byte swizzle)
+            const uint8_t* ab = smem + C::kWOffset + b * C::kWBox;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= sb;
+            for (int q = 0; q < 4; ++q) {
+              const uint4 u = *reinterpret_cast<const uint4*>(ab + store_box_offset(lrow, q));
+              const T16* h = reinterpret_cast<const T16*>(&u);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[8 * q + e] = fmaf(s2, v[8 * q + e], s1 * Store16<PREC>::back(h[e]));
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&wempty[b]);   // this warp is done with A buffer b
+          if (threadIdx.x == 64 && ch + C::kWBufs < kBN / 32) w_issue(td, md, cd, row0, b, ch + C::kWBufs);
           const int dj = row - col0;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (j == dj) v[j] += diag;
           uint4 packed[4];
           pack32<PREC>(v, packed);
-          stager.put(p.tmaps + cd.tm_base + TM_B_ST, lrow, packed, col0, row0, md.z);
+          stager.put(p.tmaps + cd.tm_base + TM_B_ST, lane, packed, col0, row0 + wrow0_off, md.z);
           if (mirror) {
-            // transpose the warp's 32 x 32 block through shared memory
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              *reinterpret_cast<uint4*>(mirror_buf + lane * C::kMirrorStride + q * 16) = packed[q];
-            __syncwarp();
-            uint4 colv[4];
-            T16* cv = reinterpret_cast<T16*>(colv);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              cv[i] = *reinterpret_cast<const T16*>(mirror_buf + i * C::kMirrorStride + lane * 2);
-            __syncwarp();
-            stager.put_mirror(p.tmaps + cd.tm_base + TM_B_MIR, quarter, lane, colv, row0, col0, md.z);
+            // B'[col0 + lane][row0 + 32 quarter + j] = B'[row0 + 32 quarter + j][col0 + lane]
+            uint4 cv[4];
+            warp_transpose32<PREC, C::kMirrorStride>(mirror_buf, lane, packed, cv);
+            stager.put(p.tmaps + cd.tm_base + TM_B_ST, lane, cv, row0 + wrow0_off, col0, md.z);
           }
         }
+        if (werr) break;
       } else {
         const float ks = kap * exp2f(static_cast<float>(-md.eb));
         const CUtensorMap* ymap = p.tmaps + cd.tm_base + TM_X_ST + (p.src ^ 1);
@@ -808,11 +820,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // of W[row0.., col0..]; tall W: box of W[col0.., row0..]).
         const bool dots = C::kLast && md.fused_dots && p.iter == md.ns_steps - 1;
         float oo = 0.f, wo = 0.f;
-        for (int ch = 0; ch < kBN / 32; ++ch) {
+        for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
           const int col0 = td.bj * kBN + ch * 32;
           float v[32];
           tmem_ld32(taddr + ch * 32, v);
-          if (ch == kBN / 32 - 1) {
+          if (ch + kChStep >= kBN / 32) {   // this warp's last chunk of the tile
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader[acc]);
           }
@@ -820,9 +832,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < 32; ++j) v[j] *= ks;
           uint4 packed[4];
           pack32<PREC>(v, packed);
-          stager.put(ymap, lrow, packed, col0, row0, md.z);
+          stager.put(ymap, lane, packed, col0, row0 + wrow0_off, md.z);
           if (C::kLast && dots) {
-            const int b = ch & 1;
+            const int b = ch % C::kWBufs;
             if (!mbar_wait(&wfull[b], wphase[b], p.err)) { werr = true; break; }
             wphase[b] ^= 1u;
             if (threadIdx.x == 64) --w_pending[b];
@@ -847,8 +859,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 wo = fmaf(w, o, wo);
               }
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");   // every thread is done with W buffer b
-            if (threadIdx.x == 64 && ch + 2 < kBN / 32) w_issue(td, md, row0, b, ch + 2);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wempty[b]);   // this warp is done with W buffer b
+            if (threadIdx.x == 64 && ch + C::kWBufs < kBN / 32) w_issue(td, md, cd, row0, b, ch + C::kWBufs);
           }
         }
         if (werr) break;
@@ -858,25 +871,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             oo += __shfl_xor_sync(0xffffffffu, oo, o);
             wo += __shfl_xor_sync(0xffffffffu, wo, o);
           }
-          if (lane == 0) {
-            red[2 * quarter] = oo;
-            red[2 * quarter + 1] = wo;
-          }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (threadIdx.x == 64) {
+          if (lane == 0) {   // one slot per (pair tile, CTA, epilogue warp)
             const int64_t slot =
-                md.ns_slot_base + (static_cast<int64_t>(td.bi) * md.ns_tiles_bj + td.bj) * 2 + rank;
-            p.part_ns[2 * slot] = ((red[0] + red[2]) + red[4]) + red[6];
-            p.part_ns[2 * slot + 1] = ((red[1] + red[3]) + red[5]) + red[7];
+                md.ns_slot_base + ((static_cast<int64_t>(td.bi) * md.ns_tiles_bj + td.bj) * 2 + rank) * 4 + quarter;
+            p.part_ns[2 * slot] = oo;
+            p.part_ns[2 * slot + 1] = wo;
           }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
         }
       }
     }
+    if (lane == 0) bulk_wait_all();   // every TMA store of this warp has completed
     if (threadIdx.x == 64) {
-      bulk_wait_all();   // every TMA store has completed
       // on a give-up path, let issued W loads land before the CTA exits
-      for (int b = 0; b < 2; ++b)
+      for (int b = 0; b < C::kWBufs; ++b)
         for (; w_pending[b] > 0; --w_pending[b]) {
           const uint64_t t0 = globaltimer();
           while (!mbar_try_wait(&wfull[b], wphase[b]) && globaltimer() - t0 < kWaitLimitNs) {
@@ -933,7 +940,7 @@ cudaError_t launch_ns_gemm_pair(int mode, int prec, const NsParams& p, int pairs
   if (p.ntiles <= 0) return cudaSuccess;
 #define MUONH_LAUNCH_PAIR(MD, PR)                                                              \
   if (mode == MD && prec == PR) {                                                              \
-    ns_gemm_pair_kernel<MD, PR><<<2 * pairs, kGemmThreads, PairCfg<PR, MD>::kSmem, s>>>(p);   \
+    ns_gemm_pair_kernel<MD, PR><<<2 * pairs, PairCfg<PR, MD>::kThreads, PairCfg<PR, MD>::kSmem, s>>>(p);   \
     return cudaGetLastError();                                                                 \
   }
   MUONH_LAUNCH_PAIR(M_GRAM, P_FP16) MUONH_LAUNCH_PAIR(M_SQUARE, P_FP16) MUONH_LAUNCH_PAIR(M_APPLY, P_FP16)

@@ -201,3 +201,35 @@ def test_ordinary_muon_rules(rule, prec, ns_tol, w_tol):
         # no projection: the norm moves, unlike MuonH
         assert abs(g["stats"][4][i]["post_norm"] - o["R"][i]) > 1e-3 * o["R"][i]
         assert np.linalg.norm(g["W"][i] - o["W"][i]) / np.linalg.norm(o["W"][i]) <= w_tol, i
+
+
+def test_phase_timing_does_not_disturb_the_step():
+    """Timing on for two steps, read the per-phase times, then keep stepping
+    with a new gradient buffer: the results match an untimed context bit for bit."""
+    import torch
+    from pretraining_optimizer_b200 import MuonH
+    dev = torch.device("cuda:0")
+    shapes = [(256, 512), (640, 384)]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    runs = []
+    for timed in (False, True):
+        W = [torch.from_numpy(w).to(dev) for w in W0]
+        opt = MuonH(W)
+        for t in range(4):
+            if timed:
+                opt.enable_timing(t < 2)
+            G = [torch.from_numpy(synth.gaussian_gradient(t, i, *s)).to(dev) for i, s in enumerate(shapes)]
+            opt.step(G, 0.01)
+            if timed and t == 1:
+                ph = opt.phase_times()
+                for name in ("momentum_norm", "ns_gram", "ns_square", "ns_apply", "project", "finalize_step"):
+                    # 5 Newton-Schulz iterations a step; the elementwise phases may take
+                    # one launch per kind of tile (wide, tall) each step
+                    ok = ph[name][1] == 10 if name.startswith("ns_") else ph[name][1] in (2, 4)
+                    assert ok and ph[name][0] > 0, (name, ph[name])
+        torch.cuda.synchronize()
+        opt.device_status()
+        runs.append([w.cpu().numpy() for w in W])
+        opt.close()
+    for a, b in zip(*runs):
+        assert np.array_equal(a, b)
