@@ -208,6 +208,7 @@ struct muonh_ctx {
     p.prec = prec;
     p.stats_out = stats_out;
     p.err = d_err;
+    p.any_rewrite = d_err + 1;
     return p;
   }
 };
@@ -533,7 +534,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part_ns),
                 std::max<int64_t>(1, 2 * ctx->n_ns_slots) * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_wmaps), n * sizeof(CUtensorMap)) != cudaSuccess ||
-      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), sizeof(int)) != cudaSuccess)
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), 2 * sizeof(int)) != cudaSuccess)   // err, any_rewrite
     return fail(MUONH_ERR_OOM, "allocation of the device tables failed");
 
   std::vector<ClassDev> cdev;
@@ -561,7 +562,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   CUDA_TRY(cudaMemcpyAsync(ctx->d_classes, cdev.data(), cdev.size() * sizeof(ClassDev), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_et_mat, et_mat.data(), n_et * sizeof(int32_t), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_scal, scal.data(), n * sizeof(MatScal), cudaMemcpyHostToDevice, s));
-  CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, sizeof(int), s));
+  CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, 2 * sizeof(int), s));
 
   // ---- Newton-Schulz tile lists, one pair per iteration (shared when equal)
   std::vector<int32_t> prev_active;

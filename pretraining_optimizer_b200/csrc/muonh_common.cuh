@@ -135,6 +135,7 @@ struct EwParams {
   int32_t prec;
   muonh_stats* stats_out;
   const int* err;
+  int* any_rewrite;          // set by finalize_input when a matrix needs write_x; cleared by finalize_step
 };
 
 // -------------------------------------------------------------- PTX helpers

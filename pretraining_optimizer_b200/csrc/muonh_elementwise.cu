@@ -372,6 +372,7 @@ __global__ void __launch_bounds__(kEwThreads, 5) momentum_norm_kernel(const EwPa
 // X_stored = xscale * X into NS buffer 0 (wide orientation, transposed for tall W).
 __global__ void __launch_bounds__(kEwThreads, 6) write_x_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
+  if (*reinterpret_cast<const volatile int*>(p.any_rewrite) == 0) return;   // every X already written
   for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
     const int mi = p.et_mat[e];
     if (!p.scal[mi].rewrite) {
@@ -650,6 +651,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwPara
         sc.kappa = static_cast<float>(ldexp(1.0, md.ex) / (sigma * (xn + static_cast<double>(p.eps))));
       }
     }
+    if (sc.rewrite) atomicOr(p.any_rewrite, 1);
     // scale for the next step's momentum kernel (not in FP32 mode: hi/lo X)
     sc.sigma = (p.prec != P_FP32 && isfinite(s) && s > 0.0) ? static_cast<float>(ldexp(1.0, md.ex - 2) / xn) : 0.f;
   }
@@ -730,6 +732,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_step_kernel(const EwParam
   const int mi = blockIdx.x;
   const MatDev& md = p.mats[mi];
   const double s = tile_partials(p, md, red);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.any_rewrite = 0;   // write_x of this step has run
   if (threadIdx.x == 0) {
     MatScal& sc = p.scal[mi];
     if (sc.mode != 2) sc.wnorm2 = s;

@@ -8,7 +8,9 @@
 // each of its 8 warps owns a fixed eighth of every tile and never waits for
 // the others: no shared memory, no block barrier.  A lane issues all of its
 // loads for a tile (8 x 16 bytes on wide tiles, 16 x 8 bytes on tall ones)
-// before the first use, so a resident warp keeps 4 KB in flight.  Tall
+// before the first use, so a resident warp keeps 4 KB in flight, and it
+// fetches the next tile's table entries while those loads are in flight
+// (three resident blocks per SM: 80 registers a thread).  Tall
 // matrices, whose X is the transpose, are tiled 64 x 64: warp w takes rows
 // 8w..8w+7 with two adjacent columns per lane, so a lane holds 8 consecutive
 // entries of two X rows and writes (or, in project, reads) each as one
@@ -54,11 +56,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, int prec) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ uint16_t* x_base(const EwParams& p, const MatDev& md, int buf) {
-  const ClassDev& cd = p.classes[md.cls];
-  return static_cast<uint16_t*>(cd.x[buf][0]) + md.z * cd.x_stride;
-}
-
 struct Tile {
   int64_t r0, c0;
   int nr, nc;        // valid rows / columns of the tile inside the matrix
@@ -88,10 +85,57 @@ __device__ __forceinline__ int64_t next_tile(const EwParams& p, int64_t e) {
   return e;
 }
 
+// Everything a warp needs to know about one tile, gathered from the device
+// tables; the kernels fetch the next tile's copy while the current tile's
+// data loads are in flight, so the dependent table reads (tile -> matrix ->
+// pointers, scalars) do not stall the data stream.
+struct TileCtx {
+  int64_t e;
+  const float* a;       // momentum: G tile origin;   project: W tile origin
+  float* b;             // momentum: M tile origin;   project: W tile origin (written)
+  uint16_t* x;          // X / O at the tile origin (wide: row r0, column c0; tall: row c0, column r0)
+  int64_t ld, xld;
+  int nr, nc, sh;       // valid rows / columns; log2(tw / 4) for wide tiles
+  float s0, s1;         // momentum: beta, sigma;     project: kw, ko
+  int flag;             // momentum: nesterov;        project: mode
+};
+
+template <bool TALL, bool PROJECT>
+__device__ __forceinline__ TileCtx tile_ctx(const EwParams& p, int64_t e) {
+  TileCtx c;
+  c.e = e;
+  if (e >= p.n_et) return c;
+  const int mi = p.et_mat[e];
+  const MatDev& md = p.mats[mi];
+  const Tile t = tile_of(md, e);
+  const ClassDev& cd = p.classes[md.cls];
+  c.ld = md.ld;
+  c.xld = cd.c_pad;
+  c.nr = t.nr;
+  c.nc = t.nc;
+  c.sh = __ffs(md.et_tw) - 3;
+  uint16_t* xg = static_cast<uint16_t*>(cd.x[PROJECT ? (md.ns_steps & 1) : 0][0]) + md.z * cd.x_stride;
+  c.x = TALL ? xg + t.c0 * c.xld + t.r0 : xg + t.r0 * c.xld + t.c0;
+  if (PROJECT) {
+    const MatScal& sc = p.scal[mi];
+    c.a = md.w + t.r0 * md.ld + t.c0;
+    c.b = md.w + t.r0 * md.ld + t.c0;
+    c.s0 = sc.kw;
+    c.s1 = sc.ko;
+    c.flag = sc.mode;
+  } else {
+    c.a = p.step[mi].g + t.r0 * md.ld + t.c0;
+    c.b = md.m + t.r0 * md.ld + t.c0;
+    c.s0 = md.beta;
+    c.s1 = p.scal[mi].sigma;
+    c.flag = md.nesterov;
+  }
+  return c;
+}
+
 // Chunk j (0..3) of lane `lane` in warp w of a wide tile: 4 consecutive
 // columns of one row; the warp covers chunks 128w .. 128w + 127.
-__device__ __forceinline__ void wide_chunk(const MatDev& md, int w, int lane, int j, int& row, int& col) {
-  const int sh = __ffs(md.et_tw) - 3;          // log2(chunks per row) = log2(tw / 4)
+__device__ __forceinline__ void wide_chunk_sh(int sh, int w, int lane, int j, int& row, int& col) {
   const int q = lane + 32 * j + 128 * w;
   row = q >> sh;
   col = (q & ((1 << sh) - 1)) * 4;
@@ -99,19 +143,11 @@ __device__ __forceinline__ void wide_chunk(const MatDev& md, int w, int lane, in
 
 // ---------------------------------------------------------------- momentum
 template <bool TALL>
-__global__ void __launch_bounds__(kWarpThreads) momentum_warp_kernel(const EwParams p) {
+__global__ void __launch_bounds__(kWarpThreads, 3) momentum_warp_kernel(const EwParams p) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int64_t e = next_tile<TALL>(p, blockIdx.x); e < p.n_et; e = next_tile<TALL>(p, e + gridDim.x)) {
-    const int mi = p.et_mat[e];
-    const MatDev& md = p.mats[mi];
-    const Tile t = tile_of(md, e);
-    const float beta = md.beta;
-    const int nesterov = md.nesterov;
-    const float sigma = p.scal[mi].sigma;
-    const float* gb = p.step[mi].g + t.r0 * md.ld + t.c0;
-    float* mb = md.m + t.r0 * md.ld + t.c0;
-    uint16_t* xg = x_base(p, md, 0);
-    const int64_t xld = p.classes[md.cls].c_pad;
+  TileCtx cur = tile_ctx<TALL, false>(p, next_tile<TALL>(p, blockIdx.x));
+  while (cur.e < p.n_et) {
+    const float beta = cur.s0, sigma = cur.s1;
     float acc = 0.f;
     if (!TALL) {
       int row[4], col[4];
@@ -119,13 +155,14 @@ __global__ void __launch_bounds__(kWarpThreads) momentum_warp_kernel(const EwPar
       float4 gv[4], mv[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        wide_chunk(md, w, lane, j, row[j], col[j]);
-        ok[j] = row[j] < t.nr && col[j] < t.nc;
+        wide_chunk_sh(cur.sh, w, lane, j, row[j], col[j]);
+        ok[j] = row[j] < cur.nr && col[j] < cur.nc;
         if (ok[j]) {
-          gv[j] = *reinterpret_cast<const float4*>(gb + row[j] * md.ld + col[j]);
-          mv[j] = *reinterpret_cast<const float4*>(mb + row[j] * md.ld + col[j]);
+          gv[j] = *reinterpret_cast<const float4*>(cur.a + row[j] * cur.ld + col[j]);
+          mv[j] = *reinterpret_cast<const float4*>(cur.b + row[j] * cur.ld + col[j]);
         }
       }
+      const TileCtx nxt = tile_ctx<TALL, false>(p, next_tile<TALL>(p, cur.e + gridDim.x));
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (!ok[j]) continue;
@@ -135,9 +172,9 @@ __global__ void __launch_bounds__(kWarpThreads) momentum_warp_kernel(const EwPar
         m.y = fmaf(beta, m.y, g.y);
         m.z = fmaf(beta, m.z, g.z);
         m.w = fmaf(beta, m.w, g.w);
-        *reinterpret_cast<float4*>(mb + row[j] * md.ld + col[j]) = m;
+        *reinterpret_cast<float4*>(cur.b + row[j] * cur.ld + col[j]) = m;
         float4 x = m;
-        if (nesterov) {
+        if (cur.flag) {
           x.x = fmaf(beta, m.x, g.x);
           x.y = fmaf(beta, m.y, g.y);
           x.z = fmaf(beta, m.z, g.z);
@@ -149,39 +186,43 @@ __global__ void __launch_bounds__(kWarpThreads) momentum_warp_kernel(const EwPar
         acc = fmaf(x.w, x.w, acc);
         if (sigma > 0.f) {
           const uint2 u = make_uint2(pack2(x.x * sigma, x.y * sigma, p.prec), pack2(x.z * sigma, x.w * sigma, p.prec));
-          *reinterpret_cast<uint2*>(xg + (t.r0 + row[j]) * xld + t.c0 + col[j]) = u;
+          *reinterpret_cast<uint2*>(cur.x + row[j] * cur.xld + col[j]) = u;
         }
       }
+      acc = warp_sum(acc);
+      if (lane == 0) p.part8[cur.e * kWarps + w] = acc;
+      cur = nxt;
     } else {
       // tall 64 x 64: warp w takes rows 8w .. 8w+7; lane l covers columns
       // c .. c+3 (c = 4 (l mod 16)) of the even rows (l < 16) or the odd rows
       const int half = lane >> 4;
       const int c = 4 * (lane & 15);
-      const bool cok = c < t.nc;   // nc is a multiple of 4
+      const bool cok = c < cur.nc;   // nc is a multiple of 4
       float4 gv[4], mv[4];
 #pragma unroll
       for (int jr = 0; jr < 4; ++jr) {
         const int r = 8 * w + 2 * jr + half;
-        if (cok && r < t.nr) {
-          gv[jr] = *reinterpret_cast<const float4*>(gb + r * md.ld + c);
-          mv[jr] = *reinterpret_cast<const float4*>(mb + r * md.ld + c);
+        if (cok && r < cur.nr) {
+          gv[jr] = *reinterpret_cast<const float4*>(cur.a + r * cur.ld + c);
+          mv[jr] = *reinterpret_cast<const float4*>(cur.b + r * cur.ld + c);
         }
       }
+      const TileCtx nxt = tile_ctx<TALL, false>(p, next_tile<TALL>(p, cur.e + gridDim.x));
       float x[4][4];
 #pragma unroll
       for (int jr = 0; jr < 4; ++jr) {
         const int r = 8 * w + 2 * jr + half;
         x[jr][0] = x[jr][1] = x[jr][2] = x[jr][3] = 0.f;   // rows past the matrix stay zero in X's padding
-        if (!cok || r >= t.nr) continue;
+        if (!cok || r >= cur.nr) continue;
         float4 m = mv[jr];
         const float4 g = gv[jr];
         m.x = fmaf(beta, m.x, g.x);
         m.y = fmaf(beta, m.y, g.y);
         m.z = fmaf(beta, m.z, g.z);
         m.w = fmaf(beta, m.w, g.w);
-        *reinterpret_cast<float4*>(mb + r * md.ld + c) = m;
+        *reinterpret_cast<float4*>(cur.b + r * cur.ld + c) = m;
         float4 xv = m;
-        if (nesterov) {
+        if (cur.flag) {
           xv.x = fmaf(beta, m.x, g.x);
           xv.y = fmaf(beta, m.y, g.y);
           xv.z = fmaf(beta, m.z, g.z);
@@ -212,92 +253,97 @@ __global__ void __launch_bounds__(kWarpThreads) momentum_warp_kernel(const EwPar
             const float own = half ? x[jr][2 + k] : x[jr][k];
             h[jr] = half ? pack2(y[jr][k], own, p.prec) : pack2(own, y[jr][k], p.prec);
           }
-          *reinterpret_cast<uint4*>(xg + (t.c0 + c + kc) * xld + t.r0 + 8 * w) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(cur.x + (c + kc) * cur.xld + 8 * w) = make_uint4(h[0], h[1], h[2], h[3]);
         }
       }
+      acc = warp_sum(acc);
+      if (lane == 0) p.part8[cur.e * kWarps + w] = acc;
+      cur = nxt;
     }
-    acc = warp_sum(acc);
-    if (lane == 0) p.part8[e * kWarps + w] = acc;
   }
 }
 
 // ----------------------------------------------------------------- project
 template <bool TALL>
-__global__ void __launch_bounds__(kWarpThreads) project_warp_kernel(const EwParams p) {
+__global__ void __launch_bounds__(kWarpThreads, 3) project_warp_kernel(const EwParams p) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int64_t e = next_tile<TALL>(p, blockIdx.x); e < p.n_et; e = next_tile<TALL>(p, e + gridDim.x)) {
-    const int mi = p.et_mat[e];
-    const MatDev& md = p.mats[mi];
-    const MatScal& sc = p.scal[mi];
-    const int mode = sc.mode;
+  TileCtx cur = tile_ctx<TALL, true>(p, next_tile<TALL>(p, blockIdx.x));
+  while (cur.e < p.n_et) {
+    const int mode = cur.flag;
+    const float kw = cur.s0, ko = cur.s1;
     float acc = 0.f;
-    if (mode != 2) {
-      const float kw = sc.kw, ko = sc.ko;
-      const Tile t = tile_of(md, e);
-      float* wb = md.w + t.r0 * md.ld + t.c0;
-      const uint16_t* xg = x_base(p, md, md.ns_steps & 1);
-      const int64_t xld = p.classes[md.cls].c_pad;
-      if (!TALL) {
-        int row[4], col[4];
-        bool ok[4];
-        float4 wv[4];
-        uint2 ov[4];
+    if (mode == 2) {   // W kept
+      const TileCtx nxt = tile_ctx<TALL, true>(p, next_tile<TALL>(p, cur.e + gridDim.x));
+      if (lane == 0) p.part8[cur.e * kWarps + w] = 0.f;
+      cur = nxt;
+      continue;
+    }
+    if (!TALL) {
+      int row[4], col[4];
+      bool ok[4];
+      float4 wv[4];
+      uint2 ov[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          wide_chunk(md, w, lane, j, row[j], col[j]);
-          ok[j] = row[j] < t.nr && col[j] < t.nc;
-          ov[j] = make_uint2(0u, 0u);
-          if (ok[j]) {
-            wv[j] = *reinterpret_cast<const float4*>(wb + row[j] * md.ld + col[j]);
-            if (mode == 0) ov[j] = *reinterpret_cast<const uint2*>(xg + (t.r0 + row[j]) * xld + t.c0 + col[j]);
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (!ok[j]) continue;
-          const float4 o = unpack4(ov[j], p.prec);
-          float4 v = wv[j];
-          v.x = fmaf(ko, o.x, kw * v.x);
-          v.y = fmaf(ko, o.y, kw * v.y);
-          v.z = fmaf(ko, o.z, kw * v.z);
-          v.w = fmaf(ko, o.w, kw * v.w);
-          *reinterpret_cast<float4*>(wb + row[j] * md.ld + col[j]) = v;
-          acc = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, acc))));
-        }
-      } else {
-        const int c = 2 * lane;
-        const bool cok = c < t.nc;
-        float2 wv[8];
-        uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
-        if (cok && mode == 0) {
-          // O(8w + i, c) = X[c0 + c][r0 + 8w + i]: 8 consecutive entries of two X rows
-          const uint16_t* src = xg + (t.c0 + c) * xld + t.r0 + 8 * w;
-          o0 = *reinterpret_cast<const uint4*>(src);
-          o1 = *reinterpret_cast<const uint4*>(src + xld);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = 8 * w + i;
-          if (cok && r < t.nr) wv[i] = *reinterpret_cast<const float2*>(wb + r * md.ld + c);
-        }
-        const float4 a0 = unpack4(make_uint2(o0.x, o0.y), p.prec), a1 = unpack4(make_uint2(o0.z, o0.w), p.prec);
-        const float4 b0 = unpack4(make_uint2(o1.x, o1.y), p.prec), b1 = unpack4(make_uint2(o1.z, o1.w), p.prec);
-        const float oa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float ob[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = 8 * w + i;
-          if (!cok || r >= t.nr) continue;
-          float2 v = wv[i];
-          v.x = fmaf(ko, oa[i], kw * v.x);
-          v.y = fmaf(ko, ob[i], kw * v.y);
-          *reinterpret_cast<float2*>(wb + r * md.ld + c) = v;
-          acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
+      for (int j = 0; j < 4; ++j) {
+        wide_chunk_sh(cur.sh, w, lane, j, row[j], col[j]);
+        ok[j] = row[j] < cur.nr && col[j] < cur.nc;
+        ov[j] = make_uint2(0u, 0u);
+        if (ok[j]) {
+          wv[j] = *reinterpret_cast<const float4*>(cur.a + row[j] * cur.ld + col[j]);
+          if (mode == 0) ov[j] = *reinterpret_cast<const uint2*>(cur.x + row[j] * cur.xld + col[j]);
         }
       }
+      const TileCtx nxt = tile_ctx<TALL, true>(p, next_tile<TALL>(p, cur.e + gridDim.x));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (!ok[j]) continue;
+        const float4 o = unpack4(ov[j], p.prec);
+        float4 v = wv[j];
+        v.x = fmaf(ko, o.x, kw * v.x);
+        v.y = fmaf(ko, o.y, kw * v.y);
+        v.z = fmaf(ko, o.z, kw * v.z);
+        v.w = fmaf(ko, o.w, kw * v.w);
+        *reinterpret_cast<float4*>(cur.b + row[j] * cur.ld + col[j]) = v;
+        acc = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, acc))));
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) p.part8[cur.e * kWarps + w] = acc;
+      cur = nxt;
+    } else {
+      const int c = 2 * lane;
+      const bool cok = c < cur.nc;
+      float2 wv[8];
+      uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
+      if (cok && mode == 0) {
+        // O(8w + i, c) = X[c0 + c][r0 + 8w + i]: 8 consecutive entries of two X rows
+        const uint16_t* src = cur.x + c * cur.xld + 8 * w;
+        o0 = *reinterpret_cast<const uint4*>(src);
+        o1 = *reinterpret_cast<const uint4*>(src + cur.xld);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * w + i;
+        if (cok && r < cur.nr) wv[i] = *reinterpret_cast<const float2*>(cur.a + r * cur.ld + c);
+      }
+      const TileCtx nxt = tile_ctx<TALL, true>(p, next_tile<TALL>(p, cur.e + gridDim.x));
+      const float4 a0 = unpack4(make_uint2(o0.x, o0.y), p.prec), a1 = unpack4(make_uint2(o0.z, o0.w), p.prec);
+      const float4 b0 = unpack4(make_uint2(o1.x, o1.y), p.prec), b1 = unpack4(make_uint2(o1.z, o1.w), p.prec);
+      const float oa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float ob[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * w + i;
+        if (!cok || r >= cur.nr) continue;
+        float2 v = wv[i];
+        v.x = fmaf(ko, oa[i], kw * v.x);
+        v.y = fmaf(ko, ob[i], kw * v.y);
+        *reinterpret_cast<float2*>(cur.b + r * cur.ld + c) = v;
+        acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) p.part8[cur.e * kWarps + w] = acc;
+      cur = nxt;
     }
-    acc = warp_sum(acc);
-    if (lane == 0) p.part8[e * kWarps + w] = acc;
   }
 }
 
