@@ -9,12 +9,12 @@ Sources (Puro-2B report):
     displacement norm over the weight norm, eta ||u||/||W||; under Eq. (1) the
     displacement eta R u_hat has norm eta R while ||W|| = R, so it equals eta.
   * Reading notes, Sec. 2.5: the same Eq. (1), restated with eta^H.
-The Muon update u itself is only named by the pages ("Muon produces a
-same-shape update", reading notes Sec. 2.5).  Its internals -- heavy-ball
-momentum with a Nesterov look-ahead, Frobenius normalisation, and a quintic
-Newton-Schulz iteration with coefficients (3.4445, -4.7750, 2.0315) -- follow
-the workload definition this library is built for; each reading is listed in
-the design notes.
+The pages name the Muon update u but do not define its internals (reading
+notes, Sec. 2.5: Muon yields an update of the weight's shape).  Its
+internals -- heavy-ball momentum with a Nesterov look-ahead, Frobenius
+normalisation, and a quintic Newton-Schulz iteration with coefficients
+(3.4445, -4.7750, 2.0315) -- are the common Muon formulation, and every
+one of them is a per-matrix parameter of both the oracle and the library.
 
 Every function computes in `dtype` (float64 unless asked otherwise) with
 NumPy's matmul as the only library primitive.
