@@ -49,6 +49,15 @@ muonh_status fail(muonh_status st, const char* fmt, ...) {
   } while (0)
 
 constexpr int kRing = 4;
+// With at least this many elements the step runs in kGroups matrix groups
+// whose elementwise phases overlap the other groups' Newton-Schulz GEMMs;
+// below it the overlap cannot pay for the extra launches.
+constexpr int64_t kTwoGroupMinElems = int64_t(1) << 24;
+constexpr int kGroups = 2;
+// Tiles per block of an elementwise launch that overlaps Newton-Schulz GEMMs:
+// short-lived blocks leave the SMs' resources to the GEMMs' blocks, which the
+// scheduler places first (they run on the highest-priority stream).
+constexpr int64_t kOverlapTilesPerBlock = 4;
 constexpr int64_t kMaxDim = 1 << 20;
 constexpr int64_t kMaxRPad = 16384;
 constexpr int32_t kMaxNsSteps = 64;
@@ -145,7 +154,18 @@ struct muonh_ctx {
 
   std::vector<MatDev> mats;
   std::vector<ClassHost> classes;
-  std::vector<TileList> gram_lists, apply_lists;   // per Newton-Schulz iteration
+  // The step runs in one or kGroups matrix groups (contiguous index ranges
+  // of about equal Newton-Schulz work): the elementwise phases of one group
+  // overlap the Newton-Schulz GEMMs of its neighbours.
+  struct Group {
+    int32_t m_first = 0, m_count = 0;
+    int64_t e_first = 0, e_end = 0;
+    bool any_unfused = false, any_general = false, any_wt[2] = {false, false};
+    std::vector<TileList> gram_lists, apply_lists;   // per Newton-Schulz iteration
+  };
+  std::vector<Group> groups;
+  cudaStream_t ns_stream = nullptr;   // highest-priority stream for the GEMMs of a grouped step
+  std::vector<cudaEvent_t> gev;       // grouped step: per group, front done (2g) and GEMMs done (2g+1)
   std::vector<void*> allocs;
 
   MatDev* d_mats = nullptr;
@@ -158,10 +178,6 @@ struct muonh_ctx {
   float* d_part_ns = nullptr;      // fused last-APPLY partials
   CUtensorMap* d_wmaps = nullptr;  // per matrix fp32 W tiles (fused matrices)
   int64_t n_ns_slots = 0;
-  bool any_unfused = true;
-  bool any_warp_tiled = false;     // matrices handled by the warp-tiled momentum/project kernels
-  bool any_wt[2] = {false, false}; // ... among them wide (0) and tall (1) ones
-  bool any_general = true;         // matrices handled by the general ones
   int ew_warp_grid[4] = {148, 148, 148, 148};   // blocks of the warp-tiled kernels (one wave each)
   float* d_part8 = nullptr;
   CUtensorMap* d_tmaps = nullptr;
@@ -191,8 +207,13 @@ struct muonh_ctx {
     return e;
   }
 
-  EwParams ew(muonh_stats* stats_out) const {
+  // whole-context launch (init) or one group's launch (g >= 0)
+  EwParams ew(muonh_stats* stats_out, int g = -1) const {
     EwParams p{};
+    p.e_first = g < 0 ? 0 : groups[g].e_first;
+    p.e_end = g < 0 ? n_et : groups[g].e_end;
+    p.m_first = g < 0 ? 0 : groups[g].m_first;
+    p.m_count = g < 0 ? n : groups[g].m_count;
     p.mats = d_mats;
     p.step = d_step;
     p.scal = d_scal;
@@ -208,7 +229,7 @@ struct muonh_ctx {
     p.prec = prec;
     p.stats_out = stats_out;
     p.err = d_err;
-    p.any_rewrite = d_err + 1;
+    p.any_rewrite = d_err + 1 + (g < 0 ? 0 : g);
     return p;
   }
 };
@@ -225,6 +246,10 @@ void release(muonh_ctx* ctx) {
   if (!ctx) return;
   for (void* p : ctx->allocs) cudaFree(p);
   ctx->allocs.clear();
+  if (ctx->ns_stream) cudaStreamDestroy(ctx->ns_stream);
+  for (cudaEvent_t e : ctx->gev)
+    if (e) cudaEventDestroy(e);
+  ctx->gev.clear();
   for (int i = 0; i < kRing; ++i) {
     if (ctx->h_step[i]) cudaFreeHost(ctx->h_step[i]);
     if (ctx->ev[i]) cudaEventDestroy(ctx->ev[i]);
@@ -283,18 +308,18 @@ muonh_status check_launch(cudaError_t e, const char* what) {
     ++launches;                                             \
   } while (0)
 
-// A launch of the step, bracketed by events when timing is on.
-#define STEP_LAUNCH(phase, expr, name)                                   \
+// A launch of the step on stream `strm`, bracketed by events when timing is on.
+#define STEP_LAUNCH_ON(phase, expr, name, strm)                          \
   do {                                                                   \
     cudaEvent_t ev_b = nullptr, ev_e = nullptr;                          \
     if (ctx->timing) {                                                   \
       ev_b = ctx->take_event();                                          \
       ev_e = ctx->take_event();                                          \
-      CUDA_TRY(cudaEventRecord(ev_b, s));                                \
+      CUDA_TRY(cudaEventRecord(ev_b, strm));                             \
     }                                                                    \
     LAUNCH_TRY(expr, name);                                              \
     if (ctx->timing) {                                                   \
-      CUDA_TRY(cudaEventRecord(ev_e, s));                                \
+      CUDA_TRY(cudaEventRecord(ev_e, strm));                             \
       ctx->timed.push_back(muonh_ctx::Timed{phase, ev_b, ev_e});         \
     }                                                                    \
   } while (0)
@@ -443,14 +468,54 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       ctx->n_ns_slots += md.ns_slots;
     }
   }
-  ctx->any_unfused = false;
-  ctx->any_warp_tiled = false;
-  ctx->any_general = false;
-  for (int32_t i = 0; i < n; ++i) {
-    ctx->any_unfused |= !ctx->mats[i].fused_dots;
-    ctx->any_warp_tiled |= ctx->mats[i].warp_tiled != 0;
-    if (ctx->mats[i].warp_tiled) ctx->any_wt[ctx->mats[i].transposed ? 1 : 0] = true;
-    ctx->any_general |= ctx->mats[i].warp_tiled == 0;
+  // ---- matrix groups: with the CTA-pair path and enough elements, split
+  // the matrices into two index ranges of about equal Newton-Schulz work
+  {
+    std::vector<double> work(n);
+    double total = 0.0;
+    int64_t elems = 0;
+    for (int32_t i = 0; i < n; ++i) {
+      const MatDev& md = ctx->mats[i];
+      const double r = md.r, c = md.c;
+      work[i] = md.ns_steps * (4.0 * r * r * c + 2.0 * r * r * r);
+      total += work[i];
+      elems += md.rows * md.cols;
+    }
+    // group g ends after the first matrix at which the running work reaches
+    // (g + 1) / kGroups of the total; every group keeps at least one matrix
+    std::vector<int32_t> bounds{0};
+    if (ctx->pairs && n >= kGroups && elems >= kTwoGroupMinElems && total > 0.0) {
+      double acc = 0.0;
+      for (int32_t i = 0; i < n && static_cast<int>(bounds.size()) < kGroups; ++i) {
+        acc += work[i];
+        const int g = static_cast<int>(bounds.size()) - 1;
+        if (acc >= total * (g + 1) / kGroups && i + 1 > bounds.back() && n - (i + 1) >= kGroups - g - 1)
+          bounds.push_back(i + 1);
+      }
+    }
+    bounds.push_back(n);
+    for (size_t g = 0; g + 1 < bounds.size(); ++g) {
+      muonh_ctx::Group gr;
+      gr.m_first = bounds[g];
+      gr.m_count = bounds[g + 1] - bounds[g];
+      const MatDev& last = ctx->mats[bounds[g + 1] - 1];
+      gr.e_first = ctx->mats[bounds[g]].et_begin;
+      gr.e_end = last.et_begin + static_cast<int64_t>(last.et_rows) * last.et_cols;
+      for (int32_t i = bounds[g]; i < bounds[g + 1]; ++i) {
+        const MatDev& md = ctx->mats[i];
+        gr.any_unfused |= !md.fused_dots;
+        gr.any_general |= md.warp_tiled == 0;
+        if (md.warp_tiled) gr.any_wt[md.transposed ? 1 : 0] = true;
+      }
+      ctx->groups.push_back(gr);
+    }
+    if (ctx->groups.size() > 1) {
+      int least = 0, greatest = 0;
+      CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+      CUDA_TRY(cudaStreamCreateWithPriority(&ctx->ns_stream, cudaStreamNonBlocking, greatest));
+      ctx->gev.assign(2 * ctx->groups.size(), nullptr);
+      for (cudaEvent_t& e : ctx->gev) CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    }
   }
 
   // ---- workspace
@@ -534,7 +599,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part_ns),
                 std::max<int64_t>(1, 2 * ctx->n_ns_slots) * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_wmaps), n * sizeof(CUtensorMap)) != cudaSuccess ||
-      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), 2 * sizeof(int)) != cudaSuccess)   // err, any_rewrite
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), (1 + kGroups) * sizeof(int)) != cudaSuccess)   // err, any_rewrite[]
     return fail(MUONH_ERR_OOM, "allocation of the device tables failed");
 
   std::vector<ClassDev> cdev;
@@ -562,17 +627,18 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   CUDA_TRY(cudaMemcpyAsync(ctx->d_classes, cdev.data(), cdev.size() * sizeof(ClassDev), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_et_mat, et_mat.data(), n_et * sizeof(int32_t), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_scal, scal.data(), n * sizeof(MatScal), cudaMemcpyHostToDevice, s));
-  CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, 2 * sizeof(int), s));
+  CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, (1 + kGroups) * sizeof(int), s));
 
-  // ---- Newton-Schulz tile lists, one pair per iteration (shared when equal)
+  // ---- Newton-Schulz tile lists, per group one pair per iteration (shared when equal)
+  for (muonh_ctx::Group& gr : ctx->groups) {
   std::vector<int32_t> prev_active;
   for (int32_t k = 0; k < ctx->max_steps; ++k) {
     std::vector<int32_t> active;
-    for (int32_t i = 0; i < n; ++i)
+    for (int32_t i = gr.m_first; i < gr.m_first + gr.m_count; ++i)
       if (ctx->mats[i].ns_steps > k) active.push_back(i);
     if (k > 0 && active == prev_active) {
-      ctx->gram_lists.push_back(ctx->gram_lists.back());
-      ctx->apply_lists.push_back(ctx->apply_lists.back());
+      gr.gram_lists.push_back(gr.gram_lists.back());
+      gr.apply_lists.push_back(gr.apply_lists.back());
       continue;
     }
     prev_active = active;
@@ -614,8 +680,9 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       CUDA_TRY(cudaMemcpyAsync(gl.dev, gram.data(), gram.size() * sizeof(TileDesc), cudaMemcpyHostToDevice, s));
     if (!apply.empty())
       CUDA_TRY(cudaMemcpyAsync(al.dev, apply.data(), apply.size() * sizeof(TileDesc), cudaMemcpyHostToDevice, s));
-    ctx->gram_lists.push_back(gl);
-    ctx->apply_lists.push_back(al);
+    gr.gram_lists.push_back(gl);
+    gr.apply_lists.push_back(al);
+  }
   }
 
   // ---- pinned staging ring for the per-step table
@@ -654,59 +721,107 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
   CUDA_TRY(cudaMemcpyAsync(ctx->d_step, ctx->h_step[slot], ctx->n * sizeof(MatStep), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaEventRecord(ctx->ev[slot], s));
 
-  const EwParams p = ctx->ew(stats);
-  const int grid = ctx->sm_count * 8;
   int launches = 0;
-  for (int tall = 0; tall < 2; ++tall)
-    if (ctx->any_wt[tall])
-      STEP_LAUNCH(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_warp(p, tall != 0, ctx->ew_warp_grid[tall], s),
-                  "momentum_warp");
-  if (ctx->any_general) STEP_LAUNCH(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_norm(p, grid, s), "momentum_norm");
-  STEP_LAUNCH(MUONH_PHASE_FINALIZE_INPUT, launch_finalize_input(p, s), "finalize_input");
-  STEP_LAUNCH(MUONH_PHASE_WRITE_X, launch_write_x(p, grid, s), "write_x");
-  for (int32_t k = 0; k < ctx->max_steps; ++k) {
-    NsParams np{};
-    np.mats = ctx->d_mats;
-    np.classes = ctx->d_classes;
-    np.tmaps = ctx->d_tmaps;
-    np.err = ctx->d_err;
-    np.src = k & 1;
-    np.iter = k;
-    np.scal = ctx->d_scal;
-    np.wmaps = ctx->d_wmaps;
-    np.part_ns = ctx->d_part_ns;
-    np.tiles = ctx->gram_lists[k].dev;
-    np.ntiles = ctx->gram_lists[k].count;
-    if (ctx->pairs) {
-      const int pairs_max = std::max(1, ctx->sm_count / 2);
-      const int gp = std::min(pairs_max, std::max(1, np.ntiles));
-      STEP_LAUNCH(MUONH_PHASE_NS_GRAM, launch_ns_gemm_pair(M_GRAM, ctx->prec, np, gp, s), "ns_gram");
-      STEP_LAUNCH(MUONH_PHASE_NS_SQUARE, launch_ns_gemm_pair(M_SQUARE, ctx->prec, np, gp, s), "ns_square");
-      np.tiles = ctx->apply_lists[k].dev;
-      np.ntiles = ctx->apply_lists[k].count;
-      const int amode = (k == ctx->max_steps - 1) ? M_APPLY_LAST : M_APPLY;
-      STEP_LAUNCH(MUONH_PHASE_NS_APPLY,
-                  launch_ns_gemm_pair(amode, ctx->prec, np, std::min(pairs_max, std::max(1, np.ntiles)), s),
-                  "ns_apply");
-    } else {
-      const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
-      STEP_LAUNCH(MUONH_PHASE_NS_GRAM, launch_ns_gemm(M_GRAM, ctx->prec, np, ggrid, s), "ns_gram");
-      STEP_LAUNCH(MUONH_PHASE_NS_SQUARE, launch_ns_gemm(M_SQUARE, ctx->prec, np, ggrid, s), "ns_square");
-      np.tiles = ctx->apply_lists[k].dev;
-      np.ntiles = ctx->apply_lists[k].count;
-      STEP_LAUNCH(MUONH_PHASE_NS_APPLY,
-                  launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), s),
-                  "ns_apply");
+  const int grid = ctx->sm_count * 8;
+  // elementwise grids: one resident wave, or short blocks when the launch
+  // overlaps the other group's GEMMs
+  auto ew_grid = [&](int kind, const muonh_ctx::Group& gr, bool overlap) {
+    if (!overlap) return ctx->ew_warp_grid[kind];
+    const int64_t tiles = gr.e_end - gr.e_first;
+    return static_cast<int>(std::max<int64_t>(1, (tiles + kOverlapTilesPerBlock - 1) / kOverlapTilesPerBlock));
+  };
+  auto front = [&](int g, cudaStream_t st, bool overlap) -> muonh_status {   // momentum, ||X||, X
+    const muonh_ctx::Group& gr = ctx->groups[g];
+    const EwParams p = ctx->ew(stats, g);
+    for (int tall = 0; tall < 2; ++tall)
+      if (gr.any_wt[tall])
+        STEP_LAUNCH_ON(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_warp(p, tall != 0, ew_grid(tall, gr, overlap), st),
+                       "momentum_warp", st);
+    if (gr.any_general) STEP_LAUNCH_ON(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_norm(p, grid, st), "momentum_norm", st);
+    STEP_LAUNCH_ON(MUONH_PHASE_FINALIZE_INPUT, launch_finalize_input(p, st), "finalize_input", st);
+    STEP_LAUNCH_ON(MUONH_PHASE_WRITE_X, launch_write_x(p, grid, st), "write_x", st);
+    return MUONH_OK;
+  };
+  auto newton_schulz = [&](int g, cudaStream_t st) -> muonh_status {
+    const muonh_ctx::Group& gr = ctx->groups[g];
+    for (int32_t k = 0; k < ctx->max_steps; ++k) {
+      NsParams np{};
+      np.mats = ctx->d_mats;
+      np.classes = ctx->d_classes;
+      np.tmaps = ctx->d_tmaps;
+      np.err = ctx->d_err;
+      np.src = k & 1;
+      np.iter = k;
+      np.scal = ctx->d_scal;
+      np.wmaps = ctx->d_wmaps;
+      np.part_ns = ctx->d_part_ns;
+      np.tiles = gr.gram_lists[k].dev;
+      np.ntiles = gr.gram_lists[k].count;
+      if (np.ntiles == 0) continue;   // no matrix of this group iterates k times
+      if (ctx->pairs) {
+        const int pairs_max = std::max(1, ctx->sm_count / 2);
+        const int gp = std::min(pairs_max, std::max(1, np.ntiles));
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_GRAM, launch_ns_gemm_pair(M_GRAM, ctx->prec, np, gp, st), "ns_gram", st);
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_SQUARE, launch_ns_gemm_pair(M_SQUARE, ctx->prec, np, gp, st), "ns_square", st);
+        np.tiles = gr.apply_lists[k].dev;
+        np.ntiles = gr.apply_lists[k].count;
+        const int amode = (k == ctx->max_steps - 1) ? M_APPLY_LAST : M_APPLY;
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_APPLY,
+                       launch_ns_gemm_pair(amode, ctx->prec, np, std::min(pairs_max, std::max(1, np.ntiles)), st),
+                       "ns_apply", st);
+      } else {
+        const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_GRAM, launch_ns_gemm(M_GRAM, ctx->prec, np, ggrid, st), "ns_gram", st);
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_SQUARE, launch_ns_gemm(M_SQUARE, ctx->prec, np, ggrid, st), "ns_square", st);
+        np.tiles = gr.apply_lists[k].dev;
+        np.ntiles = gr.apply_lists[k].count;
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_APPLY,
+                       launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), st),
+                       "ns_apply", st);
+      }
     }
+    return MUONH_OK;
+  };
+  auto back = [&](int g, cudaStream_t st, bool overlap) -> muonh_status {   // dots, projection, stats
+    const muonh_ctx::Group& gr = ctx->groups[g];
+    const EwParams p = ctx->ew(stats, g);
+    if (gr.any_unfused) STEP_LAUNCH_ON(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, st), "update_dots", st);
+    STEP_LAUNCH_ON(MUONH_PHASE_FINALIZE_UPDATE, launch_finalize_update(p, st), "finalize_update", st);
+    for (int tall = 0; tall < 2; ++tall)
+      if (gr.any_wt[tall])
+        STEP_LAUNCH_ON(MUONH_PHASE_PROJECT, launch_project_warp(p, tall != 0, ew_grid(2 + tall, gr, overlap), st),
+                       "project_warp", st);
+    if (gr.any_general) STEP_LAUNCH_ON(MUONH_PHASE_PROJECT, launch_project(p, grid, st), "project", st);
+    STEP_LAUNCH_ON(MUONH_PHASE_FINALIZE_STEP, launch_finalize_step(p, st), "finalize_step", st);
+    return MUONH_OK;
+  };
+  muonh_status st;
+  if (ctx->groups.size() == 1) {
+    if ((st = front(0, s, false)) || (st = newton_schulz(0, s)) || (st = back(0, s, false))) return st;
+  } else {
+    // caller's stream: front(0) | front(1) | back(0), front(2) | ... | back(G-1)
+    // GEMM stream:              | NS(0) ...| NS(1) ............| ... |
+    // group g's front work overlaps NS(g-1), its back work NS(g+1)
+    cudaStream_t hs = ctx->ns_stream;
+    const int G = static_cast<int>(ctx->groups.size());
+    if ((st = front(0, s, false))) return st;
+    CUDA_TRY(cudaEventRecord(ctx->gev[0], s));
+    for (int g = 0; g < G; ++g) {
+      CUDA_TRY(cudaStreamWaitEvent(hs, ctx->gev[2 * g], 0));
+      if ((st = newton_schulz(g, hs))) return st;
+      CUDA_TRY(cudaEventRecord(ctx->gev[2 * g + 1], hs));
+      if (g + 1 < G) {
+        if ((st = front(g + 1, s, true))) return st;
+        CUDA_TRY(cudaEventRecord(ctx->gev[2 * (g + 1)], s));   // before back(g - 1): NS(g + 1) need not wait for it
+      }
+      if (g >= 1) {
+        CUDA_TRY(cudaStreamWaitEvent(s, ctx->gev[2 * (g - 1) + 1], 0));
+        if ((st = back(g - 1, s, true))) return st;
+      }
+    }
+    CUDA_TRY(cudaStreamWaitEvent(s, ctx->gev[2 * (G - 1) + 1], 0));
+    if ((st = back(G - 1, s, false))) return st;
   }
-  if (ctx->any_unfused) STEP_LAUNCH(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, s), "update_dots");
-  STEP_LAUNCH(MUONH_PHASE_FINALIZE_UPDATE, launch_finalize_update(p, s), "finalize_update");
-  for (int tall = 0; tall < 2; ++tall)
-    if (ctx->any_wt[tall])
-      STEP_LAUNCH(MUONH_PHASE_PROJECT, launch_project_warp(p, tall != 0, ctx->ew_warp_grid[2 + tall], s),
-                  "project_warp");
-  if (ctx->any_general) STEP_LAUNCH(MUONH_PHASE_PROJECT, launch_project(p, grid, s), "project");
-  STEP_LAUNCH(MUONH_PHASE_FINALIZE_STEP, launch_finalize_step(p, s), "finalize_step");
   ctx->last_launches = launches;
   ctx->last_stream = s;
   ++ctx->step_count;

@@ -126,6 +126,10 @@ struct EwParams {
   const ClassDev* classes;
   const int32_t* et_mat;     // elementwise tile -> matrix
   int64_t n_et;
+  // the part of the step one launch covers: elementwise tiles [e_first,
+  // e_end) and matrices [m_first, m_first + m_count) (one finalize block each)
+  int64_t e_first, e_end;
+  int32_t m_first, m_count;
   float* part;               // per-tile partials
   float* part8;              // warp-tiled kernels: one partial per (tile, warp), 8 per tile
   double* part64;
@@ -135,7 +139,8 @@ struct EwParams {
   int32_t prec;
   muonh_stats* stats_out;
   const int* err;
-  int* any_rewrite;          // set by finalize_input when a matrix needs write_x; cleared by finalize_step
+  int* any_rewrite;          // this matrix group: set by finalize_input when a matrix needs write_x,
+                             // cleared by finalize_step
 };
 
 // -------------------------------------------------------------- PTX helpers

@@ -250,7 +250,7 @@ __device__ __forceinline__ int64_t skip_matrix(const MatDev& md, int64_t e) {
 // ------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kEwThreads) init_norm_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+  for (int64_t e = p.e_first + blockIdx.x; e < p.e_end; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     double acc = 0.0;
@@ -347,7 +347,7 @@ __device__ __forceinline__ float momentum_tile(const EwParams& p, const MatDev& 
 __global__ void __launch_bounds__(kEwThreads, 5) momentum_norm_kernel(const EwParams p) {
   __shared__ float red[kEwThreads / 32];
   __shared__ float tile[kEwTile][kEwTile + 1];
-  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+  for (int64_t e = p.e_first + blockIdx.x; e < p.e_end; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     if (md.warp_tiled) {
@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kEwThreads, 5) momentum_norm_kernel(const EwPa
 __global__ void __launch_bounds__(kEwThreads, 6) write_x_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   if (*reinterpret_cast<const volatile int*>(p.any_rewrite) == 0) return;   // every X already written
-  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+  for (int64_t e = p.e_first + blockIdx.x; e < p.e_end; e += gridDim.x) {
     const int mi = p.et_mat[e];
     if (!p.scal[mi].rewrite) {
       // the momentum kernel already wrote this matrix's X: jump past its tiles
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kEwThreads, 6) write_x_kernel(const EwParams p
 __global__ void __launch_bounds__(kEwThreads, 8) update_dots_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   __shared__ float red[kEwThreads / 32];
-  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+  for (int64_t e = p.e_first + blockIdx.x; e < p.e_end; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     if (md.fused_dots) continue;   // the last APPLY produced this matrix's partials
@@ -531,7 +531,7 @@ __device__ __forceinline__ float project_tile(const EwParams& p, const MatDev& m
 __global__ void __launch_bounds__(kEwThreads, 6) project_kernel(const EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
   __shared__ float red[kEwThreads / 32];
-  for (int64_t e = blockIdx.x; e < p.n_et; e += gridDim.x) {
+  for (int64_t e = p.e_first + blockIdx.x; e < p.e_end; e += gridDim.x) {
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     if (md.warp_tiled) {
@@ -603,7 +603,7 @@ __device__ double tile_partials(const EwParams& p, const MatDev& md, double* red
 
 __global__ void __launch_bounds__(kEwThreads) finalize_init_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = blockIdx.x;
+  const int mi = p.m_first + blockIdx.x;
   const MatDev& md = p.mats[mi];
   const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
   const double s = matrix_sum(p.part64, md.et_begin, cnt, 1, 0, red);
@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_init_kernel(const EwParam
 
 __global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = blockIdx.x;
+  const int mi = p.m_first + blockIdx.x;
   const MatDev& md = p.mats[mi];
   const double s = tile_partials(p, md, red);
   if (threadIdx.x == 0) {
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwPara
 
 __global__ void __launch_bounds__(kEwThreads) finalize_update_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = blockIdx.x;
+  const int mi = p.m_first + blockIdx.x;
   const MatDev& md = p.mats[mi];
   double soo, swo;
   if (md.fused_dots) {
@@ -729,7 +729,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_update_kernel(const EwPar
 
 __global__ void __launch_bounds__(kEwThreads) finalize_step_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = blockIdx.x;
+  const int mi = p.m_first + blockIdx.x;
   const MatDev& md = p.mats[mi];
   const double s = tile_partials(p, md, red);
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.any_rewrite = 0;   // write_x of this step has run
@@ -750,39 +750,39 @@ inline int ew_grid(int64_t n_et, int grid) {
 }  // namespace
 
 cudaError_t launch_init_norm(const EwParams& p, int grid, cudaStream_t s) {
-  init_norm_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  init_norm_kernel<<<ew_grid(p.e_end - p.e_first, grid), kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_finalize_init(const EwParams& p, cudaStream_t s) {
-  finalize_init_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  finalize_init_kernel<<<p.m_count, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_momentum_norm(const EwParams& p, int grid, cudaStream_t s) {
-  momentum_norm_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  momentum_norm_kernel<<<ew_grid(p.e_end - p.e_first, grid), kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_finalize_input(const EwParams& p, cudaStream_t s) {
-  finalize_input_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  finalize_input_kernel<<<p.m_count, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_write_x(const EwParams& p, int grid, cudaStream_t s) {
-  write_x_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  write_x_kernel<<<ew_grid(p.e_end - p.e_first, grid), kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_update_dots(const EwParams& p, int grid, cudaStream_t s) {
-  update_dots_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  update_dots_kernel<<<ew_grid(p.e_end - p.e_first, grid), kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_finalize_update(const EwParams& p, cudaStream_t s) {
-  finalize_update_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  finalize_update_kernel<<<p.m_count, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_project(const EwParams& p, int grid, cudaStream_t s) {
-  project_kernel<<<ew_grid(p.n_et, grid), kEwThreads, 0, s>>>(p);
+  project_kernel<<<ew_grid(p.e_end - p.e_first, grid), kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_finalize_step(const EwParams& p, cudaStream_t s) {
-  finalize_step_kernel<<<p.n, kEwThreads, 0, s>>>(p);
+  finalize_step_kernel<<<p.m_count, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_export_update(const EwParams& p, int mat, float* dst, int64_t ld, cudaStream_t s) {

@@ -73,10 +73,10 @@ __device__ __forceinline__ Tile tile_of(const MatDev& md, int64_t e) {
 }
 
 // Next tile of this block that belongs to a warp-tiled matrix of the
-// kernel's kind (wide or tall), or n_et.
+// kernel's kind (wide or tall), or e_end.
 template <bool TALL>
 __device__ __forceinline__ int64_t next_tile(const EwParams& p, int64_t e) {
-  while (e < p.n_et) {
+  while (e < p.e_end) {
     const MatDev& md = p.mats[p.et_mat[e]];
     if (md.warp_tiled && (md.transposed != 0) == TALL) return e;
     const int64_t end = md.et_begin + static_cast<int64_t>(md.et_rows) * md.et_cols;
@@ -104,7 +104,7 @@ template <bool TALL, bool PROJECT>
 __device__ __forceinline__ TileCtx tile_ctx(const EwParams& p, int64_t e) {
   TileCtx c;
   c.e = e;
-  if (e >= p.n_et) return c;
+  if (e >= p.e_end) return c;
   const int mi = p.et_mat[e];
   const MatDev& md = p.mats[mi];
   const Tile t = tile_of(md, e);
@@ -145,8 +145,8 @@ __device__ __forceinline__ void wide_chunk_sh(int sh, int w, int lane, int j, in
 template <bool TALL>
 __global__ void __launch_bounds__(kWarpThreads, 3) momentum_warp_kernel(const EwParams p) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  TileCtx cur = tile_ctx<TALL, false>(p, next_tile<TALL>(p, blockIdx.x));
-  while (cur.e < p.n_et) {
+  TileCtx cur = tile_ctx<TALL, false>(p, next_tile<TALL>(p, p.e_first + blockIdx.x));
+  while (cur.e < p.e_end) {
     const float beta = cur.s0, sigma = cur.s1;
     float acc = 0.f;
     if (!TALL) {
@@ -267,8 +267,8 @@ __global__ void __launch_bounds__(kWarpThreads, 3) momentum_warp_kernel(const Ew
 template <bool TALL>
 __global__ void __launch_bounds__(kWarpThreads, 3) project_warp_kernel(const EwParams p) {
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  TileCtx cur = tile_ctx<TALL, true>(p, next_tile<TALL>(p, blockIdx.x));
-  while (cur.e < p.n_et) {
+  TileCtx cur = tile_ctx<TALL, true>(p, next_tile<TALL>(p, p.e_first + blockIdx.x));
+  while (cur.e < p.e_end) {
     const int mode = cur.flag;
     const float kw = cur.s0, ko = cur.s1;
     float acc = 0.f;
