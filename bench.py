@@ -77,8 +77,18 @@ def ns_flops(shapes, steps):
 
 
 def apply_flops(shapes):
-    """One APPLY launch (Y' = aY + BY for every matrix): 2 r^2 c per matrix."""
+    """One APPLY pass over the set (Y' = aY + BY for every matrix): 2 r^2 c
+    per matrix.  A step makes ns_steps such passes; a large set splits each
+    pass into one launch per matrix group."""
     return sum(2 * min(a, b) ** 2 * max(a, b) for a, b in shapes)
+
+
+def apply_bytes(shapes):
+    """Algorithmic HBM bytes of one APPLY pass: read B' (r x r) and Y (r x c),
+    write Y', 16-bit, on the 256-padded Newton-Schulz buffers."""
+    def pad(v):
+        return (v + 255) // 256 * 256
+    return sum(2 * pad(min(a, b)) ** 2 + 4 * pad(min(a, b)) * pad(max(a, b)) for a, b in shapes)
 
 
 def load_peaks():
@@ -136,8 +146,9 @@ class ClockSampler:
 
 
 def committed_traffic(kernel_file, workload, prec):
-    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
-    or None when the kernel source changed since the counters were taken."""
+    """DRAM bytes of one APPLY pass over the set (the dominant kernel) from a
+    committed ncu summary, or None when the kernel source changed since the
+    counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -151,7 +162,7 @@ def committed_traffic(kernel_file, workload, prec):
         digest = hashlib.sha256(f.read()).hexdigest()
     if d[key].get("source_sha256") != digest:
         return None
-    return d[key]["dram_bytes_per_launch"]
+    return d[key]["dram_bytes_per_pass"]
 
 
 def max_over_ranks(value: float, world: int) -> float:
@@ -411,13 +422,16 @@ def run_ours(args):
         if name in KERNEL_BYTES:
             entry["gbps"] = KERNEL_BYTES[name] * elems / (tms / args.steps / 1000.0) / 1e9
         kernels[name] = entry
+    # APPLY FLOPs of the timed region over the APPLY launches' summed device time
     apply_ms, apply_n = phases["ns_apply"]
-    ap_flops = apply_flops(shapes)
-    achieved = ap_flops / (apply_ms / apply_n / 1000.0) / 1e12
+    ap_flops = apply_flops(shapes) * wl.ns_steps * args.steps
+    achieved = ap_flops / (apply_ms / 1000.0) / 1e12
     peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     roofline = {"bound": "tensor", "kernel": "ns_apply", "achieved": achieved, "peak": peak_t,
                 "unit": "TFLOP/s", "frac": achieved / peak_t,
                 "traffic": committed_traffic("muonh_ns_gemm.cu", args.workload, args.ns_precision),
+                "per": "one APPLY pass over the set (5 a step; one launch per matrix group)",
+                "algorithmic_bytes": apply_bytes(shapes),
                 "peak_source": f"bf16_tflops_sustained ({peak_src}); fp16 operands run at the bf16 rate"}
     ns_ms = sum(phases[k][0] for k in ("ns_gram", "ns_square", "ns_apply")) / args.steps
     ew_ms = sum(phases[k][0] for k in ELEMENTWISE) / args.steps
