@@ -138,7 +138,10 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
  *   stats  NULL, or device-accessible memory (device, managed or mapped
  *          pinned host) for n muonh_stats, written by the last kernel.
  * Updates every w and m in place.  Enqueued on `stream`; the caller
- * synchronises before reading w, m or stats. */
+ * synchronises before reading w, m or stats.  A large set (>= 16M elements)
+ * also runs its Newton-Schulz GEMMs on an internal stream of the context;
+ * `stream` waits for that work before the step's last kernels, so the step
+ * is complete in `stream`'s order like any single-stream launch sequence. */
 muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* grads,
                         muonh_stats* stats, void* stream);
 

@@ -4,17 +4,22 @@
 // (r_pad x c_pad, r = min(rows, cols) on the wide orientation, both padded
 // to multiples of 256), allocates one zero-filled workspace per shape class
 // ([count][r_pad][c_pad] iterate ping-pong buffers and [count][r_pad][r_pad]
-// buffers for A = Y Y^T, C = b I + c A and B' = a I + A C), encodes one TMA descriptor per buffer and
-// box shape, and builds the tile lists of the grouped GEMM launches.  Zero
-// padding is exact for the iteration: padded rows and columns of Y, A and B
-// stay zero, so no GEMM tile is ragged.
+// buffers for A = Y Y^T and B' = a I + b A + c A A, plus C = b I + c A in
+// FP32 mode), encodes one TMA descriptor per buffer and box shape, and
+// builds the tile lists of the grouped GEMM launches.  Zero padding is exact
+// for the iteration: padded rows and columns of Y, A and B' stay zero, so no
+// GEMM tile is ragged.
 //
-// muonh_step enqueues, on the caller's stream:
-//   momentum_norm  (M update, ||X||^2 partials)      -> finalize_input
-//   write_x        (X / (||X|| + eps), 16-bit, wide orientation)
-//   ns_steps x { GRAM, SQUARE, APPLY }               (tcgen05 GEMMs)
-//   update_dots    (||O||^2, <W, O> partials)        -> finalize_update
-//   project        (W <- R (W - lr R O/||O||) / ||.||, Eq. (1)) -> finalize_step
+// muonh_step enqueues, per matrix group:
+//   momentum       (M update, ||X||^2 partials, 16-bit X)       -> finalize_input
+//   write_x        (rewrites X where the momentum pass's scale was unsafe)
+//   ns_steps x { GRAM, SQUARE, APPLY }   (tcgen05 GEMMs; the last APPLY also
+//                                         forms ||O||^2 and <W, O>)
+//   update_dots    (only matrices the last APPLY does not cover) -> finalize_update
+//   project        (W <- R (W - lr R O/||O||) / ||.||, Eq. (1))  -> finalize_step
+// One group runs everything on the caller's stream.  With two groups the
+// GEMMs move to an internal highest-priority stream, and each group's
+// elementwise launches overlap the other group's GEMMs (see muonh_step).
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>

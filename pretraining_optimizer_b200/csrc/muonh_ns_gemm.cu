@@ -4,7 +4,7 @@
 //   Y' = a Y + (b A + c A A) Y,   A = Y Y^T
 // (quintic iteration of the Muon update; the MuonH wrapper of the Puro-2B
 // report, Sec. 3.3, normalises its output), runs as three products with the
-// polynomial folded into the products:
+// polynomial folded into the products (16-bit operands, CTA pairs):
 //   GRAM    A  = Y Y^T  (and, FP32 mode, C = b I + c A)    M = r, N = r, K = c   (symmetric)
 //   SQUARE  B' = c A A + b A + a I  (FP32 mode: A C + a I)  M = r, N = r, K = r   (symmetric)
 //   APPLY   Y' = B' Y                                      M = r, N = c, K = r
