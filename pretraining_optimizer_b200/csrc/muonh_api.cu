@@ -583,9 +583,6 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           return st;
         if ((st = encode_map(&m[TM_B_ST], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
-        // SQUARE epilogue: A chunks of 128 rows x 32 columns
-        if ((st = encode_map(&m[TM_A_EPI], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, 128, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
-          return st;
       }
     }
   }

@@ -28,7 +28,7 @@ enum Mode { M_GRAM = 0, M_SQUARE = 1, M_APPLY = 2, M_APPLY_LAST = 3 };   // LAST
 
 // Tensor-map slots of one shape class.  "hi" buffers hold the 16-bit
 // operand (fp16/bf16), "lo" buffers the fp16 residual in FP32 mode.  The
-// CTA-pair kernels (16-bit operands) use the store boxes and TM_A_EPI; the
+// CTA-pair kernels (16-bit operands) use the store boxes; the
 // FP32-mode kernel stores directly and also reads C = b I + c A.
 enum TmSlot {
   TM_X_K128 = 0,   // X[buf] as K-major operand, 128-row box   (+buf, +2*part)
@@ -40,8 +40,7 @@ enum TmSlot {
   TM_X_ST = 18,    // X[buf] store box 32 x 32 (64-byte swizzle)   (+buf)
   TM_A_ST = 20,    // A store box (direct and mirrored blocks)
   TM_B_ST = 21,    // B' store box (direct and mirrored blocks)
-  TM_A_EPI = 22,   // A box of 128 rows x 32 columns staged by the SQUARE epilogue (64-byte swizzle)
-  TM_PER_CLASS = 23
+  TM_PER_CLASS = 22
 };
 __host__ __device__ inline int tm_x(int base, int buf, int part) { return base + buf + 2 * part; }
 

@@ -457,9 +457,8 @@ struct PairCfg {
   // the last APPLY gives staging space to the fp32 W boxes of its <W, O> partials
   static constexpr bool kLast = MODE == M_APPLY_LAST;
   static constexpr bool kSquare = MODE == M_SQUARE;
-  // SQUARE trades an operand stage for deeper staging of its epilogue A boxes
-  static constexpr int kStages = kSquare ? 4 : 5;
-  static constexpr int kWBufs = kSquare ? 4 : 2;
+  static constexpr int kStages = 5;
+  static constexpr int kWBufs = 2;
   static constexpr int kABytes = 128 * kBK * 2;                 // 16 KB: this CTA's 128 rows
   static constexpr int kBBytes = 128 * kBK * 2;                 // 16 KB: this CTA's half of N
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -478,13 +477,11 @@ struct PairCfg {
   static constexpr int kWarpBox = 32 * 32 * 2;
   static constexpr int kWarpBufs = kLast ? 2 : 4;
   static constexpr int kStoreOffset = (kMirrorOffset + kMirrorBytes + 1023) / 1024 * 1024;
-  // Epilogue operand staging, kWBufs buffers filled kWBufs chunks ahead: the
-  // last APPLY's fp32 W boxes (128 rows x 32 columns, or 32 x 128 for a tall
-  // W) for the <W, O> partials; SQUARE's 16-bit A boxes (128 rows x 32
-  // columns, 64-byte swizzle) for its b A term
-  static constexpr int kWBox = kLast ? 128 * 32 * 4 : 128 * 32 * 2;
+  // Last APPLY: kWBufs fp32 W boxes (128 rows x 32 columns, or 32 x 128 for
+  // a tall W) filled kWBufs chunks ahead, for the <W, O> partials
+  static constexpr int kWBox = 128 * 32 * 4;
   static constexpr int kWOffset = kStoreOffset + kEpiWarps * kWarpBufs * kWarpBox;
-  static constexpr int kSmem = kWOffset + ((kLast || kSquare) ? kWBufs * kWBox : 0) + 1024;
+  static constexpr int kSmem = kWOffset + (kLast ? kWBufs * kWBox : 0) + 1024;
 };
 
 // Row `r` (0..31) of a 32 x 32 16-bit box, 16-byte piece q, in the 64-byte
@@ -702,8 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
     int w_pending[C::kWBufs] = {};     // thread 64: staged loads issued and not yet consumed
     int w_issued[C::kWBufs] = {};      // thread 64: loads issued into each buffer so far
     bool werr = false;
-    // thread 64 loads the epilogue operand of chunk `chk` into buffer b: the
-    // last APPLY's W box, or SQUARE's A box (rows row0.., chunk columns)
+    // thread 64 loads the last APPLY's W box of chunk `chk` into buffer b
     auto w_issue = [&](const TileDesc& td, const MatDev& md, const ClassDev& cd, int row0, int b, int chk) {
       const int c0 = td.bj * kBN + chk * 32;
       // the buffer's previous contents must have been read by all epilogue warps
@@ -714,9 +710,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
       ++w_issued[b];
       mbar_expect_tx(&wfull[b], C::kWBox);
       uint8_t* dst = smem + C::kWOffset + b * C::kWBox;
-      if (C::kSquare)
-        tma_load_3d(dst, p.tmaps + cd.tm_base + TM_A_EPI, &wfull[b], c0, row0, md.z);
-      else if (!md.transposed)
+      (void)cd;
+      if (!md.transposed)
         tma_load_2d(dst, p.wmaps + td.mat, &wfull[b], c0, row0);
       else
         tma_load_2d(dst, p.wmaps + td.mat, &wfull[b], row0, c0);
@@ -729,9 +724,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
       const ClassDev& cd = p.classes[md.cls];
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      if (threadIdx.x == 64 && (C::kSquare || (C::kLast && md.fused_dots && p.iter == md.ns_steps - 1))) {
+      if (threadIdx.x == 64 && C::kLast && md.fused_dots && p.iter == md.ns_steps - 1) {
         const int r0 = td.bi * kPairM + static_cast<int>(rank) * 128;
         for (int b = 0; b < C::kWBufs; ++b) w_issue(td, md, cd, r0, b, b);   // first chunks while the MMAs run
+      }
+      // SQUARE reads A[row][bj block] (written by GRAM, read-only here) for its
+      // b A term straight from L2, one 32-column chunk ahead
+      const uint16_t* arow = nullptr;
+      uint4 a_next[4];
+      if (C::kSquare) {
+        const int row_a = td.bi * kPairM + static_cast<int>(rank) * 128 + lrow;
+        arow = static_cast<const uint16_t*>(cd.a[0]) + md.z * cd.a_stride + static_cast<int64_t>(row_a) * cd.r_pad +
+               td.bj * kBN;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a_next[q] = __ldg(reinterpret_cast<const uint4*>(arow + ch0 * 32) + q);
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
       tc_fence_after();
@@ -766,7 +772,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         }
       } else if (MODE == M_SQUARE) {
         // stored B' = 2^eb (c A A + b A + a I), from the product of the stored
-        // A (2^ea A) with itself and the staged 2^ea A of this chunk
+        // A (2^ea A) with itself and the stored A of this chunk (read from L2)
         const float s2 = md.c_coef * exp2f(static_cast<float>(md.eb - 2 * md.ea));
         const float s1 = md.b * exp2f(static_cast<float>(md.eb - md.ea));
         const float diag = md.a * exp2f(static_cast<float>(md.eb));
@@ -779,24 +785,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader[acc]);
           }
-          const int b = ch % C::kWBufs;
-          if (!mbar_wait(&wfull[b], wphase[b], p.err)) { werr = true; break; }
-          wphase[b] ^= 1u;
-          if (threadIdx.x == 64) --w_pending[b];
-          {
-            // row lrow of the staged 128 x 32 box (64-byte swizzle)
-            const uint8_t* ab = smem + C::kWOffset + b * C::kWBox;
+          uint4 a_cur[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 u = *reinterpret_cast<const uint4*>(ab + store_box_offset(lrow, q));
-              const T16* h = reinterpret_cast<const T16*>(&u);
+          for (int q = 0; q < 4; ++q) a_cur[q] = a_next[q];
+          if (ch + kChStep < kBN / 32) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) v[8 * q + e] = fmaf(s2, v[8 * q + e], s1 * Store16<PREC>::back(h[e]));
-            }
+            for (int q = 0; q < 4; ++q) a_next[q] = __ldg(reinterpret_cast<const uint4*>(arow + (ch + kChStep) * 32) + q);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&wempty[b]);   // this warp is done with A buffer b
-          if (threadIdx.x == 64 && ch + C::kWBufs < kBN / 32) w_issue(td, md, cd, row0, b, ch + C::kWBufs);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const T16* h = reinterpret_cast<const T16*>(&a_cur[q]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[8 * q + e] = fmaf(s2, v[8 * q + e], s1 * Store16<PREC>::back(h[e]));
+          }
           const int dj = row - col0;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
