@@ -216,6 +216,14 @@ def blas_threads():
         return os.cpu_count()
 
 
+def bench_config(args, wl, shapes, world):
+    """The workload description both arms report."""
+    return {"workload": args.workload, "matrices": len(shapes), "params": sum(a * b for a, b in shapes),
+            "ns_steps": wl.ns_steps, "ns_precision": args.ns_precision, "state": "fp32 W, M, G",
+            "lr": "workload schedule", "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"{world} independent replica(s)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -238,7 +246,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * full_step_s,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "ns_steps": wl.ns_steps},
+            "data": "synthetic", "config": bench_config(args, wl, shapes, 1),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -463,11 +471,7 @@ def run_ours(args):
                 "vs_baseline": None, "dtype": "f16" if args.ns_precision == "fp16" else
                 ("bf16" if args.ns_precision == "bf16" else "f32"),
                 "data": "synthetic",
-                "config": {"workload": args.workload, "matrices": n, "params": elems,
-                           "ns_steps": wl.ns_steps, "ns_precision": args.ns_precision,
-                           "state": "fp32 W, M, G", "lr": "workload schedule",
-                           "l2": "inputs larger than L2 (no flush)",
-                           "parallelism": f"{world} independent replica(s)"},
+                "config": bench_config(args, wl, shapes, world),
                 "roofline": roofline, "summary": summary, "kernels": kernels, "clocks": clocks,
                 "gpu_launches": launches_per_step * args.steps, "e2e": e2e, "cpu_baseline": cpu,
                 "aux_kernels": aux}
