@@ -257,3 +257,20 @@ def test_two_group_schedule_with_general_path_matrices():
     for t, lr in enumerate(lrs):
         st = g["stats"][t][0]
         assert st["flags"] == 0 and abs(st["post_norm"] - R0) <= NORM_TOL * R0 and abs(st["elr"] - lr) <= NORM_TOL * lr
+
+
+@pytest.mark.parametrize("prec", ["fp16", "bf16"])
+@pytest.mark.parametrize("shape", [(256, 512), (1000, 300)])
+def test_error_matches_the_storage_emulation(prec, shape):
+    """The kernel stores Y, A and B' in 16 bits and accumulates in fp32: its
+    NS error against fp64 matches the oracle's 16-bit storage emulation (the
+    same roundings, in another summation order) to within 25 %."""
+    from oracle import emulate
+    W0 = [synth.initial_weight(0, *shape)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shape)
+    g = run_gpu(W0, grad, [0.01], prec=prec, keep_updates=(0,))
+    M, X = oracle.momentum_update(np.zeros(shape), grad(0, 0), 0.95, True)
+    ref = oracle.newton_schulz(X)
+    emu = rel_fro(emulate.newton_schulz_stored(X, storage=prec), ref)
+    err = rel_fro(g["O"][0][0], ref)
+    assert 0.8 * emu <= err <= 1.25 * emu, (err, emu)

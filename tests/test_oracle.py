@@ -6,6 +6,7 @@ import numpy as np
 import pytest
 
 import oracle
+import synth
 from oracle import QUINTIC
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -195,3 +196,36 @@ def test_elr_aligned_rule_hits_the_prescribed_elr():
         assert np.allclose(W1, W3, rtol=0, atol=1e-15)
         # no projection: the norm drifts from ||W_0||
         assert abs(np.linalg.norm(W1) - np.linalg.norm(W)) > 1e-6
+
+
+# ---------------------------------------------------------------- 16-bit storage emulation
+def test_storage_emulation_without_rounding_is_the_oracle():
+    from oracle import emulate
+    X = synth.gaussian_gradient(0, 0, 64, 160)
+    assert np.allclose(emulate.newton_schulz_stored(X, storage="fp64"), oracle.newton_schulz(X), rtol=0, atol=1e-13)
+
+
+def test_round_helpers_match_their_formats():
+    """fp16: the library cast after an exact power-of-two scaling; bf16: the
+    top 16 bits of fp32, rounded to nearest even (ties checked by hand)."""
+    from oracle import emulate
+    x = np.random.default_rng(0).standard_normal(1000) * 1e-4
+    r = emulate.round_fp16(x)
+    assert np.all(np.abs(r - x) <= 2.0 ** -11 * np.abs(x) + 1e-300)
+    # 1 + 2^-8 is a bf16 tie between 1 and 1 + 2^-7: even mantissa wins (1.0);
+    # 1 + 3 * 2^-8 ties between 1 + 2^-7 and 1 + 2^-6: 1 + 2^-6 is even
+    ties = emulate.round_bf16(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -9)]))
+    assert list(ties) == [1.0, 1 + 2.0 ** -6, -1.0]
+
+
+@pytest.mark.parametrize("storage,lo,hi", [("fp16", 4e-4, 2e-3), ("bf16", 3e-3, 1.6e-2)])
+def test_storage_error_of_each_operand_format(storage, lo, hi):
+    """5 tuned quintic steps on a 256 x 512 Gaussian input: storing the
+    operands in fp16 (10+1 significand bits) costs ~1e-3 relative error,
+    bf16 (7+1 bits) about 8x more; the 1e-2 gate admits fp16 with margin."""
+    from oracle import emulate
+    X = synth.gaussian_gradient(0, 0, 256, 512)
+    ref = oracle.newton_schulz(X)
+    O = emulate.newton_schulz_stored(X, storage=storage)
+    err = np.linalg.norm(O - ref) / np.linalg.norm(ref)
+    assert lo <= err <= hi, err
