@@ -12,7 +12,9 @@ something other than itself: the singular-value form of the Newton-Schulz
 polynomial checked with a library SVD, convergence to the polar factor with
 a convergent coefficient set, the closed-form hyperball invariants
 (||W_{t+1}||_F = R, effective LR = lr), a hand-solved two-element example,
-and the geometric-sum form of the momentum buffer.
+and the geometric-sum form of the momentum buffer.  oracle.aux (checkpoint
+averaging, AdamW) and oracle.emulate (16-bit storage emulation of the
+iteration) are pinned in tests/test_oracle_aux.py and tests/test_oracle.py.
 """
 from .muonh import (  # noqa: F401
     QUINTIC, FLAG_NONFINITE_INPUT, FLAG_ZERO_UPDATE, FLAG_NONFINITE_UPDATE,
