@@ -370,26 +370,37 @@ def run_ours(args):
     # ---------------- end to end through the public API, host buffers
     e2e = None
     if not args.no_e2e:
-        host = [torch.empty(s, dtype=torch.float32, pin_memory=True) for s in shapes]
-        for h, g in zip(host, G):
+        # gradients as views of one contiguous arena (a training framework's
+        # gradient buffer), host side in pinned memory: one copy per step
+        sizes = [a * b for a, b in shapes]
+        offs = [0]
+        for sz in sizes:
+            offs.append(offs[-1] + (sz + 63) // 64 * 64)   # 256-byte aligned views
+
+        def views(flat):
+            return [flat[o:o + sz].view(s) for o, sz, s in zip(offs, sizes, shapes)]
+
+        host_flat = torch.empty(offs[-1], dtype=torch.float32, pin_memory=True)
+        for h, g in zip(views(host_flat), G):
             h.copy_(g)
         stats_dev = torch.empty(n * 6, dtype=torch.int32, device=dev)
         stats_host = torch.empty(n * 6, dtype=torch.int32, pin_memory=True)
         e2e_steps = max(1, min(args.steps, 10))
-        # two device gradient buffers: the upload of step k+1's gradients (copy
+        # two device gradient arenas: the upload of step k+1's gradients (copy
         # stream) overlaps step k; each step waits for its own upload
         copy = torch.cuda.Stream(device=dev)
-        gbuf = [G, [torch.empty_like(g) for g in G]]
+        dev_flat = [torch.empty(offs[-1], dtype=torch.float32, device=dev) for _ in range(2)]
+        gbuf = [views(f) for f in dev_flat]
         ready = [torch.cuda.Event(), torch.cuda.Event()]
         free = [torch.cuda.Event(), torch.cuda.Event()]
 
         def upload(b):
             with torch.cuda.stream(copy):
-                for g, h in zip(gbuf[b], host):
-                    g.copy_(h, non_blocking=True)
+                dev_flat[b].copy_(host_flat, non_blocking=True)
                 ready[b].record(copy)
 
-        opt.step(G, lrs[0])
+        upload(0)
+        opt.step(gbuf[0], lrs[0])      # warm the arena's gradient maps and pages
         torch.cuda.synchronize()
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
@@ -411,11 +422,11 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-        h2d = sum(4 * a * b for a, b in shapes)
+        h2d = 4 * offs[-1]
         e2e = {"value": whole_job_rate(world, e2e_steps, e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": 24 * n, "steps": e2e_steps,
                "pipeline": "gradient upload of step k+1 (pinned host -> device, copy stream) overlaps step k"}
-        del host, gbuf
+        del host_flat, gbuf, dev_flat
 
     # ---------------- rooflines from the live per-kernel events
     peaks, peak_src = load_peaks()
