@@ -57,3 +57,51 @@ def test_status_strings_and_argument_checks_without_a_gpu():
     d[0] = B.MatrixDesc(0x1000, 0x2000, 4, 8, 8, 0.0, 0.95, 1, 5, 3.4445, -4.775, 2.0315)
     assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(cfg_bad), None) == 1
     assert lib.muonh_step(None, None, None, None, None) == 1
+
+
+def _desc(**kw):
+    base = dict(w=0x1000, m=0x2000, rows=4, cols=8, ld=8, radius=0.0, beta=0.95, nesterov=1, ns_steps=5,
+                ns_a=3.4445, ns_b=-4.775, ns_c=2.0315, update_rule=0, weight_decay=0.0, update_scale=1.0)
+    base.update(kw)
+    d = (B.MatrixDesc * 1)()
+    d[0] = B.MatrixDesc(*[base[f] for f, _ in B.MatrixDesc._fields_])
+    return d
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(rows=0), 1), (dict(cols=0), 1),                      # empty matrices
+    (dict(rows=1 << 21), 1),                                   # beyond the largest dimension
+    (dict(rows=16640, cols=16640, ld=16640), 6),               # Newton-Schulz side above 16384: unsupported
+    (dict(update_rule=3), 1),                                  # unknown update rule
+    (dict(update_rule=1, update_scale=0.0), 1),                # ordinary Muon needs a positive scale
+    (dict(beta=float("nan")), 1),                              # non-finite momentum
+])
+def test_descriptor_edge_cases_without_a_gpu(kw, status):
+    """Every descriptor check runs before the first CUDA call."""
+    lib = P.library()
+    ctx = ctypes.c_void_p()
+    cfg = B.Config(0, 1e-7)
+    assert lib.muonh_init(ctypes.byref(ctx), _desc(**kw), 1, ctypes.byref(cfg), None) == status
+    assert ctx.value is None and lib.muonh_last_error()
+
+
+def test_auxiliary_argument_checks_without_a_gpu():
+    lib = P.library()
+    ptrs = (ctypes.c_void_p * 17)(*([0x1000] * 17))
+    assert lib.muonh_average(0x1000, 0, ptrs, 0, 0, 16, None) == 1       # k = 0
+    assert lib.muonh_average(0x1000, 0, ptrs, 0, 17, 16, None) == 1      # k above 16
+    assert lib.muonh_average(0x1000, 5, ptrs, 0, 2, 16, None) == 1       # unknown dtype
+    assert lib.muonh_average(0x1000, 0, ptrs, 0, 2, -1, None) == 1       # negative count
+    assert lib.muonh_average(0x1004, 0, ptrs, 0, 2, 16, None) == 2       # misaligned output
+    assert lib.muonh_average(None, 0, ptrs, 0, 2, 0, None) == 0          # empty: nothing to do
+    cfg = B.AdamWConfig(1e-3, 0.9, 0.95, 1e-8, 0.1)
+    t = (B.AdamWTensor * 1)(B.AdamWTensor(0x1000, 0x2000, 0x3000, 0x4000, 8))
+    assert lib.muonh_adamw_step(t, 1, ctypes.byref(cfg), 0, None) == 1   # step counts from 1
+    bad = B.AdamWConfig(1e-3, 1.0, 0.95, 1e-8, 0.1)
+    assert lib.muonh_adamw_step(t, 1, ctypes.byref(bad), 1, None) == 1   # beta1 must be < 1
+    t[0] = B.AdamWTensor(0x1002, 0x2000, 0x3000, 0x4000, 8)
+    assert lib.muonh_adamw_step(t, 1, ctypes.byref(cfg), 1, None) == 2   # not 4-byte aligned
+    assert lib.muonh_adamw_step(t, 0, ctypes.byref(cfg), 1, None) == 0   # no tensors
+    x = ctypes.c_void_p(0x5000)
+    assert lib.muonh_momentum_norm_noalloc(0x1000, 0x2000, 0, 8, 8, 0.95, 1, x, None) == 1   # empty
+    assert lib.muonh_momentum_norm_noalloc(0x1008, 0x2000, 4, 8, 8, 0.95, 1, x, None) == 2  # misaligned
