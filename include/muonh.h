@@ -275,6 +275,16 @@ typedef struct {
 muonh_status muonh_adamw_step(const muonh_adamw_tensor* tensors, int32_t n, const muonh_adamw_config* cfg,
                               int64_t step, void* stream);
 
+/* Diagnostic of the failure path every pipelined kernel uses (the report has
+ * no counterpart).  Launches one thread that waits on an mbarrier nothing
+ * will ever complete, with the same bounded wait as the kernels but a limit
+ * of `seconds` (0 < seconds <= 10) instead of 2 s.  The wait gives up,
+ * records the failure in a device flag, and the kernel returns, so no GPU
+ * hangs.  Returns MUONH_ERR_TIMEOUT when that happened, which is the
+ * expected outcome; MUONH_ERR_CUDA if the wait did not give up or a CUDA
+ * call failed.  Allocates and frees a 4-byte flag; synchronises `stream`. */
+muonh_status muonh_check_wait_timeout(double seconds, void* stream);
+
 void muonh_destroy(muonh_ctx* ctx);
 
 const char* muonh_status_string(muonh_status s);

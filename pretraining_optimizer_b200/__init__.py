@@ -9,5 +9,5 @@ from .muonh import (  # noqa: F401
     MuonH, MuonHError, QUINTIC, NS_FP16, NS_BF16, NS_FP32,
     FLAG_NONFINITE_INPUT, FLAG_ZERO_UPDATE, FLAG_NONFINITE_UPDATE, FLAG_DEGENERATE,
     FLAG_TIMEOUT, PHASES, library, library_path, EXPORTED_SYMBOLS, momentum_norm_noalloc,
-    average, adamw_step,
+    average, adamw_step, check_wait_timeout,
 )

@@ -929,6 +929,23 @@ muonh_status muonh_device_status(muonh_ctx* ctx) {
 
 int32_t muonh_last_launch_count(const muonh_ctx* ctx) { return ctx ? ctx->last_launches : 0; }
 
+muonh_status muonh_check_wait_timeout(double seconds, void* stream) {
+  g_last_error.clear();
+  if (!(seconds > 0.0 && seconds <= 10.0)) return fail(MUONH_ERR_INVALID_ARG, "seconds must be in (0, 10]");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* d_flag = nullptr;
+  CUDA_TRY(cudaMalloc(&d_flag, sizeof(int)));
+  int flag = 0;
+  cudaError_t e = cudaMemsetAsync(d_flag, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = launch_wait_probe(d_flag, static_cast<uint64_t>(seconds * 1e9), s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&flag, d_flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  cudaFree(d_flag);
+  if (e != cudaSuccess) return fail(MUONH_ERR_CUDA, "wait probe: %s", cudaGetErrorString(e));
+  if (!flag) return fail(MUONH_ERR_CUDA, "wait probe: the bounded wait did not give up");
+  return fail(MUONH_ERR_TIMEOUT, "wait probe: the bounded wait gave up as designed");
+}
+
 muonh_status muonh_enable_timing(muonh_ctx* ctx, int32_t enable) {
   g_last_error.clear();
   if (!ctx) return fail(MUONH_ERR_INVALID_ARG, "ctx is NULL");

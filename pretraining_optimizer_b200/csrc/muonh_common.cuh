@@ -182,16 +182,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity; gives up after kWaitLimitNs or
-// when another role already recorded an error.  Returns false on give-up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// Wait for the phase with the given parity; gives up after limit_ns (every
+// kernel uses kWaitLimitNs) or when another role already recorded an error.
+// Returns false on give-up, after recording the error in *err.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((spin & 255u) == 0u) {
       if (*reinterpret_cast<volatile int*>(err) != 0) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         atomicOr(err, 1);
         return false;
       }
@@ -414,6 +416,7 @@ cudaError_t launch_finalize_update(const EwParams& p, cudaStream_t s);
 cudaError_t launch_project(const EwParams& p, int grid, cudaStream_t s);
 cudaError_t launch_finalize_step(const EwParams& p, cudaStream_t s);
 cudaError_t launch_export_update(const EwParams& p, int mat, float* dst, int64_t ld, cudaStream_t s);
+cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s);
 int ew_warp_blocks_per_sm(int kind);
 cudaError_t launch_momentum_warp(const EwParams& p, bool tall, int grid, cudaStream_t s);
 cudaError_t launch_project_warp(const EwParams& p, bool tall, int grid, cudaStream_t s);

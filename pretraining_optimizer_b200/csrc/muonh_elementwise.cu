@@ -743,6 +743,18 @@ __global__ void __launch_bounds__(kEwThreads) finalize_step_kernel(const EwParam
   }
 }
 
+// One thread waits on an mbarrier that nothing arrives on, with the bounded
+// wait of the pipelined kernels: it must give up after limit_ns and record
+// the failure in *err.
+__global__ void wait_probe_kernel(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0u, err, limit_ns);
+  }
+}
+
 inline int ew_grid(int64_t n_et, int grid) {
   return static_cast<int>(n_et < grid ? (n_et > 0 ? n_et : 1) : grid);
 }
@@ -781,6 +793,11 @@ cudaError_t launch_project(const EwParams& p, int grid, cudaStream_t s) {
   project_kernel<<<ew_grid(p.e_end - p.e_first, grid), kEwThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
+cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_finalize_step(const EwParams& p, cudaStream_t s) {
   finalize_step_kernel<<<p.m_count, kEwThreads, 0, s>>>(p);
   return cudaGetLastError();

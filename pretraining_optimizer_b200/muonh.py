@@ -25,7 +25,7 @@ EXPORTED_SYMBOLS = (
     "muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
     "muonh_export_state", "muonh_import_state", "muonh_device_status", "muonh_last_launch_count",
     "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc", "muonh_average",
-    "muonh_adamw_step", "muonh_destroy", "muonh_status_string", "muonh_last_error",
+    "muonh_adamw_step", "muonh_check_wait_timeout", "muonh_destroy", "muonh_status_string", "muonh_last_error",
 )
 DTYPE_F32, DTYPE_BF16 = 0, 1
 AVERAGE_MAX_INPUTS = 16
@@ -97,6 +97,7 @@ def library() -> ctypes.CDLL:
                                                 c_int32, c_void_p, c_void_p]
     lib.muonh_average.argtypes = [c_void_p, c_int32, POINTER(c_void_p), c_int32, c_int32, c_int64, c_void_p]
     lib.muonh_adamw_step.argtypes = [POINTER(AdamWTensor), c_int32, POINTER(AdamWConfig), c_int64, c_void_p]
+    lib.muonh_check_wait_timeout.argtypes = [ctypes.c_double, c_void_p]
     lib.muonh_destroy.argtypes = [c_void_p]
     lib.muonh_destroy.restype = None
     lib.muonh_status_string.argtypes = [c_int32]
@@ -106,7 +107,7 @@ def library() -> ctypes.CDLL:
     for name in ("muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
                  "muonh_export_state", "muonh_import_state", "muonh_device_status",
                  "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc",
-                 "muonh_average", "muonh_adamw_step"):
+                 "muonh_average", "muonh_adamw_step", "muonh_check_wait_timeout"):
         getattr(lib, name).restype = c_int32
     _LIB = lib
     return lib
@@ -149,6 +150,12 @@ def momentum_norm_noalloc(m, g, beta=0.95, nesterov=True, x_norm=None, stream=No
     _check(library().muonh_momentum_norm_noalloc(mp, gp, rows, cols, ld, float(beta), int(bool(nesterov)),
                                                  x_norm.data_ptr(), _stream_handle(stream)))
     return x_norm
+
+
+def check_wait_timeout(seconds: float = 0.2, stream=None) -> int:
+    """Run the bounded-wait failure probe (see muonh_check_wait_timeout);
+    returns its status: 5 (MUONH_ERR_TIMEOUT) when the wait gave up as designed."""
+    return int(library().muonh_check_wait_timeout(float(seconds), _stream_handle(stream)))
 
 
 def _flat_view(t, what: str, dtypes):

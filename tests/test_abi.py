@@ -105,3 +105,9 @@ def test_auxiliary_argument_checks_without_a_gpu():
     x = ctypes.c_void_p(0x5000)
     assert lib.muonh_momentum_norm_noalloc(0x1000, 0x2000, 0, 8, 8, 0.95, 1, x, None) == 1   # empty
     assert lib.muonh_momentum_norm_noalloc(0x1008, 0x2000, 4, 8, 8, 0.95, 1, x, None) == 2  # misaligned
+
+
+def test_wait_probe_argument_check_without_a_gpu():
+    lib = P.library()
+    assert lib.muonh_check_wait_timeout(0.0, None) == 1
+    assert lib.muonh_check_wait_timeout(11.0, None) == 1

@@ -275,3 +275,20 @@ def test_error_matches_the_storage_emulation(prec, shape):
     emu = rel_fro(emulate.newton_schulz_stored(X, storage=prec), ref)
     err = rel_fro(g["O"][0][0], ref)
     assert 0.8 * emu <= err <= 1.25 * emu, (err, emu)
+
+
+def test_bounded_wait_gives_up_and_the_gpu_stays_usable():
+    """Failure path without a fault: a wait that can never complete gives up
+    after its limit and reports MUONH_ERR_TIMEOUT; the GPU then runs a
+    normal step that matches the oracle."""
+    import time
+    from pretraining_optimizer_b200 import check_wait_timeout
+    t0 = time.perf_counter()
+    st = check_wait_timeout(0.3)
+    dt = time.perf_counter() - t0
+    assert st == 5, st
+    assert 0.25 <= dt <= 5.0, dt
+    wl, W0 = _single()
+    g = run_gpu(W0, wl.grad, wl.lrs[:1], keep_updates=(0,))
+    o = run_oracle(W0, wl.grad, wl.lrs[:1], keep_updates=(0,))
+    assert rel_fro(g["O"][0][0], o["O"][0][0]) <= FP16_NS_TOL
