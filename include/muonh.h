@@ -33,6 +33,10 @@
  *   - Conditions found on the device (non-finite input, zero update, a
  *     bounded wait that gave up) never abort a step: they set per-matrix
  *     flags in muonh_stats and are reported by muonh_device_status().
+ *   - A context is not thread-safe: calls on one context must not overlap
+ *     in time.  Distinct contexts are independent.  The context-free
+ *     functions (averaging, AdamW, the diagnostics) are reentrant, except
+ *     muonh_momentum_norm_noalloc (one shared scratch array, see there).
  */
 #ifndef MUONH_H_
 #define MUONH_H_
