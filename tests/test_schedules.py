@@ -57,3 +57,23 @@ def test_wsd_matches_the_workload_schedule():
     import synth
     lrs = [S.wsd_lr(k, 20, 0.012, 2, 8 / 20) for k in range(20)]
     assert lrs == pytest.approx(synth.wsd_lr())
+
+
+def test_production_schedule_is_continuous_and_decaying():
+    """Eq. (10) hands over to Eq. (11) at the Phase-1 endpoint with no jump
+    beyond the report's rounding of eta0 (1.04e-3), both decay afterwards,
+    and the CMA continuation holds its constant."""
+    k1 = S.PHASE1_TOKENS / S.TOKENS_PER_STEP
+    before = S.production_base_lr(int(k1), cma_from=None)
+    after = S.production_base_lr(int(k1) + 1, cma_from=None)
+    assert abs(after - before) <= 0.005 * before
+    ks = list(range(1001, 300000, 997))
+    lrs = [S.production_base_lr(k, cma_from=None) for k in ks]
+    assert all(b <= a + 1e-15 for a, b in zip(lrs, lrs[1:]))
+    assert all(S.production_base_lr(k) == S.CMA_BASE_LR for k in (218000, 250000, 400000))
+
+
+def test_hyperball_lr_scales_the_base_lr():
+    """Sec. 3.3.1: the Hyperball LR is m times the base LR (m = 10 in production)."""
+    assert S.hyperball_lr(1e-3) == pytest.approx(1e-2)
+    assert S.hyperball_lr(1e-3, m=2) == pytest.approx(2e-3)
