@@ -25,6 +25,19 @@ MUTATIONS = {
     "Eq. (3) without weight decay": ("W_new = (1.0 - weight_decay * eta) * W - eta * u", "W_new = W - eta * u"),
 }
 
+# mistakes in the auxiliary oracles: (file, pin tests, old, new)
+AUX_MUTATIONS = {
+    "AdamW without bias correction": ("aux.py", "tests/test_oracle_aux.py",
+                                      "m_hat = m / (1.0 - beta1 ** t)", "m_hat = m"),
+    "AdamW without weight decay": ("aux.py", "tests/test_oracle_aux.py",
+                                   "p = np.asarray(p, dtype=dtype) * (1.0 - lr * weight_decay)",
+                                   "p = np.asarray(p, dtype=dtype)"),
+    "average over k - 1": ("aux.py", "tests/test_oracle_aux.py",
+                           "return acc / len(thetas)", "return acc / max(1, len(thetas) - 1)"),
+    "bf16 rounding by truncation": ("emulate.py", "tests/test_oracle.py",
+                                    "u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000", "u = u & 0xFFFF0000"),
+}
+
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_planted_mistake(name, tmp_path):
@@ -39,3 +52,32 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "tests/test_oracle.py", "-m", "not gpu",
                         "-p", "no:cacheprovider"], cwd=tmp_path, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0, f"pins did not catch: {name}"
+
+
+@pytest.mark.parametrize("name", sorted(AUX_MUTATIONS))
+def test_aux_pins_catch_planted_mistake(name, tmp_path):
+    fname, tests, old, new = AUX_MUTATIONS[name]
+    for d in ("oracle", "synth", "tests", "pretraining_optimizer_b200"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__", "*.so", "csrc"))
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), tmp_path / "pytest.ini")
+    src = tmp_path / "oracle" / fname
+    text = src.read_text()
+    assert old in text, "the oracle changed: update this mutation"
+    src.write_text(text.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", tests, "-m", "not gpu",
+                        "-p", "no:cacheprovider"], cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, f"pins did not catch: {name}"
+
+
+@pytest.mark.parametrize("tests", ["tests/test_oracle.py", "tests/test_oracle_aux.py"])
+def test_harness_passes_without_a_mistake(tests, tmp_path):
+    """Control: the copied tree passes its pins when nothing is planted, so a
+    failure above comes from the planted mistake, not from the copy."""
+    for d in ("oracle", "synth", "tests", "pretraining_optimizer_b200"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__", "*.so", "csrc"))
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), tmp_path / "pytest.ini")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", tests, "-m", "not gpu",
+                        "-p", "no:cacheprovider"], cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout[-2000:]
