@@ -59,3 +59,6 @@ def test_reference_arm_under_two_ranks_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "steps/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    # the same workload description the CUDA arm reports at this world size
+    assert d["config"]["workload"] == "single_256x512" and d["config"]["matrices"] == 1
+    assert d["config"]["parallelism"] == "2 independent replica(s)"
