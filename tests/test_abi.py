@@ -111,3 +111,25 @@ def test_wait_probe_argument_check_without_a_gpu():
     lib = P.library()
     assert lib.muonh_check_wait_timeout(0.0, None) == 1
     assert lib.muonh_check_wait_timeout(11.0, None) == 1
+
+
+def test_binding_rejects_cpu_tensors():
+    """No CPU fallback: host tensors are refused before anything runs."""
+    import torch
+    from pretraining_optimizer_b200 import MuonH, adamw_step, average
+    w = torch.zeros(8, 16)
+    with pytest.raises(TypeError):
+        MuonH([w])
+    with pytest.raises(TypeError):
+        average([w.flatten(), w.flatten()])
+    with pytest.raises(TypeError):
+        adamw_step([w], [w.clone()], [w.clone()], [w.clone()], 1, 1e-3)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """Without libmuonh.so the binding raises instead of falling back."""
+    from pretraining_optimizer_b200 import muonh as M
+    monkeypatch.setattr(M, "_LIB", None)
+    monkeypatch.setattr(M, "library_path", lambda: str(tmp_path / "libmuonh.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        M.library()
