@@ -229,3 +229,22 @@ def test_storage_error_of_each_operand_format(storage, lo, hi):
     O = emulate.newton_schulz_stored(X, storage=storage)
     err = np.linalg.norm(O - ref) / np.linalg.norm(ref)
     assert lo <= err <= hi, err
+
+
+def test_newton_schulz_is_orthogonally_equivariant():
+    """NS(U X V^T) = U NS(X) V^T for orthogonal U, V: the iteration acts on
+    singular values only (a max-norm or element-wise scaling would break this)."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((24, 40))
+    U, _ = np.linalg.qr(rng.standard_normal((24, 24)))
+    V, _ = np.linalg.qr(rng.standard_normal((40, 40)))
+    lhs = oracle.newton_schulz(U @ X @ V.T)
+    rhs = U @ oracle.newton_schulz(X) @ V.T
+    assert np.allclose(lhs, rhs, rtol=0, atol=1e-12)
+
+
+def test_newton_schulz_ignores_the_input_scale():
+    """The input is Frobenius-normalised first, so a positive scale of X
+    changes nothing beyond the eps guard."""
+    X = _rand((32, 48), seed=4)
+    assert np.allclose(oracle.newton_schulz(3.7 * X, eps=0.0), oracle.newton_schulz(X, eps=0.0), rtol=0, atol=1e-12)
