@@ -2,7 +2,8 @@
 """MuonH optimizer-step benchmark on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qwen3_1.7b|qwen3_0.6b|single_256x512] [--ns-precision fp16|bf16|fp32]
+                    [--workload qwen3_1.7b|qwen3_0.6b|single_256x512|sweep_<rows>x<cols>]
+                    [--ns-precision fp16|bf16|fp32]
 
 One step = one muonh_step over the whole matrix set (momentum, Newton-Schulz,
 hyperball projection of every matrix).  Inputs are synthetic (W0 ~ N(0,0.02^2),
@@ -188,6 +189,22 @@ def whole_job_rate(world: int, steps: int, max_ms: float) -> float:
 
 
 # ------------------------------------------------------------------ oracle arm
+# NS FLOPs of the oracle's timed sample: one Qwen3-1.7B layer (about 6 s of
+# fp64 NumPy on 16 host cores); a set of larger matrices samples fewer.
+CPU_SAMPLE_FLOPS = 2.5e12
+
+
+def cpu_sample(shapes, ns_steps):
+    """Indices of the leading matrices of the set (at most 7, one Qwen3 layer)
+    whose Newton-Schulz work stays within CPU_SAMPLE_FLOPS; at least one."""
+    idx = [0]
+    for i in range(1, min(7, len(shapes))):
+        if ns_flops(shapes[:i + 1], ns_steps) > CPU_SAMPLE_FLOPS:
+            break
+        idx.append(i)
+    return idx
+
+
 def oracle_sample_rate(shapes, wl, sample_idx, steps=1):
     """Time the oracle (as it stands, fp64) on a sample of the set for `steps`
     steps; return (steps/s scaled to the whole set, seconds, sample FLOPs share)."""
@@ -467,14 +484,14 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_aux and args.workload == "qwen3_1.7b":
         aux = measure_aux(dev, stream, peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), elems)
 
-    # ---------------- CPU baseline: the oracle on layer 0, rank 0, N = 1
+    # ---------------- CPU baseline: the oracle on the leading matrices, rank 0, N = 1
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sample = list(range(min(7, n)))
+        sample = cpu_sample(shapes, wl.ns_steps)
         rate, dt, share = oracle_sample_rate(shapes, wl, sample)
         cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"layer 0 ({len(sample)} of {n} matrices, {share:.4f} of the NS FLOPs), one fp64 step "
-                         f"({dt:.1f} s), scaled to the whole set"}
+               "sample": f"the leading {len(sample)} of {n} matrices ({share:.4f} of the NS FLOPs; layer 0 of a "
+                         f"Qwen3 set), one fp64 step ({dt:.1f} s), scaled to the whole set"}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -203,7 +203,9 @@ class Workload:
 
 
 def workload(name: str) -> Workload:
-    """Named workloads; "<set>:L" keeps the first L layers of a Qwen3 set."""
+    """Named workloads; "<set>:L" keeps the first L layers of a Qwen3 set;
+    "sweep_<rows>x<cols>" is one shape of the roofline sweep, batched to at
+    least 1 GiB of fp32 weights, at a constant lr of 0.01."""
     if ":" in name:
         base, layers = name.split(":")
         wl = workload(base)
@@ -218,4 +220,18 @@ def workload(name: str) -> Workload:
         return Workload(name, qwen3_1p7b(), linear_decay_lr(50))
     if name == "qwen3_1.7b_illcond":
         return Workload(name, qwen3_1p7b(), linear_decay_lr(100), gradient="ill_conditioned")
+    if name.startswith("sweep_"):
+        rows, cols = parse_sweep_name(name)
+        return Workload(name, sweep_set(rows, cols, sweep_batch_size(rows, cols)), constant_lr(10, 0.01))
     raise KeyError(name)
+
+
+def parse_sweep_name(name: str) -> tuple[int, int]:
+    """"sweep_<rows>x<cols>" -> (rows, cols), for a shape of SWEEP_SHAPES."""
+    try:
+        rows, cols = (int(v) for v in name[len("sweep_"):].split("x"))
+    except ValueError:
+        raise KeyError(name) from None
+    if (rows, cols) not in SWEEP_SHAPES:
+        raise KeyError(name)
+    return rows, cols
