@@ -47,6 +47,18 @@ def round_bf16(x):
 ROUND = {"fp16": round_fp16, "bf16": round_bf16, "fp64": lambda x: np.asarray(x, dtype=np.float64)}
 
 
+def mirror_upper_tiles(P, tile=256):
+    """A symmetric product as a kernel that computes only the tiles on and
+    above the diagonal stores it: every block below the diagonal is the
+    transpose of its mirror block."""
+    out = np.array(P, dtype=np.float64, copy=True)
+    n = out.shape[0]
+    for i in range(0, n, tile):
+        for j in range(0, i, tile):
+            out[i:i + tile, j:j + tile] = out[j:j + tile, i:i + tile].T
+    return out
+
+
 def newton_schulz_stored(X, steps=5, coeffs=QUINTIC, eps=1e-7, storage="fp16"):
     """Newton-Schulz with every stored operand rounded to `storage`
     ("fp16", "bf16" or "fp64" = no rounding).  Returns O as fp64."""
@@ -61,4 +73,43 @@ def newton_schulz_stored(X, steps=5, coeffs=QUINTIC, eps=1e-7, storage="fp16"):
         A = r(Y @ Y.T)
         Bp = r(a * eye + b * A + c * (A @ A))
         Y = r(Bp @ Y)
+    return Y.T.copy() if tall else Y
+
+
+def newton_schulz_gram_stored(X, groups=(3, 2), coeffs=QUINTIC, eps=1e-7, storage="fp16", tile=256):
+    """The same quintic iteration restated in Gram space, with restarts.
+
+    With A_k = Y_k Y_k^T and p(A) = a I + b A + c A A, one iteration is
+    Y_{k+1} = p(A_k) Y_k, so A_{k+1} = p(A_k) A_k p(A_k) = A_k p(A_k)^2 (the
+    factors are polynomials in one symmetric matrix and commute), and g
+    iterations in a row apply Q = p(A_{k+g-1}) ... p(A_k) to Y_k once.  Each
+    entry of `groups` is such a run of iterations, entered from a fresh Gram
+    matrix of the current Y (a restart) and left through Y <- r(Q Y); the
+    entries sum to the step count.  groups = (1,)*steps is the Y-space form
+    of newton_schulz_stored.  In exact arithmetic every grouping gives the
+    same O; they differ only in where the 16-bit storage rounds (r(), as in
+    newton_schulz_stored), and every r x r product here is symmetric, so it
+    is stored through mirror_upper_tiles.  Returns O as fp64."""
+    r = ROUND[storage]
+    a, b, c = coeffs
+    if any(g < 1 for g in groups):
+        raise ValueError("groups must be positive run lengths")
+    X = np.asarray(X, dtype=np.float64)
+    tall = X.shape[0] > X.shape[1]
+    Y = X.T if tall else X
+    Y = r(Y / (np.linalg.norm(Y) + eps))
+    eye = np.eye(Y.shape[0])
+
+    def sym(P):
+        return r(mirror_upper_tiles(P, tile))
+
+    for g in groups:
+        A = sym(Y @ Y.T)
+        Q = None
+        for j in range(g):
+            Bp = sym(a * eye + b * A + c * (A @ A))
+            Q = Bp if Q is None else sym(Bp @ Q)
+            if j + 1 < g:
+                A = sym(sym(A @ Bp) @ Bp)
+        Y = r(Q @ Y)
     return Y.T.copy() if tall else Y

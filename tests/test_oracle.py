@@ -248,3 +248,40 @@ def test_newton_schulz_ignores_the_input_scale():
     changes nothing beyond the eps guard."""
     X = _rand((32, 48), seed=4)
     assert np.allclose(oracle.newton_schulz(3.7 * X, eps=0.0), oracle.newton_schulz(X, eps=0.0), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("groups", [(5,), (3, 2), (2, 2, 1), (1, 4)])
+def test_gram_space_form_without_rounding_is_the_oracle(groups):
+    """A_{k+1} = A_k p(A_k)^2 and one Q = prod p(A_k) per run of iterations
+    reproduce the Y-space iteration exactly (up to fp64 rounding)."""
+    from oracle import emulate
+    for X in (_rand((256, 512), seed=5), _rand((640, 384), seed=6),
+              synth.ill_conditioned_gradient(1, 0, 256, 512).astype(np.float64)):
+        O = emulate.newton_schulz_gram_stored(X, groups, storage="fp64")
+        assert np.linalg.norm(O - oracle.newton_schulz(X)) <= 1e-10 * np.linalg.norm(O)
+
+
+@pytest.mark.parametrize("storage", ["fp16", "bf16"])
+def test_gram_space_form_with_unit_runs_is_the_y_space_emulation(storage):
+    from oracle import emulate
+    X = _rand((256, 512), seed=7)
+    assert np.array_equal(emulate.newton_schulz_gram_stored(X, (1,) * 5, storage=storage),
+                          emulate.newton_schulz_stored(X, storage=storage))
+
+
+def test_gram_space_form_needs_restarts_in_fp16():
+    """Stored in fp16, runs of three and two iterations stay inside the 1e-2
+    bar and within 2x of the Y-space form's storage error, while one run of
+    five loses an ill-conditioned input: Q's entries span up to a^5
+    (p(0) = a) and fp16 keeps 11 bits of them."""
+    from oracle import emulate
+    gauss = synth.gaussian_gradient(0, 0, 256, 512).astype(np.float64)
+    ill = synth.ill_conditioned_gradient(1, 0, 256, 512).astype(np.float64)
+    for X in (gauss, ill):
+        ref = oracle.newton_schulz(X)
+        err = np.linalg.norm(emulate.newton_schulz_gram_stored(X, (3, 2)) - ref) / np.linalg.norm(ref)
+        err_y = np.linalg.norm(emulate.newton_schulz_stored(X) - ref) / np.linalg.norm(ref)
+        assert err <= 1e-2 and err <= 2 * err_y
+    ref = oracle.newton_schulz(ill)
+    err5 = np.linalg.norm(emulate.newton_schulz_gram_stored(ill, (5,)) - ref) / np.linalg.norm(ref)
+    assert err5 > 1e-1

@@ -36,6 +36,13 @@ AUX_MUTATIONS = {
                            "return acc / len(thetas)", "return acc / max(1, len(thetas) - 1)"),
     "bf16 rounding by truncation": ("emulate.py", "tests/test_oracle.py",
                                     "u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000", "u = u & 0xFFFF0000"),
+    "Gram update with one factor of p(A)": ("emulate.py", "tests/test_oracle.py",
+                                            "A = sym(sym(A @ Bp) @ Bp)", "A = sym(A @ Bp)"),
+    "Q kept from the last iteration only": ("emulate.py", "tests/test_oracle.py",
+                                            "Q = Bp if Q is None else sym(Bp @ Q)", "Q = Bp"),
+    "lower tiles left unwritten": ("emulate.py", "tests/test_oracle.py",
+                                   "out[i:i + tile, j:j + tile] = out[j:j + tile, i:i + tile].T",
+                                   "out[i:i + tile, j:j + tile] = 0.0"),
 }
 
 
