@@ -490,8 +490,9 @@ def run_ours(args):
         sample = cpu_sample(shapes, wl.ns_steps)
         rate, dt, share = oracle_sample_rate(shapes, wl, sample)
         cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"the leading {len(sample)} of {n} matrices ({share:.4f} of the NS FLOPs; layer 0 of a "
-                         f"Qwen3 set), one fp64 step ({dt:.1f} s), scaled to the whole set"}
+               "sample": f"the leading {len(sample)} of {n} matrices"
+                         f"{' (layer 0)' if args.workload.startswith('qwen3') else ''}, {share:.4f} of the NS "
+                         f"FLOPs, one fp64 step ({dt:.1f} s), scaled to the whole set"}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
