@@ -28,8 +28,12 @@
  *     asynchronously on it; argument checking is synchronous.
  *   - Device pointers are CUDA device (or managed) addresses on the current
  *     device.  The library never frees memory it did not allocate.
- *   - A non-OK status leaves every caller buffer untouched; the message of
- *     the last failure on the calling thread is in muonh_last_error().
+ *   - Argument errors (INVALID_ARG, ALIGNMENT, UNSUPPORTED) are found before
+ *     any work is enqueued and leave every caller buffer untouched.  After
+ *     MUONH_ERR_CUDA from a call that launches several kernels (muonh_step,
+ *     muonh_init) the caller's buffers are unspecified: kernels enqueued
+ *     before the failing launch still run.  The message of the last failure
+ *     on the calling thread is in muonh_last_error().
  *   - Conditions found on the device (non-finite input, zero update, a
  *     bounded wait that gave up) never abort a step: they set per-matrix
  *     flags in muonh_stats and are reported by muonh_device_status().
