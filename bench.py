@@ -77,6 +77,22 @@ def ns_flops(shapes, steps):
     return tot
 
 
+def ns_flops_executed(shapes, steps, prec="fp16"):
+    """Tensor-core FLOPs the Newton-Schulz kernels execute: GRAM and SQUARE
+    run the tiles of the upper block triangle (256 x 256 CTA-pair tiles, or
+    128 x 256 single-CTA tiles with three products each in FP32 mode), APPLY
+    every tile of Y, all on the 256-padded buffers."""
+    tm, mult = (128, 3) if prec == "fp32" else (256, 1)
+    tot = 0
+    for a, b in shapes:
+        r = (min(a, b) + 255) // 256 * 256
+        c = (max(a, b) + 255) // 256 * 256
+        upper = sum(1 for bi in range(r // tm) for bj in range(r // 256) if bj * 256 + 255 >= bi * tm)
+        tile = 2 * tm * 256
+        tot += steps * mult * (upper * tile * c + upper * tile * r + (r // tm) * (c // 256) * tile * r)
+    return tot
+
+
 def apply_flops(shapes):
     """One APPLY pass over the set (Y' = aY + BY for every matrix): 2 r^2 c
     per matrix.  A step makes ns_steps such passes; a large set splits each
@@ -473,6 +489,7 @@ def run_ours(args):
     ew_ms = sum(phases[k][0] for k in ELEMENTWISE) / args.steps
     summary = {
         "ns_tflops_dense": ns_flops(shapes, wl.ns_steps) / (ns_ms / 1000.0) / 1e12,
+        "ns_tflops_executed": ns_flops_executed(shapes, wl.ns_steps, args.ns_precision) / (ns_ms / 1000.0) / 1e12,
         "ns_ms_per_step": ns_ms,
         "elementwise_ms_per_step": ew_ms,
         "elementwise_gbps_algorithmic": ALGO_BYTES_PER_ELEM * elems / (ew_ms / 1000.0) / 1e9,
