@@ -14,6 +14,9 @@ MUTATIONS = {
     "dropped A^2 term": ("B = b * A + c * (A @ A)", "B = b * A"),
     "wrong sign of B Y": ("Y = a * Y + B @ Y", "Y = a * Y - B @ Y"),
     "scaled Gram": ("A = Y @ Y.T", "A = 1.0001 * (Y @ Y.T)"),
+    "transposed Gram (Y^T Y on square inputs)": ("A = Y @ Y.T", "A = Y.T @ Y if Y.shape[0] == Y.shape[1] else Y @ Y.T"),
+    "product order B Y -> Y B (square inputs)": ("Y = a * Y + B @ Y",
+                                                 "Y = a * Y + (Y @ B if Y.shape[0] == Y.shape[1] else B @ Y)"),
     "||W|| used for R": ("displacement = (lr * R / o_norm) * O", "displacement = (lr * w_norm / o_norm) * O"),
     "projection onto ||W||": ("W_new = (R / wt_norm) * W_tilde", "W_new = (R / w_norm) * W_tilde"),
     "lerp momentum": ("M_new = beta * M + G", "M_new = beta * M + (1 - beta) * G"),
