@@ -12,6 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 MUTATIONS = {
     "dropped A^2 term": ("B = b * A + c * (A @ A)", "B = b * A"),
+    "b and c swapped": ("B = b * A + c * (A @ A)", "B = c * A + b * (A @ A)"),
+    "O not normalised": ("displacement = (lr * R / o_norm) * O", "displacement = (lr * R) * O"),
     "wrong sign of B Y": ("Y = a * Y + B @ Y", "Y = a * Y - B @ Y"),
     "scaled Gram": ("A = Y @ Y.T", "A = 1.0001 * (Y @ Y.T)"),
     "transposed Gram (Y^T Y on square inputs)": ("A = Y @ Y.T", "A = Y.T @ Y if Y.shape[0] == Y.shape[1] else Y @ Y.T"),
