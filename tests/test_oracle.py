@@ -100,6 +100,40 @@ def test_hyperball_hand_solved_cases():
         assert abs(st["elr"] - elr) < 1e-15
 
 
+def test_radius_hand_solved_cases():
+    """R = ||W_0||_F (Sec. 3.3, Eq. (1)) on hand-solved matrices, two of which
+    have a spectral norm different from the Frobenius norm."""
+    rows = _golden_rows("radius_hand_solved.txt")
+    assert len(rows) == 5
+    for lhs, (R,) in rows:
+        r, c = int(lhs[0]), int(lhs[1])
+        W = np.array(lhs[2:], dtype=np.float64).reshape(r, c)
+        assert abs(oracle.radius(W) - R) <= 1e-15 * max(1.0, R), (W, oracle.radius(W), R)
+        # float32 input is read in fp64: the same R for exactly representable entries
+        assert abs(oracle.radius(W.astype(np.float32)) - R) <= 1e-15 * max(1.0, R)
+
+
+def test_run_steps_carries_momentum_and_fixes_the_radius():
+    """run_steps over three steps: the radius is ||W_0||_F of each matrix
+    (hand-known here) and the momentum buffer carries across steps,
+    M_k = sum_j beta^(k-j) G_j, with the reported input norm
+    ||G_k + beta M_k||_F at every step."""
+    beta = 0.95
+    shapes = [(4, 9), (9, 4)]
+    W0 = [np.full(shapes[0], 0.5), np.full(shapes[1], -0.25)]   # ||.||_F = 0.5*6 = 3, 0.25*6 = 1.5
+    Gs = {(t, i): _rand(shapes[i], seed=300 + 10 * t + i) * 1e-3 for t in range(3) for i in range(2)}
+    out = oracle.run_steps(W0, lambda t, i: Gs[(t, i)], [0.01, 0.02, 0.005], beta=beta)
+    assert out["R"] == [3.0, 1.5]
+    for i in range(2):
+        for k in range(3):
+            geo = sum(beta ** (k - j) * Gs[(j, i)] for j in range(k + 1))
+            x_norm = np.linalg.norm(Gs[(k, i)] + beta * geo)
+            assert abs(out["stats"][k][i]["input_norm"] - x_norm) <= 1e-13 * x_norm, (i, k)
+        geo = sum(beta ** (2 - j) * Gs[(j, i)] for j in range(3))
+        assert np.allclose(out["M"][i], geo, rtol=0, atol=1e-16)
+        assert abs(np.linalg.norm(out["W"][i]) - out["R"][i]) <= 1e-13 * out["R"][i]
+
+
 def test_hyperball_invariants():
     """||W_{t+1}|| = R and effective LR = lr (Sec. 3.3.1)."""
     rng = np.random.default_rng(5)

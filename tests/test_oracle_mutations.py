@@ -28,6 +28,12 @@ MUTATIONS = {
                    "elr = float(np.linalg.norm(displacement)) / R"),
     "Eq. (5) without the update scale": ("else lr * w_norm / u_norm", "else lr * w_norm / o_norm"),
     "Eq. (3) without weight decay": ("W_new = (1.0 - weight_decay * eta) * W - eta * u", "W_new = W - eta * u"),
+    "spectral norm for R": ("return float(np.linalg.norm(np.asarray(W0, dtype=dtype)))",
+                            "return float(np.linalg.norm(np.asarray(W0, dtype=dtype), 2))"),
+    "squared norm for R": ("return float(np.linalg.norm(np.asarray(W0, dtype=dtype)))",
+                           "return float(np.linalg.norm(np.asarray(W0, dtype=dtype)) ** 2)"),
+    "momentum reset every step in run_steps": ("W[i], M[i], O, st = muonh_step(W[i], M[i], grad_fn(t, i)",
+                                               "W[i], M[i], O, st = muonh_step(W[i], 0 * M[i], grad_fn(t, i)"),
 }
 
 # mistakes in the auxiliary oracles: (file, pin tests, old, new)
