@@ -7,14 +7,15 @@
 // A block walks elementwise tiles (4096 elements of W) in a grid-stride loop;
 // each of its 8 warps owns a fixed eighth of every tile and never waits for
 // the others: no shared memory, no block barrier.  A lane issues all of its
-// loads for a tile (8 x 16 bytes on wide tiles, 16 x 8 bytes on tall ones)
-// before the first use, so a resident warp keeps 4 KB in flight, and it
-// fetches the next tile's table entries while those loads are in flight
-// (three resident blocks per SM: 80 registers a thread).  Tall
-// matrices, whose X is the transpose, are tiled 64 x 64: warp w takes rows
-// 8w..8w+7 with two adjacent columns per lane, so a lane holds 8 consecutive
-// entries of two X rows and writes (or, in project, reads) each as one
-// 16-byte access.
+// loads for a tile (8 x 16 bytes) before the first use, so a resident warp
+// keeps 4 KB in flight, and it fetches the next tile's table entries while
+// those loads are in flight (three resident blocks per SM: 80 registers a
+// thread).  Tall matrices, whose X is the transpose, are tiled 64 x 64: warp
+// w takes a 16 x 32 block and each lane a 4 x 4 sub-block of it (four
+// consecutive rows, four columns), so a column of the sub-block is 8
+// consecutive bytes of one 16-bit X row and the four lanes sharing a column
+// write (or, in project, read) that row's whole 32-byte sector in one
+// instruction.
 //
 // Every warp writes its partial sum of a tile to a fixed slot (8 per tile);
 // the finalize kernels add the slots of a matrix in a fixed order in fp64, so
@@ -114,7 +115,7 @@ __device__ __forceinline__ TileCtx tile_ctx(const EwParams& p, int64_t e) {
   c.nr = t.nr;
   c.nc = t.nc;
   c.sh = __ffs(md.et_tw) - 3;
-  uint16_t* xg = static_cast<uint16_t*>(cd.x[PROJECT ? (md.ns_steps & 1) : 0][0]) + md.z * cd.x_stride;
+  uint16_t* xg = static_cast<uint16_t*>(cd.x[PROJECT ? md.o_buf : 0][0]) + md.z * cd.x_stride;
   c.x = TALL ? xg + t.c0 * c.xld + t.r0 : xg + t.r0 * c.xld + t.c0;
   if (PROJECT) {
     const MatScal& sc = p.scal[mi];
@@ -193,34 +194,38 @@ __global__ void __launch_bounds__(kWarpThreads, 3) momentum_warp_kernel(const Ew
       if (lane == 0) p.part8[cur.e * kWarps + w] = acc;
       cur = nxt;
     } else {
-      // tall 64 x 64: warp w takes rows 8w .. 8w+7; lane l covers columns
-      // c .. c+3 (c = 4 (l mod 16)) of the even rows (l < 16) or the odd rows
-      const int half = lane >> 4;
-      const int c = 4 * (lane & 15);
-      const bool cok = c < cur.nc;   // nc is a multiple of 4
+      // tall 64 x 64 tile, X holding its transpose: warp w takes the 16 x 32
+      // block of W rows 16 (w >> 1) .. +15 and columns 32 (w & 1) .. +31, and
+      // lane l its 4 x 4 sub-block of rows rb .. rb+3 and columns cb .. cb+3.
+      // A load instruction then covers four whole 128-byte W rows, and a
+      // column of the lane's sub-block is four consecutive entries (8 bytes)
+      // of one X row: the four lanes sharing cb write a whole 32-byte sector.
+      const int rb = 16 * (w >> 1) + 4 * (lane >> 3);
+      const int cb = 32 * (w & 1) + 4 * (lane & 7);
+      const bool cok = cb < cur.nc;   // nc is a multiple of 4
       float4 gv[4], mv[4];
 #pragma unroll
-      for (int jr = 0; jr < 4; ++jr) {
-        const int r = 8 * w + 2 * jr + half;
+      for (int j = 0; j < 4; ++j) {
+        const int r = rb + j;
         if (cok && r < cur.nr) {
-          gv[jr] = *reinterpret_cast<const float4*>(cur.a + r * cur.ld + c);
-          mv[jr] = *reinterpret_cast<const float4*>(cur.b + r * cur.ld + c);
+          gv[j] = *reinterpret_cast<const float4*>(cur.a + r * cur.ld + cb);
+          mv[j] = *reinterpret_cast<const float4*>(cur.b + r * cur.ld + cb);
         }
       }
       const TileCtx nxt = tile_ctx<TALL, false>(p, next_tile<TALL>(p, cur.e + gridDim.x));
-      float x[4][4];
+      float x[4][4];   // [row j][column q], scaled by sigma
 #pragma unroll
-      for (int jr = 0; jr < 4; ++jr) {
-        const int r = 8 * w + 2 * jr + half;
-        x[jr][0] = x[jr][1] = x[jr][2] = x[jr][3] = 0.f;   // rows past the matrix stay zero in X's padding
+      for (int j = 0; j < 4; ++j) {
+        const int r = rb + j;
+        x[j][0] = x[j][1] = x[j][2] = x[j][3] = 0.f;   // rows past the matrix stay zero in X's padding
         if (!cok || r >= cur.nr) continue;
-        float4 m = mv[jr];
-        const float4 g = gv[jr];
+        float4 m = mv[j];
+        const float4 g = gv[j];
         m.x = fmaf(beta, m.x, g.x);
         m.y = fmaf(beta, m.y, g.y);
         m.z = fmaf(beta, m.z, g.z);
         m.w = fmaf(beta, m.w, g.w);
-        *reinterpret_cast<float4*>(cur.b + r * cur.ld + c) = m;
+        *reinterpret_cast<float4*>(cur.b + r * cur.ld + cb) = m;
         float4 xv = m;
         if (cur.flag) {
           xv.x = fmaf(beta, m.x, g.x);
@@ -229,31 +234,16 @@ __global__ void __launch_bounds__(kWarpThreads, 3) momentum_warp_kernel(const Ew
           xv.w = fmaf(beta, m.w, g.w);
         }
         acc = fmaf(xv.x, xv.x, fmaf(xv.y, xv.y, fmaf(xv.z, xv.z, fmaf(xv.w, xv.w, acc))));
-        x[jr][0] = xv.x * sigma;
-        x[jr][1] = xv.y * sigma;
-        x[jr][2] = xv.z * sigma;
-        x[jr][3] = xv.w * sigma;
+        x[j][0] = xv.x * sigma;
+        x[j][1] = xv.y * sigma;
+        x[j][2] = xv.z * sigma;
+        x[j][3] = xv.w * sigma;
       }
-      // X row c + k holds rows 8w .. 8w+7 of column k: the even-row lane
-      // writes columns c, c+1 and the odd-row lane (lane ^ 16) columns c+2,
-      // c+3, each taking the other's half of the rows by one exchange
-      float y[4][2];
-#pragma unroll
-      for (int jr = 0; jr < 4; ++jr)
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-          y[jr][k] = __shfl_xor_sync(0xffffffffu, half ? x[jr][k] : x[jr][2 + k], 16);
       if (sigma > 0.f && cok) {
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int kc = 2 * half + k;   // column of this X row inside the lane's four
-          uint32_t h[4];
-#pragma unroll
-          for (int jr = 0; jr < 4; ++jr) {   // rows 8w + 2jr (even) and 8w + 2jr + 1 (odd)
-            const float own = half ? x[jr][2 + k] : x[jr][k];
-            h[jr] = half ? pack2(y[jr][k], own, p.prec) : pack2(own, y[jr][k], p.prec);
-          }
-          *reinterpret_cast<uint4*>(cur.x + (c + kc) * cur.xld + 8 * w) = make_uint4(h[0], h[1], h[2], h[3]);
+        for (int q = 0; q < 4; ++q) {   // X row cb + q, entries rb .. rb+3
+          const uint2 u = make_uint2(pack2(x[0][q], x[1][q], p.prec), pack2(x[2][q], x[3][q], p.prec));
+          *reinterpret_cast<uint2*>(cur.x + (cb + q) * cur.xld + rb) = u;
         }
       }
       acc = warp_sum(acc);
@@ -310,35 +300,40 @@ __global__ void __launch_bounds__(kWarpThreads, 3) project_warp_kernel(const EwP
       if (lane == 0) p.part8[cur.e * kWarps + w] = acc;
       cur = nxt;
     } else {
-      const int c = 2 * lane;
-      const bool cok = c < cur.nc;
-      float2 wv[8];
-      uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
-      if (cok && mode == 0) {
-        // O(8w + i, c) = X[c0 + c][r0 + 8w + i]: 8 consecutive entries of two X rows
-        const uint16_t* src = cur.x + c * cur.xld + 8 * w;
-        o0 = *reinterpret_cast<const uint4*>(src);
-        o1 = *reinterpret_cast<const uint4*>(src + cur.xld);
+      // tall 64 x 64 tile: the block of each warp and lane of the momentum
+      // kernel; the lane reads O as four 8-byte pieces of X rows cb .. cb+3
+      const int rb = 16 * (w >> 1) + 4 * (lane >> 3);
+      const int cb = 32 * (w & 1) + 4 * (lane & 7);
+      const bool cok = cb < cur.nc;
+      float4 wv[4];
+      uint2 ov[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        ov[q] = make_uint2(0u, 0u);
+        // O(rb + j, cb + q) = X[c0 + cb + q][r0 + rb + j]; X's padding columns are zero
+        if (cok && mode == 0) ov[q] = *reinterpret_cast<const uint2*>(cur.x + (cb + q) * cur.xld + rb);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * w + i;
-        if (cok && r < cur.nr) wv[i] = *reinterpret_cast<const float2*>(cur.a + r * cur.ld + c);
+      for (int j = 0; j < 4; ++j) {
+        const int r = rb + j;
+        if (cok && r < cur.nr) wv[j] = *reinterpret_cast<const float4*>(cur.a + r * cur.ld + cb);
       }
       const TileCtx nxt = tile_ctx<TALL, true>(p, next_tile<TALL>(p, cur.e + gridDim.x));
-      const float4 a0 = unpack4(make_uint2(o0.x, o0.y), p.prec), a1 = unpack4(make_uint2(o0.z, o0.w), p.prec);
-      const float4 b0 = unpack4(make_uint2(o1.x, o1.y), p.prec), b1 = unpack4(make_uint2(o1.z, o1.w), p.prec);
-      const float oa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float ob[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float4 o0 = unpack4(ov[0], p.prec), o1 = unpack4(ov[1], p.prec);
+      const float4 o2 = unpack4(ov[2], p.prec), o3 = unpack4(ov[3], p.prec);
+      const float oc[4][4] = {{o0.x, o1.x, o2.x, o3.x}, {o0.y, o1.y, o2.y, o3.y},
+                              {o0.z, o1.z, o2.z, o3.z}, {o0.w, o1.w, o2.w, o3.w}};   // [row j][column q]
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * w + i;
+      for (int j = 0; j < 4; ++j) {
+        const int r = rb + j;
         if (!cok || r >= cur.nr) continue;
-        float2 v = wv[i];
-        v.x = fmaf(ko, oa[i], kw * v.x);
-        v.y = fmaf(ko, ob[i], kw * v.y);
-        *reinterpret_cast<float2*>(cur.b + r * cur.ld + c) = v;
-        acc = fmaf(v.x, v.x, fmaf(v.y, v.y, acc));
+        float4 v = wv[j];
+        v.x = fmaf(ko, oc[j][0], kw * v.x);
+        v.y = fmaf(ko, oc[j][1], kw * v.y);
+        v.z = fmaf(ko, oc[j][2], kw * v.z);
+        v.w = fmaf(ko, oc[j][3], kw * v.w);
+        *reinterpret_cast<float4*>(cur.b + r * cur.ld + cb) = v;
+        acc = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, acc))));
       }
       acc = warp_sum(acc);
       if (lane == 0) p.part8[cur.e * kWarps + w] = acc;
