@@ -25,7 +25,10 @@ static __device__ __align__(256) float g_noalloc_partials[kNoAllocMaxTiles];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
+// Per device ordinal, looked up once in the primary context: the scratch
+// array's device address and the SM count that sizes the grid.
 float* g_partials_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
 
 struct OneMatrix {
   float* m;
@@ -174,19 +177,23 @@ extern "C" muonh_status muonh_momentum_norm_noalloc(float* m, const float* g, in
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return na_fail(MUONH_ERR_CUDA, "cudaGetDevice failed");
   float* partials = nullptr;
+  int sms = 0;
   {
     std::lock_guard<std::mutex> lock(g_setup_mutex);
     if (!g_partials_ptr[dev]) {
       void* ptr = nullptr;
       if (cudaGetSymbolAddress(&ptr, g_noalloc_partials) != cudaSuccess || !ptr)
         return na_fail(MUONH_ERR_CUDA, "cudaGetSymbolAddress of the scratch array failed");
+      int count = 0;
+      if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || count <= 0)
+        return na_fail(MUONH_ERR_CUDA, "cudaDeviceGetAttribute(multiProcessorCount) failed");
+      g_sm_count[dev] = count;
       g_partials_ptr[dev] = static_cast<float*>(ptr);
     }
     partials = g_partials_ptr[dev];
+    sms = g_sm_count[dev];
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = std::min<int64_t>(a.tiles, static_cast<int64_t>(sms) * 8);
   momentum_norm_noalloc_kernel<<<static_cast<int>(grid), kEwThreads, 0, s>>>(a, partials);
   if (cudaGetLastError() != cudaSuccess) return na_fail(MUONH_ERR_CUDA, "launch of momentum_norm_noalloc failed");
