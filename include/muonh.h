@@ -113,9 +113,37 @@ typedef struct {
   float update_scale;     /* u = update_scale * O for the ordinary rules     */
 } muonh_matrix_desc;
 
+/* Context-wide settings.
+ *   groups  0: automatic.  A set of at least 16M elements on the 16-bit path
+ *              then runs as two matrix groups, whose elementwise kernels
+ *              overlap the other group's Newton-Schulz GEMMs on an internal
+ *              stream.
+ *           1: one group.  Every kernel runs on the caller's stream, one
+ *              after another; the context creates no stream of its own.
+ *           Other values are rejected (MUONH_ERR_INVALID_ARG).  The results
+ *           are the same bit for bit either way.
+ *   ns_form  how the Newton-Schulz iteration is evaluated (MUONH_NS_FORM_*).
+ *           Y-space: every iteration forms A = Y Y^T, B' = a I + b A + c A A
+ *           and Y <- B' Y (three products, two of them over the r x c Y).
+ *           Gram-space: runs of up to three iterations are carried on r x r
+ *           matrices, A_{k+1} = A_k p(A_k)^2 with p(A) = a I + b A + c A A,
+ *           and each run ends with one Y <- Q Y, Q the product of the run's
+ *           p(A_k) (fewer FLOPs where c >= 3r; a restart every three
+ *           iterations keeps fp16 storage accurate).  In exact arithmetic
+ *           both give the same O; their fp16 rounding differs.  The Gram
+ *           form needs FP16 operands and ns_steps equal to the largest
+ *           ns_steps of the context; other matrices use the Y-space form.
+ *           Values outside MUONH_NS_FORM_* are rejected. */
+enum {
+  MUONH_NS_FORM_AUTO = 0,    /* Gram form for classes with r >= 2048, c >= 3r  */
+  MUONH_NS_FORM_Y = 1,       /* Y-space form for every matrix                   */
+  MUONH_NS_FORM_GRAM = 2     /* Gram form for every matrix that can take it     */
+};
 typedef struct {
   int32_t ns_precision;   /* MUONH_NS_FP16 / _BF16 / _FP32                  */
   float eps;              /* Newton-Schulz input: X/(||X||_F + eps), >= 0    */
+  int32_t groups;         /* 0 = automatic, 1 = a single group              */
+  int32_t ns_form;        /* MUONH_NS_FORM_*                                */
 } muonh_config;
 
 /* Per-matrix result of one step (24 bytes, plain fp32 + uint32). */
@@ -191,7 +219,8 @@ enum {
   MUONH_PHASE_FINALIZE_UPDATE = 7, /* Eq. (1) scalars per matrix            */
   MUONH_PHASE_PROJECT = 8,         /* W <- R (W - lr R u^)/||.||            */
   MUONH_PHASE_FINALIZE_STEP = 9,   /* ||W_t+1||, stats                      */
-  MUONH_NUM_PHASES = 10
+  MUONH_PHASE_NS_PRODUCT = 10,     /* Gram form: products of r x r factors  */
+  MUONH_NUM_PHASES = 11
 };
 
 /* With enable != 0, every following muonh_step brackets each kernel with a
@@ -204,6 +233,13 @@ muonh_status muonh_enable_timing(muonh_ctx* ctx, int32_t enable);
  * (launches_out[MUONH_NUM_PHASES], may be NULL) since the previous call;
  * then clears the record. */
 muonh_status muonh_phase_times(muonh_ctx* ctx, float* ms_out, int64_t* launches_out);
+
+/* Tensor-core FLOPs that the Newton-Schulz launches of the last muonh_step
+ * executed, per phase (flops_out[MUONH_NUM_PHASES]; 0 for the elementwise
+ * phases): for each launch, its tiles' 2 M N K on the padded buffers, three
+ * products per tile in FP32 mode.  Symmetric products count only the tiles
+ * they compute (those that touch the upper block triangle). */
+muonh_status muonh_phase_flops(const muonh_ctx* ctx, double* flops_out);
 
 /* Allocation-free momentum stage for one matrix (the report has no
  * counterpart; this is a deployment convenience).  Computes, like the first
@@ -220,7 +256,11 @@ muonh_status muonh_phase_times(muonh_ctx* ctx, float* ms_out, int64_t* launches_
  *   limit  at most 65,536 tiles (268,435,456 elements); a larger matrix
  *          returns MUONH_ERR_UNSUPPORTED and touches nothing.
  * The first call on a device looks up the scratch array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * (cudaGetSymbolAddress) and the SM count, and keeps both for that device
+ * ordinal; make that first call before any stream capture.  The address is
+ * the one in the device's primary context (the CUDA runtime's default, which
+ * PyTorch uses): call it only with the primary context current, and not
+ * after cudaDeviceReset, which invalidates the kept address.
  * All calls share the one scratch array, so calls whose kernels overlap on
  * the GPU (different streams without ordering) race; calls on one stream are
  * ordered and safe.  Enqueued on `stream`. */

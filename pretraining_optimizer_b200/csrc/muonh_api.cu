@@ -71,10 +71,22 @@ constexpr uint32_t kStateMagic = 0x484E554Du;   // "MUNH"
 struct TileList {
   TileDesc* dev = nullptr;
   int32_t count = 0;
+  int64_t sum_nk = 0, sum_nk_sq = 0;   // k-blocks over the tiles, as GRAM/APPLY and as SQUARE
 };
+
+// Run lengths of the Gram-space form for `steps` iterations: as few runs of
+// at most three as possible, longer runs first (5 -> 3, 2).
+std::vector<int> gram_runs(int steps) {
+  std::vector<int> runs;
+  if (steps <= 0) return runs;
+  const int nruns = (steps + 2) / 3;
+  for (int j = 0; j < nruns; ++j) runs.push_back(steps / nruns + (j < steps % nruns ? 1 : 0));
+  return runs;
+}
 
 struct ClassHost {
   int32_t r_pad, c_pad, count = 0;
+  bool gram = false;         // holds a matrix in the Gram-space form (P1, T buffers)
   ClassDev dev{};
 };
 
@@ -138,6 +150,45 @@ void scale_exponents(float a, float b, float c, int steps, int prec, int32_t* ex
   *eb = safe_exponent(std::max(bmax, 1e-30));
 }
 
+// Scale of a stored product Q of `run` consecutive factors p(A_k) = a I +
+// b A_k + c A_k^2 (Gram-space form).  On a singular direction of the run's
+// first Y with value s, Q acts as prod_k q(s_k), q(s) = a + b s^2 + c s^4 and
+// s_{k+1} = s_k q(s_k); |Q| is bounded by the largest such product over s in
+// [0, smax], smax the bound on every iterate's singular values (at s = 0 it
+// is a^run).  The products A_k p(A_k) are bounded like A (they act as
+// s_k s_{k+1}) and share A's scale.
+int q_exponent(float a, float b, float c, int run, double smax) {
+  double qmax = 0.0;
+  const int n = 8192;
+  for (int i = 0; i <= n; ++i) {
+    double s = smax * i / n, q = 1.0;
+    for (int k = 0; k < run; ++k) {
+      const double f = a + b * s * s + c * s * s * s * s;
+      q *= f;
+      s *= f;
+    }
+    qmax = std::max(qmax, std::fabs(q));
+  }
+  return safe_exponent(std::max(qmax * 1.02, 1e-30));
+}
+
+// Bound on the singular values of every iterate (the s_all of scale_exponents).
+double iterate_bound(float a, float b, float c, int steps) {
+  double smax = 1.0, s_all = 1.0;
+  for (int k = 0; k < steps; ++k) {
+    double m = 0.0;
+    const int n = 8192;
+    for (int i = 0; i <= n; ++i) {
+      const double s = smax * i / n;
+      m = std::max(m, std::fabs(a * s + b * s * s * s + c * s * s * s * s * s));
+    }
+    smax = std::max(m * 1.001, 1e-30);
+    s_all = std::max(s_all, smax);
+    if (!std::isfinite(s_all) || s_all > 1e6) break;
+  }
+  return s_all * 1.02;
+}
+
 int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 }  // namespace
@@ -152,6 +203,8 @@ struct muonh_ctx {
   int sm_count = 148;
   int32_t max_steps = 0;
   bool pairs = false;        // 16-bit operands: CTA-pair GEMMs on 256 x 256 tiles
+  std::vector<int> runs;     // Gram-space form: iterations per run
+  double step_flops[MUONH_NUM_PHASES] = {};   // tensor-core FLOPs of the last step's launches
   int64_t n_et = 0;
   int64_t step_count = 0;
   int32_t last_launches = 0;
@@ -166,7 +219,9 @@ struct muonh_ctx {
     int32_t m_first = 0, m_count = 0;
     int64_t e_first = 0, e_end = 0;
     bool any_unfused = false, any_general = false, any_wt[2] = {false, false};
-    std::vector<TileList> gram_lists, apply_lists;   // per Newton-Schulz iteration
+    std::vector<TileList> gram_lists, apply_lists;   // per Newton-Schulz iteration (Y-space form)
+    bool any_gram = false;                           // Gram-space form: its upper and APPLY tiles
+    TileList gram_upper, gram_apply;
   };
   std::vector<Group> groups;
   cudaStream_t ns_stream = nullptr;   // highest-priority stream for the GEMMs of a grouped step
@@ -357,6 +412,10 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   if (cfg->ns_precision < 0 || cfg->ns_precision > 2)
     return fail(MUONH_ERR_INVALID_ARG, "ns_precision %d is not FP16, BF16 or FP32", cfg->ns_precision);
   if (!(cfg->eps >= 0.f) || !std::isfinite(cfg->eps)) return fail(MUONH_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (cfg->groups < 0 || cfg->groups > 1)
+    return fail(MUONH_ERR_INVALID_ARG, "groups %d is not 0 (automatic) or 1 (one group)", cfg->groups);
+  if (cfg->ns_form < MUONH_NS_FORM_AUTO || cfg->ns_form > MUONH_NS_FORM_GRAM)
+    return fail(MUONH_ERR_INVALID_ARG, "ns_form %d is not MUONH_NS_FORM_AUTO, _Y or _GRAM", cfg->ns_form);
   for (int32_t i = 0; i < n; ++i) {
     const muonh_matrix_desc& d = mats[i];
     if (!d.w || !d.m) return fail(MUONH_ERR_INVALID_ARG, "matrix %d: w or m is NULL", i);
@@ -394,6 +453,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   ctx->sm_count = prop.multiProcessorCount;
   for (int k = 0; k < 4; ++k) ctx->ew_warp_grid[k] = ctx->sm_count * ew_warp_blocks_per_sm(k);
   ctx->pairs = cfg->ns_precision != P_FP32;
+  const bool single_group = cfg->groups == 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ctx->last_stream = s;
 
@@ -460,6 +520,25 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   }
   ctx->n_et = n_et;
 
+  // ---- Newton-Schulz form per matrix: the Gram-space form (fp16 CTA pairs,
+  // the context's full step count) where it saves FLOPs, r >= 2048 and
+  // c >= 3r, or wherever it can run when asked for
+  ctx->runs = gram_runs(ctx->max_steps);
+  for (int32_t i = 0; i < n; ++i) {
+    MatDev& md = ctx->mats[i];
+    ClassHost& ch = ctx->classes[md.cls];
+    const bool can = ctx->pairs && ctx->prec == P_FP16 && md.ns_steps == ctx->max_steps && md.ns_steps > 1;
+    const bool pays = ch.r_pad >= 2048 && ch.c_pad >= 3 * ch.r_pad;
+    md.gram = (can && (cfg->ns_form == MUONH_NS_FORM_GRAM || (cfg->ns_form == MUONH_NS_FORM_AUTO && pays))) ? 1 : 0;
+    md.eq = 0;
+    if (md.gram) {
+      const int longest = *std::max_element(ctx->runs.begin(), ctx->runs.end());
+      md.eq = q_exponent(md.a, md.b, md.c_coef, longest, iterate_bound(md.a, md.b, md.c_coef, md.ns_steps));
+      ch.gram = true;
+    }
+    md.o_buf = md.gram ? static_cast<int32_t>(ctx->runs.size() & 1) : (md.ns_steps & 1);
+  }
+
   // ---- fused ||O||^2, <W, O> in the last APPLY (CTA pairs, vector path,
   // matrices whose last iteration is the last launch): 2 slots per pair tile
   for (int32_t i = 0; i < n; ++i) {
@@ -483,13 +562,17 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       const MatDev& md = ctx->mats[i];
       const double r = md.r, c = md.c;
       work[i] = md.ns_steps * (4.0 * r * r * c + 2.0 * r * r * r);
+      if (md.gram) {   // per run: Y Y^T and Q Y, plus 4 g - 3 products of r x r factors
+        work[i] = 0.0;
+        for (int g : ctx->runs) work[i] += 6.0 * r * r * c + (4.0 * g - 3.0) * 2.0 * r * r * r;
+      }
       total += work[i];
       elems += md.rows * md.cols;
     }
     // group g ends after the first matrix at which the running work reaches
     // (g + 1) / kGroups of the total; every group keeps at least one matrix
     std::vector<int32_t> bounds{0};
-    if (ctx->pairs && n >= kGroups && elems >= kTwoGroupMinElems && total > 0.0) {
+    if (ctx->pairs && !single_group && n >= kGroups && elems >= kTwoGroupMinElems && total > 0.0) {
       double acc = 0.0;
       for (int32_t i = 0; i < n && static_cast<int>(bounds.size()) < kGroups; ++i) {
         acc += work[i];
@@ -511,6 +594,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
         gr.any_unfused |= !md.fused_dots;
         gr.any_general |= md.warp_tiled == 0;
         if (md.warp_tiled) gr.any_wt[md.transposed ? 1 : 0] = true;
+        gr.any_gram |= md.gram != 0;
       }
       ctx->groups.push_back(gr);
     }
@@ -548,6 +632,18 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       CUDA_TRY(cudaMemsetAsync(cd.b[part], 0, ab, s));
       if (!ctx->pairs) CUDA_TRY(cudaMemsetAsync(cd.c[part], 0, ab, s));
     }
+    if (ctx->prec == P_BF16) {   // residual of B's stored diagonal, per matrix and row
+      const size_t db = static_cast<size_t>(ch.r_pad) * ch.count * sizeof(float);
+      if (dev_alloc(ctx, reinterpret_cast<void**>(&cd.bdiag), db) != cudaSuccess)
+        return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", db);
+      CUDA_TRY(cudaMemsetAsync(cd.bdiag, 0, db, s));
+    }
+    if (ch.gram) {   // Gram-space form: the second p(A) buffer and the product buffer
+      if (dev_alloc(ctx, &cd.p1, ab) != cudaSuccess || dev_alloc(ctx, &cd.t, ab) != cudaSuccess)
+        return fail(MUONH_ERR_OOM, "workspace allocation of %zu bytes failed", ab);
+      CUDA_TRY(cudaMemsetAsync(cd.p1, 0, ab, s));
+      CUDA_TRY(cudaMemsetAsync(cd.t, 0, ab, s));
+    }
   }
 
   // ---- tensor maps: TM_PER_CLASS per class
@@ -583,6 +679,15 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           return st;
         if ((st = encode_map(&m[TM_B_ST], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
+        if (ctx->classes[ci].gram) {
+          if ((st = encode_map(&m[TM_P1_K128], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
+          if ((st = encode_map(&m[TM_T_K128], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
+          if ((st = encode_map(&m[TM_P1_ST], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, 32, 32,
+                               CU_TENSOR_MAP_SWIZZLE_64B)))
+            return st;
+          if ((st = encode_map(&m[TM_T_ST], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+            return st;
+        }
       }
     }
   }
@@ -631,19 +736,11 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   CUDA_TRY(cudaMemcpyAsync(ctx->d_scal, scal.data(), n * sizeof(MatScal), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, (1 + kGroups) * sizeof(int), s));
 
-  // ---- Newton-Schulz tile lists, per group one pair per iteration (shared when equal)
-  for (muonh_ctx::Group& gr : ctx->groups) {
-  std::vector<int32_t> prev_active;
-  for (int32_t k = 0; k < ctx->max_steps; ++k) {
-    std::vector<int32_t> active;
-    for (int32_t i = gr.m_first; i < gr.m_first + gr.m_count; ++i)
-      if (ctx->mats[i].ns_steps > k) active.push_back(i);
-    if (k > 0 && active == prev_active) {
-      gr.gram_lists.push_back(gr.gram_lists.back());
-      gr.apply_lists.push_back(gr.apply_lists.back());
-      continue;
-    }
-    prev_active = active;
+  // ---- Newton-Schulz tile lists: per group, one pair (upper-triangle tiles,
+  // APPLY tiles) per iteration of the Y-space form (shared when equal), and
+  // one pair for the matrices in the Gram-space form
+  const int tm = ctx->pairs ? 2 * kBM : kBM;   // tile rows: 128 (single CTA, FP32 mode) or 256 (CTA pairs)
+  auto make_lists = [&](const std::vector<int32_t>& active, TileList& gl, TileList& al) -> muonh_status {
     // longest tiles first (the K extent), then matrix by matrix for L2 reuse
     std::vector<int32_t> order = active;
     std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
@@ -652,8 +749,6 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       if (cx.c_pad != cy.c_pad) return cx.c_pad > cy.c_pad;
       return cx.r_pad > cy.r_pad;
     });
-    // Tile rows are 128 (single-CTA kernel, FP32 mode) or 256 (CTA pairs).
-    const int tm = ctx->pairs ? 2 * kBM : kBM;
     std::vector<TileDesc> gram, apply;
     for (int32_t i : order) {
       const ClassHost& ch = ctx->classes[ctx->mats[i].cls];
@@ -670,9 +765,13 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
         for (int bj = 0; bj < ch.c_pad / kBN; ++bj)
           apply.push_back(TileDesc{i, int16_t(bi), int16_t(bj), ch.r_pad / kBK, ch.r_pad / kBK});
     }
-    TileList gl, al;
     gl.count = static_cast<int32_t>(gram.size());
     al.count = static_cast<int32_t>(apply.size());
+    for (const TileDesc& td : gram) {
+      gl.sum_nk += td.nk;
+      gl.sum_nk_sq += td.nk_sq;
+    }
+    for (const TileDesc& td : apply) al.sum_nk += td.nk;
     if (dev_alloc(ctx, reinterpret_cast<void**>(&gl.dev), std::max<size_t>(1, gram.size()) * sizeof(TileDesc)) !=
             cudaSuccess ||
         dev_alloc(ctx, reinterpret_cast<void**>(&al.dev), std::max<size_t>(1, apply.size()) * sizeof(TileDesc)) !=
@@ -682,9 +781,33 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       CUDA_TRY(cudaMemcpyAsync(gl.dev, gram.data(), gram.size() * sizeof(TileDesc), cudaMemcpyHostToDevice, s));
     if (!apply.empty())
       CUDA_TRY(cudaMemcpyAsync(al.dev, apply.data(), apply.size() * sizeof(TileDesc), cudaMemcpyHostToDevice, s));
-    gr.gram_lists.push_back(gl);
-    gr.apply_lists.push_back(al);
-  }
+    return MUONH_OK;
+  };
+  for (muonh_ctx::Group& gr : ctx->groups) {
+    std::vector<int32_t> prev_active;
+    for (int32_t k = 0; k < ctx->max_steps; ++k) {
+      std::vector<int32_t> active;
+      for (int32_t i = gr.m_first; i < gr.m_first + gr.m_count; ++i)
+        if (ctx->mats[i].ns_steps > k && !ctx->mats[i].gram) active.push_back(i);
+      if (k > 0 && active == prev_active) {
+        gr.gram_lists.push_back(gr.gram_lists.back());
+        gr.apply_lists.push_back(gr.apply_lists.back());
+        continue;
+      }
+      prev_active = active;
+      TileList gl, al;
+      muonh_status st;
+      if ((st = make_lists(active, gl, al))) return st;
+      gr.gram_lists.push_back(gl);
+      gr.apply_lists.push_back(al);
+    }
+    if (gr.any_gram) {
+      std::vector<int32_t> active;
+      for (int32_t i = gr.m_first; i < gr.m_first + gr.m_count; ++i)
+        if (ctx->mats[i].gram) active.push_back(i);
+      muonh_status st;
+      if ((st = make_lists(active, gr.gram_upper, gr.gram_apply))) return st;
+    }
   }
 
   // ---- pinned staging ring for the per-step table
@@ -744,32 +867,47 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
     STEP_LAUNCH_ON(MUONH_PHASE_WRITE_X, launch_write_x(p, grid, st), "write_x", st);
     return MUONH_OK;
   };
+  for (double& f : ctx->step_flops) f = 0.0;
+  // tensor-core FLOPs of a launch over `sum_k` k-blocks of tiles (tile rows x 256 x 64 each)
+  const double tile_flops = 2.0 * (ctx->pairs ? 2 * kBM : kBM) * kBN * kBK * (ctx->pairs ? 1 : 3);
   auto newton_schulz = [&](int g, cudaStream_t st) -> muonh_status {
     const muonh_ctx::Group& gr = ctx->groups[g];
+    NsParams base{};
+    base.mats = ctx->d_mats;
+    base.classes = ctx->d_classes;
+    base.tmaps = ctx->d_tmaps;
+    base.err = ctx->d_err;
+    base.scal = ctx->d_scal;
+    base.wmaps = ctx->d_wmaps;
+    base.part_ns = ctx->d_part_ns;
+    const int pairs_max = std::max(1, ctx->sm_count / 2);
+    auto pair_grid = [&](int ntiles) { return std::min(pairs_max, std::max(1, ntiles)); };
+    // ---- Y-space form: A = Y Y^T, B' = a I + b A + c A A, Y <- B' Y per iteration
     for (int32_t k = 0; k < ctx->max_steps; ++k) {
-      NsParams np{};
-      np.mats = ctx->d_mats;
-      np.classes = ctx->d_classes;
-      np.tmaps = ctx->d_tmaps;
-      np.err = ctx->d_err;
+      NsParams np = base;
       np.src = k & 1;
       np.iter = k;
-      np.scal = ctx->d_scal;
-      np.wmaps = ctx->d_wmaps;
-      np.part_ns = ctx->d_part_ns;
+      np.lhs = RR_A;
+      np.rhs = RR_A;
+      np.out = RR_B;
       np.tiles = gr.gram_lists[k].dev;
       np.ntiles = gr.gram_lists[k].count;
-      if (np.ntiles == 0) continue;   // no matrix of this group iterates k times
+      if (np.ntiles == 0) continue;   // no matrix of this group iterates k times in this form
+      ctx->step_flops[MUONH_PHASE_NS_GRAM] += tile_flops * gr.gram_lists[k].sum_nk;
+      ctx->step_flops[MUONH_PHASE_NS_SQUARE] += tile_flops * gr.gram_lists[k].sum_nk_sq;
+      ctx->step_flops[MUONH_PHASE_NS_APPLY] += tile_flops * gr.apply_lists[k].sum_nk;
       if (ctx->pairs) {
-        const int pairs_max = std::max(1, ctx->sm_count / 2);
-        const int gp = std::min(pairs_max, std::max(1, np.ntiles));
-        STEP_LAUNCH_ON(MUONH_PHASE_NS_GRAM, launch_ns_gemm_pair(M_GRAM, ctx->prec, np, gp, st), "ns_gram", st);
-        STEP_LAUNCH_ON(MUONH_PHASE_NS_SQUARE, launch_ns_gemm_pair(M_SQUARE, ctx->prec, np, gp, st), "ns_square", st);
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_GRAM, launch_ns_gemm_pair(M_GRAM, ctx->prec, np, pair_grid(np.ntiles), st),
+                       "ns_gram", st);
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_SQUARE, launch_ns_gemm_pair(M_SQUARE, ctx->prec, np, pair_grid(np.ntiles), st),
+                       "ns_square", st);
         np.tiles = gr.apply_lists[k].dev;
         np.ntiles = gr.apply_lists[k].count;
+        np.lhs = RR_B;
+        np.lhs_kind = RK_P;
+        np.apply_kappa = k == 0;
         const int amode = (k == ctx->max_steps - 1) ? M_APPLY_LAST : M_APPLY;
-        STEP_LAUNCH_ON(MUONH_PHASE_NS_APPLY,
-                       launch_ns_gemm_pair(amode, ctx->prec, np, std::min(pairs_max, std::max(1, np.ntiles)), st),
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_APPLY, launch_ns_gemm_pair(amode, ctx->prec, np, pair_grid(np.ntiles), st),
                        "ns_apply", st);
       } else {
         const int ggrid = std::min(ctx->sm_count, std::max(1, np.ntiles));
@@ -780,6 +918,74 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
         STEP_LAUNCH_ON(MUONH_PHASE_NS_APPLY,
                        launch_ns_gemm(M_APPLY, ctx->prec, np, std::min(ctx->sm_count, std::max(1, np.ntiles)), st),
                        "ns_apply", st);
+      }
+    }
+    // ---- Gram-space form, run by run (see muonh_ns_gemm.cu): A_0 = Y Y^T; per
+    // iteration P = p(A) into B' or P1 (alternating); between iterations
+    // T = A P, A = T P; the run's product Q = P1 P0 (into T) and P2 Q (into
+    // P1); one Y <- Q Y (or P0 Y for a run of one) ends the run
+    if (gr.any_gram) {
+      const TileList& up = gr.gram_upper;
+      const TileList& ap = gr.gram_apply;
+      int k0 = 0;
+      for (size_t j = 0; j < ctx->runs.size(); ++j) {
+        const int run = ctx->runs[j];
+        NsParams np = base;
+        np.src = static_cast<int>(j & 1);
+        np.iter = k0;
+        np.tiles = up.dev;
+        np.ntiles = up.count;
+        ctx->step_flops[MUONH_PHASE_NS_GRAM] += tile_flops * up.sum_nk;
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_GRAM, launch_ns_gemm_pair(M_GRAM, ctx->prec, np, pair_grid(up.count), st),
+                       "ns_gram", st);
+        auto product = [&](int lhs, int lk, int rhs, int rk, int out, int ok) -> muonh_status {
+          NsParams pp = np;
+          pp.lhs = lhs;
+          pp.lhs_kind = lk;
+          pp.rhs = rhs;
+          pp.rhs_kind = rk;
+          pp.out = out;
+          pp.out_kind = ok;
+          ctx->step_flops[MUONH_PHASE_NS_PRODUCT] += tile_flops * up.sum_nk_sq;
+          STEP_LAUNCH_ON(MUONH_PHASE_NS_PRODUCT, launch_ns_gemm_pair(M_SYMPROD, ctx->prec, pp, pair_grid(up.count), st),
+                         "ns_product", st);
+          return MUONH_OK;
+        };
+        int qbuf = RR_B, qkind = RK_P;
+        for (int i = 0; i < run; ++i) {
+          const int pbuf = (i & 1) ? RR_P1 : RR_B;
+          np.iter = k0 + i;
+          np.lhs = RR_A;
+          np.rhs = RR_A;
+          np.out = pbuf;
+          ctx->step_flops[MUONH_PHASE_NS_SQUARE] += tile_flops * up.sum_nk_sq;
+          STEP_LAUNCH_ON(MUONH_PHASE_NS_SQUARE, launch_ns_gemm_pair(M_SQUARE, ctx->prec, np, pair_grid(up.count), st),
+                         "ns_square", st);
+          muonh_status ps;
+          if (i + 1 < run) {   // A_{k+1} = (A_k P_k) P_k
+            if ((ps = product(RR_A, RK_A, pbuf, RK_P, RR_T, RK_A)) || (ps = product(RR_T, RK_A, pbuf, RK_P, RR_A, RK_A)))
+              return ps;
+          }
+          if (i == 1) {        // Q = P1 P0
+            if ((ps = product(RR_P1, RK_P, RR_B, RK_P, RR_T, RK_Q))) return ps;
+            qbuf = RR_T;
+            qkind = RK_Q;
+          } else if (i == 2) { // Q = P2 Q (P2 is in B')
+            if ((ps = product(RR_B, RK_P, RR_T, RK_Q, RR_P1, RK_Q))) return ps;
+            qbuf = RR_P1;
+          }
+        }
+        np.iter = k0 + run - 1;
+        np.tiles = ap.dev;
+        np.ntiles = ap.count;
+        np.lhs = qbuf;
+        np.lhs_kind = qkind;
+        np.apply_kappa = j == 0;
+        ctx->step_flops[MUONH_PHASE_NS_APPLY] += tile_flops * ap.sum_nk;
+        const int amode = (j + 1 == ctx->runs.size()) ? M_APPLY_LAST : M_APPLY;
+        STEP_LAUNCH_ON(MUONH_PHASE_NS_APPLY, launch_ns_gemm_pair(amode, ctx->prec, np, pair_grid(ap.count), st),
+                       "ns_apply", st);
+        k0 += run;
       }
     }
     return MUONH_OK;
@@ -972,6 +1178,13 @@ muonh_status muonh_phase_times(muonh_ctx* ctx, float* ms_out, int64_t* launches_
     ms_out[i] = static_cast<float>(acc[i]);
     if (launches_out) launches_out[i] = cnt[i];
   }
+  return MUONH_OK;
+}
+
+muonh_status muonh_phase_flops(const muonh_ctx* ctx, double* flops_out) {
+  g_last_error.clear();
+  if (!ctx || !flops_out) return fail(MUONH_ERR_INVALID_ARG, "ctx or flops_out is NULL");
+  for (int i = 0; i < MUONH_NUM_PHASES; ++i) flops_out[i] = ctx->step_flops[i];
   return MUONH_OK;
 }
 

@@ -24,7 +24,16 @@ constexpr int kGemmThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2-5 epilog
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
 
 enum Prec { P_FP16 = 0, P_BF16 = 1, P_FP32 = 2 };
-enum Mode { M_GRAM = 0, M_SQUARE = 1, M_APPLY = 2, M_APPLY_LAST = 3 };   // LAST: also ||O||^2, <W, O>
+// LAST: also ||O||^2, <W, O>.  SYMPROD: product of two symmetric r x r
+// operands that commute (Gram-space form), stored with its mirror.
+enum Mode { M_GRAM = 0, M_SQUARE = 1, M_APPLY = 2, M_APPLY_LAST = 3, M_SYMPROD = 4 };
+
+// r x r buffers of a shape class, as operands of SQUARE / SYMPROD / APPLY.
+// The Y-space iteration uses A and B'; the Gram-space form also P1 and T.
+enum RrBuf { RR_A = 0, RR_B = 1, RR_P1 = 2, RR_T = 3 };
+// Power-of-two scale of a stored r x r operand: A-like (A, T = A P), P-like
+// (B' = p(A)), Q-like (a product of several p(A)).
+enum RrKind { RK_A = 0, RK_P = 1, RK_Q = 2 };
 
 // Tensor-map slots of one shape class.  "hi" buffers hold the 16-bit
 // operand (fp16/bf16), "lo" buffers the fp16 residual in FP32 mode.  The
@@ -40,8 +49,18 @@ enum TmSlot {
   TM_X_ST = 18,    // X[buf] store box 32 x 32 (64-byte swizzle)   (+buf)
   TM_A_ST = 20,    // A store box (direct and mirrored blocks)
   TM_B_ST = 21,    // B' store box (direct and mirrored blocks)
-  TM_PER_CLASS = 22
+  TM_P1_K128 = 22, // Gram-space form: P1, 128-row box
+  TM_T_K128 = 23,  // Gram-space form: T, 128-row box
+  TM_P1_ST = 24,   // P1 store box
+  TM_T_ST = 25,    // T store box
+  TM_PER_CLASS = 26
 };
+__host__ __device__ inline int tm_rr_k128(int buf) {
+  return buf == RR_A ? TM_A_K128 : buf == RR_B ? TM_B_K128 : buf == RR_P1 ? TM_P1_K128 : TM_T_K128;
+}
+__host__ __device__ inline int tm_rr_st(int buf) {
+  return buf == RR_A ? TM_A_ST : buf == RR_B ? TM_B_ST : buf == RR_P1 ? TM_P1_ST : TM_T_ST;
+}
 __host__ __device__ inline int tm_x(int base, int buf, int part) { return base + buf + 2 * part; }
 
 struct MatDev {
@@ -57,6 +76,9 @@ struct MatDev {
   int32_t ns_steps;
   float a, b, c_coef;
   int32_t ex, ea, ec, eb;    // power-of-two scales of stored X, A, C, B'
+  int32_t eq;                // Gram-space form: scale of a stored product of p(A) factors
+  int32_t gram;              // 1: Newton-Schulz in the Gram-space form (runs of <= 3 iterations)
+  int32_t o_buf;             // Y buffer that holds O after the last iteration
   int32_t rule;              // MUONH_RULE_*
   float wd, uscale;          // ordinary-Muon weight decay and update scale
   int32_t et_rows, et_cols;  // elementwise tile grid
@@ -75,6 +97,9 @@ struct ClassDev {
   void* a[2];                // [part]: A = Y Y^T
   void* c[2];                // C = b I + c A
   void* b[2];                // B' = a I + A C
+  void* p1;                  // Gram-space form only: second p(A) buffer
+  void* t;                   // Gram-space form only: A P, or a product of p(A) factors
+  float* bdiag;              // bf16 operands only: [count][r_pad] fp32 residual of B's stored diagonal
   int64_t x_stride, a_stride;   // elements per matrix
 };
 
@@ -116,7 +141,17 @@ struct NsParams {
   const ClassDev* classes;
   const CUtensorMap* tmaps;
   int* err;
+  // r x r operands of SQUARE / SYMPROD (lhs, rhs, out) and APPLY (lhs), as
+  // RrBuf ids, and the RrKind of each (which power-of-two scale it holds)
+  int32_t lhs, rhs, out;
+  int32_t lhs_kind, rhs_kind, out_kind;
+  int32_t apply_kappa;       // APPLY reads the momentum kernel's X: apply kappa
 };
+
+// Scale exponent of a stored r x r operand of the given RrKind.
+__host__ __device__ inline int rr_exp(const MatDev& md, int kind) {
+  return kind == RK_A ? md.ea : kind == RK_P ? md.eb : md.eq;
+}
 
 struct EwParams {
   const MatDev* mats;

@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(kEwThreads, 8) update_dots_kernel(const EwPara
     const TileCoord tc = tile_coord(p, e);
     const MatDev& md = p.mats[tc.mi];
     if (md.fused_dots) continue;   // the last APPLY produced this matrix's partials
-    const XView xv = x_view(p, md, md.ns_steps & 1);
+    const XView xv = x_view(p, md, md.o_buf);
     if (md.transposed) {
       __syncthreads();
       load_o_tile_t(xv, tc, p.prec, tile);
@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(kEwThreads, 6) project_kernel(const EwParams p
       continue;
     }
     const float kw = sc.kw, ko = sc.ko;
-    const XView xv = x_view(p, md, md.ns_steps & 1);
+    const XView xv = x_view(p, md, md.o_buf);
     if (mode == 0 && md.transposed) {
       __syncthreads();
       load_o_tile_t(xv, tc, p.prec, tile);
@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(kEwThreads) export_update_kernel(const EwParam
   __shared__ float tile[kEwTile][kEwTile + 1];
   const MatDev& md = p.mats[mi];
   const float unscale = exp2f(static_cast<float>(-md.ex));
-  const XView xv = x_view(p, md, md.ns_steps & 1);
+  const XView xv = x_view(p, md, md.o_buf);
   const int64_t n_tiles = static_cast<int64_t>(md.et_rows) * md.et_cols;
   for (int64_t local = blockIdx.x; local < n_tiles; local += gridDim.x) {
     const TileCoord tc = tile_coord(p, md.et_begin + local);

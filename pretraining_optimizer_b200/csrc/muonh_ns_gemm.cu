@@ -8,6 +8,12 @@
 //   GRAM    A  = Y Y^T  (and, FP32 mode, C = b I + c A)    M = r, N = r, K = c   (symmetric)
 //   SQUARE  B' = c A A + b A + a I  (FP32 mode: A C + a I)  M = r, N = r, K = r   (symmetric)
 //   APPLY   Y' = B' Y                                      M = r, N = c, K = r
+// The Gram-space form (fp16 operands) runs g <= 3 iterations on r x r
+// matrices between two passes over Y: with P_k = p(A_k) = a I + b A_k + c A_k^2,
+// A_{k+1} = Y_{k+1} Y_{k+1}^T = P_k A_k P_k = (A_k P_k) P_k, since all these
+// factors are polynomials in one symmetric matrix and commute; the run ends
+// with Y <- Q Y, Q = P_{g-1} ... P_0.  Its r x r products are
+//   SYMPROD out = L R   (L, R symmetric and commuting)      M = r, N = r, K = r   (symmetric)
 // Every launch covers the tiles of all matrices of the step (grouped), in a
 // persistent grid of one CTA per SM (one CTA pair per two SMs for 16-bit
 // operands).  Symmetric products compute only the tiles that touch the upper
@@ -599,7 +605,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         const MatDev& md = p.mats[td.mat];
         const ClassDev& cd = p.classes[md.cls];
         const int z = md.z;
-        const int nk = (MODE == M_SQUARE) ? td.nk_sq : td.nk;
+        const int nk = (MODE == M_SQUARE || MODE == M_SYMPROD) ? td.nk_sq : td.nk;
         const int abase = td.bi * kPairM, bbase = td.bj * kBN;                // tile origin
         const int arow = abase + static_cast<int>(rank) * 128;              // this CTA's A rows
         const int bcol = bbase + static_cast<int>(rank) * 128;              // this CTA's B half
@@ -613,16 +619,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
           if (MODE == M_GRAM) {
             tma_load_3d_pair(sa, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, arow, z);
             tma_load_3d_pair(sb, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, bcol, z);
-          } else if (MODE == M_SQUARE) {
-            // A A with A stored whole (GRAM writes every block and its mirror):
-            // both operands K-major; A is symmetric, so its rows serve as the
-            // N x K operand
-            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_A_K128, bar, k0, arow, z);
-            tma_load_3d_pair(sb, p.tmaps + cd.tm_base + TM_A_K128, bar, k0, bcol, z);
+          } else if (MODE == M_SQUARE || MODE == M_SYMPROD) {
+            // A A (SQUARE) or L R (SYMPROD) with both operands stored whole
+            // (every block and its mirror): both K-major; the right operand is
+            // symmetric, so its rows serve as the N x K operand
+            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
+            tma_load_3d_pair(sb, p.tmaps + cd.tm_base + tm_rr_k128(p.rhs), bar, k0, bcol, z);
           } else {
-            // APPLY: rows of B' (stored with its mirror, K-major) times Y,
+            // APPLY: rows of B' or Q (stored with its mirror, K-major) times Y,
             // read as an MN-major operand
-            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + TM_B_K128, bar, k0, arow, z);
+            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
             const CUtensorMap* bm = p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, 0);
             tma_load_3d_pair(sb, bm, bar, bcol, k0, z);
             tma_load_3d_pair(sb + 64 * kBK * 2, bm, bar, bcol + 64, k0, z);   // second 64-wide MN chunk
@@ -654,7 +660,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
       TileDesc td = pair < p.ntiles ? p.tiles[pair] : TileDesc{};
       for (int t = pair; t < p.ntiles && ok; t += npairs, ++local) {
         const TileDesc next = (t + npairs < p.ntiles) ? p.tiles[t + npairs] : td;   // prefetch
-        const int nk = (MODE == M_SQUARE) ? td.nk_sq : td.nk;
+        const int nk = (MODE == M_SQUARE || MODE == M_SYMPROD) ? td.nk_sq : td.nk;
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) { ok = false; break; }
@@ -745,11 +751,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
       const int row = row0 + lrow;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       // iteration 0 reads X at the momentum kernel's scale: kappa corrects it
-      const float kap = (p.iter == 0) ? p.scal[td.mat].kappa : 1.f;
+      const float kap = (MODE == M_GRAM && p.iter == 0) ? p.scal[td.mat].kappa : 1.f;
       uint8_t* mirror_buf = smem + C::kMirrorOffset + epi * 32 * C::kMirrorStride;
       const bool mirror = td.bj > td.bi;   // off-diagonal block: also store its transpose
-      if (MODE == M_GRAM) {
-        const float sa = kap * kap * exp2f(static_cast<float>(md.ea - 2 * md.ex));
+      if (MODE == M_GRAM || MODE == M_SYMPROD) {
+        // GRAM: stored A = 2^ea Y Y^T from the stored Y (2^ex Y);
+        // SYMPROD: stored out = 2^e_out L R from the stored L and R
+        const float sa = MODE == M_GRAM
+                             ? kap * kap * exp2f(static_cast<float>(md.ea - 2 * md.ex))
+                             : exp2f(static_cast<float>(rr_exp(md, p.out_kind) - rr_exp(md, p.lhs_kind) -
+                                                        rr_exp(md, p.rhs_kind)));
+        const CUtensorMap* omap = p.tmaps + cd.tm_base + (MODE == M_GRAM ? TM_A_ST : tm_rr_st(p.out));
         for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
           const int col0 = td.bj * kBN + ch * 32;
           float v[32];
@@ -762,12 +774,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
           for (int j = 0; j < 32; ++j) v[j] *= sa;
           uint4 pv[4];
           pack32<PREC>(v, pv);
-          stager.put(p.tmaps + cd.tm_base + TM_A_ST, lane, pv, col0, row0 + wrow0_off, md.z);
+          stager.put(omap, lane, pv, col0, row0 + wrow0_off, md.z);
           if (mirror) {
-            // A is symmetric: A[col][row] = A[row][col]
+            // the product is symmetric: out[col][row] = out[row][col]
             uint4 cv[4];
             warp_transpose32<PREC, C::kMirrorStride>(mirror_buf, lane, pv, cv);
-            stager.put(p.tmaps + cd.tm_base + TM_A_ST, lane, cv, row0 + wrow0_off, col0, md.z);
+            stager.put(omap, lane, cv, row0 + wrow0_off, col0, md.z);
           }
         }
       } else if (MODE == M_SQUARE) {
@@ -776,6 +788,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         const float s2 = md.c_coef * exp2f(static_cast<float>(md.eb - 2 * md.ea));
         const float s1 = md.b * exp2f(static_cast<float>(md.eb - md.ea));
         const float diag = md.a * exp2f(static_cast<float>(md.eb));
+        const CUtensorMap* omap = p.tmaps + cd.tm_base + tm_rr_st(p.out);
         using T16 = typename Store16<PREC>::T;
         for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
           const int col0 = td.bj * kBN + ch * 32;
@@ -801,26 +814,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
           const int dj = row - col0;
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j == dj) v[j] += diag;
+            if (j == dj) {
+              v[j] += diag;
+              // bf16 keeps 8 significant bits of the diagonal (near a = 3.44
+              // in early iterations): APPLY adds back the rounding residual
+              if (PREC == P_BF16)
+                cd.bdiag[static_cast<int64_t>(md.z) * cd.r_pad + row] = v[j] - Store16<PREC>::back(Store16<PREC>::cvt(v[j]));
+            }
           uint4 packed[4];
           pack32<PREC>(v, packed);
-          stager.put(p.tmaps + cd.tm_base + TM_B_ST, lane, packed, col0, row0 + wrow0_off, md.z);
+          stager.put(omap, lane, packed, col0, row0 + wrow0_off, md.z);
           if (mirror) {
             // B'[col0 + lane][row0 + 32 quarter + j] = B'[row0 + 32 quarter + j][col0 + lane]
             uint4 cv[4];
             warp_transpose32<PREC, C::kMirrorStride>(mirror_buf, lane, packed, cv);
-            stager.put(p.tmaps + cd.tm_base + TM_B_ST, lane, cv, row0 + wrow0_off, col0, md.z);
+            stager.put(omap, lane, cv, row0 + wrow0_off, col0, md.z);
           }
         }
         if (werr) break;
       } else {
-        const float ks = kap * exp2f(static_cast<float>(-md.eb));
+        // Y' = 2^ex (B' or Q) Y from the stored operand and Y; kappa where Y
+        // is the momentum kernel's X
+        const float ks = (p.apply_kappa ? p.scal[td.mat].kappa : 1.f) *
+                         exp2f(static_cast<float>(-rr_exp(md, p.lhs_kind)));
         const CUtensorMap* ymap = p.tmaps + cd.tm_base + TM_X_ST + (p.src ^ 1);
         // Last APPLY: Y' is the update O; accumulate ||O||^2 and <W, O> over
         // the stored values, W staged per 32-column chunk by TMA (wide W: box
         // of W[row0.., col0..]; tall W: box of W[col0.., row0..]).
         const bool dots = C::kLast && md.fused_dots && p.iter == md.ns_steps - 1;
         float oo = 0.f, wo = 0.f;
+        // bf16 operands: Y' = (B'_stored + diag(residual)) Y, the residual of
+        // this row times its own Y row, read from L2 one chunk ahead
+        float dres = 0.f;
+        const uint16_t* yrow = nullptr;
+        uint4 y_next[4];
+        if (PREC == P_BF16) {
+          dres = cd.bdiag[static_cast<int64_t>(md.z) * cd.r_pad + row];
+          yrow = static_cast<const uint16_t*>(cd.x[p.src][0]) + md.z * cd.x_stride +
+                 static_cast<int64_t>(row) * cd.c_pad + td.bj * kBN;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) y_next[q] = __ldg(reinterpret_cast<const uint4*>(yrow + ch0 * 32) + q);
+        }
         for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
           const int col0 = td.bj * kBN + ch * 32;
           float v[32];
@@ -828,6 +862,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
           if (ch + kChStep >= kBN / 32) {   // this warp's last chunk of the tile
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader[acc]);
+          }
+          if (PREC == P_BF16) {
+            uint4 y_cur[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) y_cur[q] = y_next[q];
+            if (ch + kChStep < kBN / 32) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) y_next[q] = __ldg(reinterpret_cast<const uint4*>(yrow + (ch + kChStep) * 32) + q);
+            }
+            using T16 = typename Store16<PREC>::T;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const T16* h = reinterpret_cast<const T16*>(&y_cur[q]);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[8 * q + e] = fmaf(dres, Store16<PREC>::back(h[e]), v[8 * q + e]);
+            }
           }
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] *= ks;
@@ -920,7 +970,7 @@ cudaError_t ns_gemm_set_attributes() {
 #define MUONH_SET_PAIR(MD, PR) \
   if ((e = set_pair_attr<MD, PR>()) != cudaSuccess) return e;
   MUONH_SET_PAIR(M_GRAM, P_FP16) MUONH_SET_PAIR(M_SQUARE, P_FP16) MUONH_SET_PAIR(M_APPLY, P_FP16)
-  MUONH_SET_PAIR(M_APPLY_LAST, P_FP16)
+  MUONH_SET_PAIR(M_APPLY_LAST, P_FP16) MUONH_SET_PAIR(M_SYMPROD, P_FP16)
   MUONH_SET_PAIR(M_GRAM, P_BF16) MUONH_SET_PAIR(M_SQUARE, P_BF16) MUONH_SET_PAIR(M_APPLY, P_BF16)
   MUONH_SET_PAIR(M_APPLY_LAST, P_BF16)
 #undef MUONH_SET_PAIR
@@ -945,7 +995,7 @@ cudaError_t launch_ns_gemm_pair(int mode, int prec, const NsParams& p, int pairs
     return cudaGetLastError();                                                                 \
   }
   MUONH_LAUNCH_PAIR(M_GRAM, P_FP16) MUONH_LAUNCH_PAIR(M_SQUARE, P_FP16) MUONH_LAUNCH_PAIR(M_APPLY, P_FP16)
-  MUONH_LAUNCH_PAIR(M_APPLY_LAST, P_FP16)
+  MUONH_LAUNCH_PAIR(M_APPLY_LAST, P_FP16) MUONH_LAUNCH_PAIR(M_SYMPROD, P_FP16)
   MUONH_LAUNCH_PAIR(M_GRAM, P_BF16) MUONH_LAUNCH_PAIR(M_SQUARE, P_BF16) MUONH_LAUNCH_PAIR(M_APPLY, P_BF16)
   MUONH_LAUNCH_PAIR(M_APPLY_LAST, P_BF16)
 #undef MUONH_LAUNCH_PAIR

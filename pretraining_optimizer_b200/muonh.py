@@ -24,14 +24,16 @@ FLAG_TIMEOUT = 16
 EXPORTED_SYMBOLS = (
     "muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
     "muonh_export_state", "muonh_import_state", "muonh_device_status", "muonh_last_launch_count",
-    "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc", "muonh_average",
+    "muonh_enable_timing", "muonh_phase_times", "muonh_phase_flops", "muonh_momentum_norm_noalloc",
+    "muonh_average",
     "muonh_adamw_step", "muonh_check_wait_timeout", "muonh_destroy", "muonh_status_string", "muonh_last_error",
 )
 DTYPE_F32, DTYPE_BF16 = 0, 1
 AVERAGE_MAX_INPUTS = 16
 ADAMW_MAX_TENSORS = 32
 PHASES = ("momentum_norm", "finalize_input", "write_x", "ns_gram", "ns_square", "ns_apply",
-          "update_dots", "finalize_update", "project", "finalize_step")
+          "update_dots", "finalize_update", "project", "finalize_step", "ns_product")
+NS_FORMS = {"auto": 0, "y": 1, "gram": 2}
 
 
 class MatrixDesc(Structure):
@@ -42,7 +44,7 @@ class MatrixDesc(Structure):
 
 
 class Config(Structure):
-    _fields_ = [("ns_precision", c_int32), ("eps", c_float)]
+    _fields_ = [("ns_precision", c_int32), ("eps", c_float), ("groups", c_int32), ("ns_form", c_int32)]
 
 
 class Stats(Structure):
@@ -93,6 +95,7 @@ def library() -> ctypes.CDLL:
     lib.muonh_last_launch_count.restype = c_int32
     lib.muonh_enable_timing.argtypes = [c_void_p, c_int32]
     lib.muonh_phase_times.argtypes = [c_void_p, POINTER(c_float), POINTER(c_int64)]
+    lib.muonh_phase_flops.argtypes = [c_void_p, POINTER(ctypes.c_double)]
     lib.muonh_momentum_norm_noalloc.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_float,
                                                 c_int32, c_void_p, c_void_p]
     lib.muonh_average.argtypes = [c_void_p, c_int32, POINTER(c_void_p), c_int32, c_int32, c_int64, c_void_p]
@@ -106,7 +109,7 @@ def library() -> ctypes.CDLL:
     lib.muonh_last_error.restype = c_char_p
     for name in ("muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
                  "muonh_export_state", "muonh_import_state", "muonh_device_status",
-                 "muonh_enable_timing", "muonh_phase_times", "muonh_momentum_norm_noalloc",
+                 "muonh_enable_timing", "muonh_phase_times", "muonh_phase_flops", "muonh_momentum_norm_noalloc",
                  "muonh_average", "muonh_adamw_step", "muonh_check_wait_timeout"):
         getattr(lib, name).restype = c_int32
     _LIB = lib
@@ -216,11 +219,19 @@ class MuonH:
     """MuonH over a list of fp32 CUDA weight matrices (updated in place).
 
     lr passed to step() is the effective LR eta^H of each matrix
-    (the caller applies the hyperball multiplier and the schedule)."""
+    (the caller applies the hyperball multiplier and the schedule).
+    beta, nesterov, ns_steps, ns_coeffs, update_rule, weight_decay and
+    update_scale take one value for every matrix or a per-matrix sequence.
+    groups=1 keeps every kernel of the step on the caller's stream (no
+    overlap of elementwise and Newton-Schulz work); 0 lets the library split
+    a large set into two overlapping groups.  ns_form picks the evaluation
+    of the Newton-Schulz iteration: "auto" (Gram-space runs where they save
+    FLOPs), "y" (Y-space for every matrix) or "gram" (Gram-space wherever
+    the fp16 path can run it)."""
 
     def __init__(self, weights, momenta=None, *, beta=0.95, nesterov=True, ns_steps=5,
                  ns_coeffs=QUINTIC, eps=1e-7, ns_precision="fp16", radii=None, stream=None,
-                 update_rule="hyperball", weight_decay=0.0, update_scale=1.0):
+                 update_rule="hyperball", weight_decay=0.0, update_scale=1.0, groups=0, ns_form="auto"):
         import torch
         self._lib = library()
         self.weights = list(weights)
@@ -246,10 +257,12 @@ class MuonH:
             rule = _RULE[rule] if isinstance(rule, str) else int(rule)
             wd = weight_decay if isinstance(weight_decay, (int, float)) else weight_decay[i]
             us = update_scale if isinstance(update_scale, (int, float)) else update_scale[i]
-            descs[i] = MatrixDesc(wp, mp, rows, cols, ld, R, bt, int(bool(nesterov)), steps, a, b, c,
+            nv = nesterov if isinstance(nesterov, (bool, int)) else nesterov[i]
+            descs[i] = MatrixDesc(wp, mp, rows, cols, ld, R, bt, int(bool(nv)), steps, a, b, c,
                                   rule, wd, us)
             self.shapes.append((rows, cols, ld))
-        cfg = Config(prec, eps)
+        form = NS_FORMS[ns_form] if isinstance(ns_form, str) else int(ns_form)
+        cfg = Config(prec, eps, int(groups), form)
         ctx = c_void_p()
         _check(self._lib.muonh_init(ctypes.byref(ctx), descs, n, ctypes.byref(cfg), _stream_handle(stream)))
         self._ctx = ctx
@@ -311,6 +324,12 @@ class MuonH:
 
     def enable_timing(self, enable: bool = True) -> None:
         _check(self._lib.muonh_enable_timing(self._ctx, int(bool(enable))))
+
+    def phase_flops(self) -> dict:
+        """{phase: tensor-core FLOPs its launches executed in the last step}."""
+        out = (ctypes.c_double * len(PHASES))()
+        _check(self._lib.muonh_phase_flops(self._ctx, out))
+        return {name: float(out[i]) for i, name in enumerate(PHASES)}
 
     def phase_times(self) -> dict:
         """{phase: (total ms, launches)} recorded since the previous call."""

@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_layouts_match_the_header():
     assert ctypes.sizeof(B.MatrixDesc) == 80
-    assert ctypes.sizeof(B.Config) == 8
+    assert ctypes.sizeof(B.Config) == 16 and B.Config.groups.offset == 8 and B.Config.ns_form.offset == 12
     assert ctypes.sizeof(B.Stats) == 24
     assert B.MatrixDesc.radius.offset == 40 and B.MatrixDesc.ns_c.offset == 64
     assert B.MatrixDesc.update_rule.offset == 68 and B.MatrixDesc.update_scale.offset == 76
@@ -56,6 +56,10 @@ def test_status_strings_and_argument_checks_without_a_gpu():
     cfg_bad = B.Config(7, 1e-7)
     d[0] = B.MatrixDesc(0x1000, 0x2000, 4, 8, 8, 0.0, 0.95, 1, 5, 3.4445, -4.775, 2.0315)
     assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(cfg_bad), None) == 1
+    assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(B.Config(0, 1e-7, 2)), None) == 1   # groups
+    assert b"groups" in lib.muonh_last_error()
+    assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(B.Config(0, 1e-7, 0, 3)), None) == 1   # ns_form
+    assert b"ns_form" in lib.muonh_last_error()
     assert lib.muonh_step(None, None, None, None, None) == 1
 
 
