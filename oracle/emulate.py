@@ -59,9 +59,22 @@ def mirror_upper_tiles(P, tile=256):
     return out
 
 
-def newton_schulz_stored(X, steps=5, coeffs=QUINTIC, eps=1e-7, storage="fp16"):
+def round_off_diagonal(B, r):
+    """B stored through r() except its diagonal, which is kept exactly (the
+    rounding residual of each diagonal entry carried separately in fp32 and
+    added back in the product that uses B)."""
+    out = r(B)
+    np.fill_diagonal(out, np.diag(np.asarray(B, dtype=np.float64)))
+    return out
+
+
+def newton_schulz_stored(X, steps=5, coeffs=QUINTIC, eps=1e-7, storage="fp16", exact_diagonal=False):
     """Newton-Schulz with every stored operand rounded to `storage`
-    ("fp16", "bf16" or "fp64" = no rounding).  Returns O as fp64."""
+    ("fp16", "bf16" or "fp64" = no rounding).  exact_diagonal=True keeps the
+    diagonal of B' = a I + b A + c A A unrounded (round_off_diagonal): once
+    the iterate's singular values approach 1, A is close to I and B' to
+    p(1) I, so B' is dominated by its diagonal, whose rounding is the
+    largest single error of a bf16 B'.  Returns O as fp64."""
     r = ROUND[storage]
     a, b, c = coeffs
     X = np.asarray(X, dtype=np.float64)
@@ -71,7 +84,8 @@ def newton_schulz_stored(X, steps=5, coeffs=QUINTIC, eps=1e-7, storage="fp16"):
     eye = np.eye(Y.shape[0])
     for _ in range(steps):
         A = r(Y @ Y.T)
-        Bp = r(a * eye + b * A + c * (A @ A))
+        Bp = a * eye + b * A + c * (A @ A)
+        Bp = round_off_diagonal(Bp, r) if exact_diagonal else r(Bp)
         Y = r(Bp @ Y)
     return Y.T.copy() if tall else Y
 

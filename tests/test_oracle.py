@@ -265,6 +265,30 @@ def test_storage_error_of_each_operand_format(storage, lo, hi):
     assert lo <= err <= hi, err
 
 
+def test_round_off_diagonal_keeps_only_the_diagonal():
+    from oracle import emulate
+    B = np.array([[3.4257, 1.0 + 2.0 ** -9, 0.3], [1.0 + 2.0 ** -9, 0.7001, -2.5e-3], [0.3, -2.5e-3, 1.1]])
+    out = emulate.round_off_diagonal(B, emulate.round_bf16)
+    assert np.array_equal(np.diag(out), np.diag(B))
+    off = ~np.eye(3, dtype=bool)
+    assert np.array_equal(out[off], emulate.round_bf16(B)[off])
+    assert out[0, 1] == 1.0                      # a bf16 tie rounded to even off the diagonal
+
+
+def test_exact_diagonal_emulation():
+    """Without rounding the exact-diagonal emulation is the oracle; with bf16
+    storage, keeping B's diagonal exact removes its largest rounding error:
+    on inputs whose iterate is small (r = 70) the error drops below the bf16
+    storage error of the plain form by a fifth or more."""
+    from oracle import emulate
+    X = synth.gaussian_gradient(0, 1, 70, 130).astype(np.float64)
+    ref = oracle.newton_schulz(X)
+    assert np.allclose(emulate.newton_schulz_stored(X, storage="fp64", exact_diagonal=True), ref, rtol=0, atol=1e-13)
+    plain = np.linalg.norm(emulate.newton_schulz_stored(X, storage="bf16") - ref) / np.linalg.norm(ref)
+    diag = np.linalg.norm(emulate.newton_schulz_stored(X, storage="bf16", exact_diagonal=True) - ref) / np.linalg.norm(ref)
+    assert diag <= 0.8 * plain and diag <= 1e-2, (diag, plain)
+
+
 def test_newton_schulz_is_orthogonally_equivariant():
     """NS(U X V^T) = U NS(X) V^T for orthogonal U, V: the iteration acts on
     singular values only (a max-norm or element-wise scaling would break this)."""

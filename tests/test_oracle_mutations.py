@@ -51,6 +51,8 @@ AUX_MUTATIONS = {
                                             "A = sym(sym(A @ Bp) @ Bp)", "A = sym(A @ Bp)"),
     "Q kept from the last iteration only": ("emulate.py", "tests/test_oracle.py",
                                             "Q = Bp if Q is None else sym(Bp @ Q)", "Q = Bp"),
+    "diagonal rounded anyway": ("emulate.py", "tests/test_oracle.py",
+                                "    np.fill_diagonal(out, np.diag(np.asarray(B, dtype=np.float64)))\n", ""),
     "lower tiles left unwritten": ("emulate.py", "tests/test_oracle.py",
                                    "out[i:i + tile, j:j + tile] = out[j:j + tile, i:i + tile].T",
                                    "out[i:i + tile, j:j + tile] = 0.0"),
