@@ -13,7 +13,7 @@ import pytest
 
 import oracle
 import synth
-from parity_helpers import FP16_NS_TOL, NORM_TOL, W_TOL_10, rel_fro
+from parity_helpers import FP16_NS_TOL, NORM_TOL, W_TOL_10, rel_fro, tile_rel_fro_max
 
 pytestmark = pytest.mark.gpu
 
@@ -115,6 +115,8 @@ def _one_step_check(run, wl, sample, t_check):
                                         wl.nesterov, wl.ns_steps, wl.ns_coeffs)
         O_gpu = run.opt.update(i).cpu().numpy()
         assert rel_fro(O_gpu, O) <= FP16_NS_TOL, (t_check, i, rel_fro(O_gpu, O))
+        worst = tile_rel_fro_max(O_gpu, O, tile=256)
+        assert worst <= FP16_NS_TOL, (t_check, i, worst)
         assert np.linalg.norm(run.W[i].cpu().numpy() - Wn) / run.R[i] <= 1e-4, (t_check, i)
         assert abs(stats[i]["update_norm"] - st["update_norm"]) <= FP16_NS_TOL * st["update_norm"]
         assert abs(stats[i]["input_norm"] - st["input_norm"]) <= NORM_TOL * st["input_norm"]
@@ -126,6 +128,9 @@ def _check_sampled_against_oracle(run, wl, sample, steps):
         W_ref, O_ref, st = ref[i]
         O_gpu = run.opt.update(i).cpu().numpy()
         assert rel_fro(O_gpu, O_ref) <= FP16_NS_TOL, (i, rel_fro(O_gpu, O_ref))
+        # every 256 x 256 block of O, the output tile of the Newton-Schulz GEMMs
+        worst = tile_rel_fro_max(O_gpu, O_ref, tile=256)
+        assert worst <= FP16_NS_TOL, (i, worst)
         assert np.linalg.norm(run.W[i].cpu().numpy() - W_ref) / R[i] <= W_TOL_10, i
 
 

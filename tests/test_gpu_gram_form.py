@@ -1,0 +1,127 @@
+"""The Gram-space evaluation of the Newton-Schulz iteration on the CUDA path
+(B200 only): runs of up to three iterations carried on r x r matrices
+(A_{k+1} = A_k p(A_k)^2, Y <- Q Y once per run), checked against the fp64
+oracle's Y-space iteration, which it equals in exact arithmetic, and against
+the oracle's fp16 storage emulation of the same form."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity_helpers import FP16_NS_TOL, NORM_TOL, W_TOL_10, rel_fro, run_gpu, run_oracle, tile_rel_fro_max
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("form", ["gram", "y"])
+def test_gram_form_matches_the_oracle(form):
+    """Wide, tall, ragged and square matrices, every one in the Gram form when
+    asked for (and in the Y-space form as the control), 10 steps."""
+    shapes = [(256, 768), (768, 256), (300, 1000), (512, 512), (130, 70), (256, 512)]
+    strides = [None, None, None, None, None, 520]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    lrs = [0.01] * 10
+    keep = (0, 9)
+    g = run_gpu(W0, grad, lrs, keep_updates=keep, strides=strides, ns_form=form)
+    o = run_oracle(W0, grad, lrs, keep_updates=keep)
+    for i, s in enumerate(shapes):
+        R = o["R"][i]
+        for t in keep:
+            err = rel_fro(g["O"][t][i], o["O"][t][i])
+            assert err <= FP16_NS_TOL, (form, i, s, t, err)
+            worst = tile_rel_fro_max(g["O"][t][i], o["O"][t][i], tile=64)
+            assert worst <= FP16_NS_TOL, (form, i, s, t, worst)
+        for t in range(len(lrs)):
+            gs, os_ = g["stats"][t][i], o["stats"][t][i]
+            assert gs["flags"] == 0
+            assert abs(gs["post_norm"] - R) <= NORM_TOL * R
+            assert abs(gs["elr"] - os_["elr"]) <= NORM_TOL * os_["elr"]
+            assert abs(gs["input_norm"] - os_["input_norm"]) <= NORM_TOL * os_["input_norm"]
+        assert np.linalg.norm(g["W"][i] - o["W"][i]) / R <= W_TOL_10, (form, i, s)
+
+
+@pytest.mark.parametrize("shape", [(256, 768), (640, 256), (512, 2048)])
+def test_gram_form_error_matches_its_storage_emulation(shape):
+    """The kernels store Y, A, T = A P, P = p(A) and Q in fp16 and accumulate
+    in fp32: the NS error against fp64 matches the oracle's fp16 emulation of
+    the Gram-space form, runs (3, 2), within 25 %."""
+    from oracle import emulate
+    W0 = [synth.initial_weight(0, *shape)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shape)
+    g = run_gpu(W0, grad, [0.01], keep_updates=(0,), ns_form="gram")
+    _, X = oracle.momentum_update(np.zeros(shape), grad(0, 0), 0.95, True)
+    ref = oracle.newton_schulz(X)
+    emu = rel_fro(emulate.newton_schulz_gram_stored(X, (3, 2), storage="fp16"), ref)
+    err = rel_fro(g["O"][0][0], ref)
+    assert 0.8 * emu <= err <= 1.25 * emu, (err, emu)
+
+
+@pytest.mark.parametrize("gradient", ["gaussian", "ill_conditioned"])
+def test_gram_form_at_the_qwen3_mlp_shapes(gradient):
+    """2048 x 6144 (down) and 6144 x 2048 (gate, up) take the Gram form by
+    default: two steps against the fp64 oracle, and the first step's error
+    against the fp16 emulation of the form."""
+    from oracle import emulate
+    shapes = [(2048, 6144), (6144, 2048)]
+    W0 = [synth.initial_weight(6 - 2 * i, *s) for i, s in enumerate(shapes)]
+
+    def grad(t, i):
+        if gradient == "gaussian":
+            return synth.gaussian_gradient(t, 6 - 2 * i, *shapes[i])
+        return synth.ill_conditioned_gradient(t, 6 - 2 * i, *shapes[i])
+
+    lrs = [0.008, 0.00784]
+    g = run_gpu(W0, grad, lrs, keep_updates=(0, 1))
+    assert g["flops"]["ns_product"] > 0          # the default form here is the Gram form
+    o = run_oracle(W0, grad, lrs, keep_updates=(0, 1))
+    for i in range(2):
+        R = o["R"][i]
+        for t in range(2):
+            err = rel_fro(g["O"][t][i], o["O"][t][i])
+            assert err <= FP16_NS_TOL, (i, t, err)
+            assert tile_rel_fro_max(g["O"][t][i], o["O"][t][i], tile=256) <= FP16_NS_TOL, (i, t)
+            assert abs(g["stats"][t][i]["post_norm"] - R) <= NORM_TOL * R
+            assert abs(g["stats"][t][i]["elr"] - lrs[t]) <= NORM_TOL * lrs[t]
+        assert np.linalg.norm(g["W"][i] - o["W"][i]) / R <= 1e-4, i
+    _, X = oracle.momentum_update(np.zeros(shapes[0]), grad(0, 0), 0.95, True)
+    ref = oracle.newton_schulz(X)
+    emu = rel_fro(emulate.newton_schulz_gram_stored(X, (3, 2), storage="fp16"), ref)
+    err = rel_fro(g["O"][0][0], ref)
+    assert 0.8 * emu <= err <= 1.25 * emu, (err, emu)
+
+
+def _upper(r_pad):
+    b = r_pad // 256
+    return b * (b + 1) // 2
+
+
+def test_executed_flops_of_each_form():
+    """The tensor-core FLOPs the library reports per phase equal the tile
+    counts of each form: Y-space per iteration Y Y^T and B' on the upper
+    256 x 256 tiles, B' Y on all; Gram-space per run of g one Y Y^T, g
+    squares and 4 g - 3 - g other products on the upper tiles, one Q Y."""
+    shapes = [(512, 1536), (256, 512)]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    tile = 2 * 256 * 256
+    flops = {}
+    for form in ("y", "gram"):
+        flops[form] = run_gpu(W0, grad, [0.01], ns_form=form)["flops"]
+    y = flops["y"]
+    exp_gram = exp_sq = exp_apply = 0
+    for r, c in shapes:
+        exp_gram += 5 * _upper(r) * tile * c
+        exp_sq += 5 * _upper(r) * tile * r
+        exp_apply += 5 * (r // 256) * (c // 256) * tile * r
+    assert (y["ns_gram"], y["ns_square"], y["ns_apply"], y["ns_product"]) == (exp_gram, exp_sq, exp_apply, 0)
+    gf = flops["gram"]
+    exp_gram = exp_sq = exp_apply = exp_prod = 0
+    for r, c in shapes:
+        for g in (3, 2):
+            exp_gram += _upper(r) * tile * c
+            exp_sq += g * _upper(r) * tile * r
+            exp_prod += (3 * g - 3) * _upper(r) * tile * r
+            exp_apply += (r // 256) * (c // 256) * tile * r
+    assert (gf["ns_gram"], gf["ns_square"], gf["ns_apply"], gf["ns_product"]) == (exp_gram, exp_sq, exp_apply,
+                                                                                   exp_prod)

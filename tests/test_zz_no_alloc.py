@@ -1,37 +1,52 @@
-"""The allocation-free momentum entry point against muonh_step (B200 only).
+"""The allocation-free momentum entry point (B200 only).
 
-Callers that cannot allocate device memory (stream capture in global mode,
-framework-owned or fixed-arena device memory, allocation-lock-free loops)
-use muonh_momentum_norm_noalloc, whose scratch is compiled into the library.
-Over two calls in a row it must reproduce what muonh_step does to the
-momentum buffer and the input norm it reports."""
+Callers that cannot allocate device memory -- code running while a stream is
+captured in the global mode, programs whose device memory belongs to a
+framework allocator or a fixed arena, loops that must not take the driver's
+allocation locks -- use muonh_momentum_norm_noalloc, whose scratch is an
+array compiled into the library.  Over two calls in a row it must give the
+fp64 oracle's momentum buffer and Newton-Schulz input norm, and agree with
+what muonh_step does to the same buffer.  This file is collected last, so a
+stop at the first failure has run every other test."""
 import numpy as np
 import pytest
 
+import oracle
 import synth
-from parity_helpers import NORM_TOL
+from parity_helpers import NORM_TOL, rel_fro
 
 pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("shape", [(256, 512), (768, 256), (96, 301)])
-def test_noalloc_momentum_matches_the_step_on_two_calls(shape):
+@pytest.mark.parametrize("nesterov", [True, False])
+def test_noalloc_momentum_matches_the_oracle_and_the_step_on_two_calls(shape, nesterov):
     import torch
     from pretraining_optimizer_b200 import MuonH, momentum_norm_noalloc
     dev = torch.device("cuda:0")
+    beta = 0.95
     W = torch.from_numpy(synth.initial_weight(0, *shape)).to(dev)
-    M_ref = torch.zeros_like(W)
-    opt = MuonH([W], [M_ref])
+    M_step = torch.zeros_like(W)
+    opt = MuonH([W], [M_step], beta=beta, nesterov=nesterov)
     M = torch.zeros_like(W)
+    M_ref = np.zeros(shape)
     x_norm = torch.empty((), dtype=torch.float64, device=dev)
     for t in range(2):
-        G = torch.from_numpy(synth.gaussian_gradient(t, 0, *shape)).to(dev)
+        g = synth.gaussian_gradient(t, 0, *shape)
+        G = torch.from_numpy(g).to(dev)
         opt.step([G], 0.01)
-        momentum_norm_noalloc(M, G, beta=0.95, nesterov=True, x_norm=x_norm)
+        momentum_norm_noalloc(M, G, beta=beta, nesterov=nesterov, x_norm=x_norm)
         torch.cuda.synchronize()
-        ref_norm = opt.stats()[0]["input_norm"]
-        assert np.array_equal(M.cpu().numpy(), M_ref.cpu().numpy()), t
-        assert abs(float(x_norm.item()) - ref_norm) <= NORM_TOL * ref_norm, (t, float(x_norm.item()), ref_norm)
+        # the oracle, fp64: M_t = beta M_{t-1} + G_t and ||X||_F
+        M_ref, X_ref = oracle.momentum_update(M_ref, g, beta, nesterov)
+        ref_norm = float(np.linalg.norm(X_ref))
+        got = float(x_norm.item())
+        assert rel_fro(M.cpu().numpy(), M_ref) <= 1e-6, (t, rel_fro(M.cpu().numpy(), M_ref))
+        assert abs(got - ref_norm) <= NORM_TOL * ref_norm, (t, got, ref_norm)
+        # the context-based step on the same inputs
+        step_norm = opt.stats()[0]["input_norm"]
+        assert rel_fro(M.cpu().numpy(), M_step.cpu().numpy()) <= 1e-6, t
+        assert abs(got - step_norm) <= NORM_TOL * step_norm, (t, got, step_norm)
     opt.close()
 
 
