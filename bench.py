@@ -43,6 +43,7 @@ KERNEL_BYTES = {
 # write_x only rewrites X for matrices whose momentum-kernel scale left the safe
 # range (every matrix on the first step); it is timed but not given a GB/s.
 ELEMENTWISE = ("momentum_norm", "write_x", "update_dots", "project")
+NS_PHASES = ("ns_gram", "ns_square", "ns_product", "ns_apply")
 # algorithmic bytes per element of the whole step (read G, M, W, O; write M, X, W)
 ALGO_BYTES_PER_ELEM = 24
 
@@ -55,9 +56,14 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3_1.7b")
     ap.add_argument("--ns-precision", default="fp16", choices=["fp16", "bf16", "fp32"])
+    ap.add_argument("--ns-form", default="auto", choices=["auto", "y", "gram"],
+                    help="Newton-Schulz evaluation: Gram-space runs where they save FLOPs (auto), "
+                         "Y-space everywhere, or Gram-space wherever fp16 allows")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-aux", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the side records (elementwise alone, bf16, Qwen3-0.6B, shape sweep)")
     return ap.parse_args()
 
 
@@ -75,37 +81,6 @@ def ns_flops(shapes, steps):
         r, c = min(rr, cc), max(rr, cc)
         tot += steps * (4 * r * r * c + 2 * r ** 3)
     return tot
-
-
-def ns_flops_executed(shapes, steps, prec="fp16"):
-    """Tensor-core FLOPs the Newton-Schulz kernels execute: GRAM and SQUARE
-    run the tiles of the upper block triangle (256 x 256 CTA-pair tiles, or
-    128 x 256 single-CTA tiles with three products each in FP32 mode), APPLY
-    every tile of Y, all on the 256-padded buffers."""
-    tm, mult = (128, 3) if prec == "fp32" else (256, 1)
-    tot = 0
-    for a, b in shapes:
-        r = (min(a, b) + 255) // 256 * 256
-        c = (max(a, b) + 255) // 256 * 256
-        upper = sum(1 for bi in range(r // tm) for bj in range(r // 256) if bj * 256 + 255 >= bi * tm)
-        tile = 2 * tm * 256
-        tot += steps * mult * (upper * tile * c + upper * tile * r + (r // tm) * (c // 256) * tile * r)
-    return tot
-
-
-def apply_flops(shapes):
-    """One APPLY pass over the set (Y' = aY + BY for every matrix): 2 r^2 c
-    per matrix.  A step makes ns_steps such passes; a large set splits each
-    pass into one launch per matrix group."""
-    return sum(2 * min(a, b) ** 2 * max(a, b) for a, b in shapes)
-
-
-def apply_bytes(shapes):
-    """Algorithmic HBM bytes of one APPLY pass: read B' (r x r) and Y (r x c),
-    write Y', 16-bit, on the 256-padded Newton-Schulz buffers."""
-    def pad(v):
-        return (v + 255) // 256 * 256
-    return sum(2 * pad(min(a, b)) ** 2 + 4 * pad(min(a, b)) * pad(max(a, b)) for a, b in shapes)
 
 
 def load_peaks():
@@ -162,16 +137,16 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
-def committed_traffic(kernel_file, workload, prec):
-    """DRAM bytes of one APPLY pass over the set (the dominant kernel) from a
+def committed_traffic(kernel_file, phase, workload, prec):
+    """DRAM bytes of one step's launches of the dominant kernel phase from a
     committed ncu summary, or None when the kernel source changed since the
-    counters were taken."""
+    counters were taken (or none were taken for this phase and workload)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    key = f"ns_apply/{workload}/{prec}"
+    key = f"{phase}/{workload}/{prec}"
     if key not in d:
         return None
     src = os.path.join(ROOT, "pretraining_optimizer_b200", "csrc", kernel_file)
@@ -179,7 +154,7 @@ def committed_traffic(kernel_file, workload, prec):
         digest = hashlib.sha256(f.read()).hexdigest()
     if d[key].get("source_sha256") != digest:
         return None
-    return d[key]["dram_bytes_per_pass"]
+    return d[key]["dram_bytes_per_step"]
 
 
 def max_over_ranks(value: float, world: int) -> float:
@@ -223,7 +198,11 @@ def cpu_sample(shapes, ns_steps):
 
 def oracle_sample_rate(shapes, wl, sample_idx, steps=1):
     """Time the oracle (as it stands, fp64) on a sample of the set for `steps`
-    steps; return (steps/s scaled to the whole set, seconds, sample FLOPs share)."""
+    steps, its Newton-Schulz products and its elementwise work (momentum,
+    norms, the Eq. (1) projection) apart, each called in the order of
+    oracle.muonh_step.  The whole-set step time is each part's time scaled by
+    its own share of the set (NS FLOPs, elements).  Returns (steps/s of the
+    whole set, seconds timed, NS FLOP share, element share)."""
     import numpy as np
     import oracle
     W0 = {i: wl.weight(i) for i in sample_idx}
@@ -231,14 +210,23 @@ def oracle_sample_rate(shapes, wl, sample_idx, steps=1):
     M = {i: np.zeros_like(W0[i], dtype=np.float64) for i in sample_idx}
     W = {i: W0[i].astype(np.float64) for i in sample_idx}
     R = {i: oracle.radius(W0[i]) for i in sample_idx}
-    t0 = time.perf_counter()
+    t_ns = t_ew = 0.0
     for t in range(steps):
         for i in sample_idx:
-            W[i], M[i], _, _ = oracle.muonh_step(W[i], M[i], Gs[(t, i)], wl.lrs[t % len(wl.lrs)], R[i],
-                                                 wl.beta, wl.nesterov, wl.ns_steps, wl.ns_coeffs)
-    dt = time.perf_counter() - t0
-    share = ns_flops([shapes[i] for i in sample_idx], wl.ns_steps) / ns_flops(shapes, wl.ns_steps)
-    return steps * share / dt, dt, share
+            t0 = time.perf_counter()
+            M[i], X = oracle.momentum_update(M[i], Gs[(t, i)], wl.beta, wl.nesterov)
+            float(np.linalg.norm(X))
+            t1 = time.perf_counter()
+            O = oracle.newton_schulz(X, wl.ns_steps, wl.ns_coeffs)
+            t2 = time.perf_counter()
+            W[i], _ = oracle.hyperball_update(W[i], O, wl.lrs[t % len(wl.lrs)], R[i])
+            t3 = time.perf_counter()
+            t_ew += (t1 - t0) + (t3 - t2)
+            t_ns += t2 - t1
+    ns_share = ns_flops([shapes[i] for i in sample_idx], wl.ns_steps) / ns_flops(shapes, wl.ns_steps)
+    el_share = sum(shapes[i][0] * shapes[i][1] for i in sample_idx) / sum(a * b for a, b in shapes)
+    full_step_s = (t_ns / ns_share + t_ew / el_share) / steps
+    return 1.0 / full_step_s, t_ns + t_ew, ns_share, el_share
 
 
 def blas_threads():
@@ -252,7 +240,8 @@ def blas_threads():
 def bench_config(args, wl, shapes, world):
     """The workload description both arms report."""
     return {"workload": args.workload, "matrices": len(shapes), "params": sum(a * b for a, b in shapes),
-            "ns_steps": wl.ns_steps, "ns_precision": args.ns_precision, "state": "fp32 W, M, G",
+            "ns_steps": wl.ns_steps, "ns_precision": args.ns_precision, "ns_form": args.ns_form,
+            "state": "fp32 W, M, G",
             "lr": "workload schedule", "l2": "inputs larger than L2 (no flush)",
             "parallelism": f"{world} independent replica(s)"}
 
@@ -263,19 +252,18 @@ def run_reference(args):
         return 0
     wl, shapes = workload_desc(args.workload)
     layer0 = list(range(min(7, len(shapes))))
-    times, shares = [], []
+    step_s = []
     for k in range(args.warmup + args.steps):
         idx = [layer0[k % len(layer0)]]           # one matrix of layer 0 per step, in rotation
-        _, dt, share = oracle_sample_rate(shapes, wl, idx)
+        rate, _, _, _ = oracle_sample_rate(shapes, wl, idx)
         if k >= args.warmup:
-            times.append(dt)
-            shares.append(share)
-    # each sampled step stands for share of a full step: full-step time = dt / share
-    full_step_s = sum(times) / sum(shares)
+            step_s.append(1.0 / rate)
+    full_step_s = sum(step_s) / len(step_s)
     value = 1.0 / full_step_s
     cores = blas_threads()
-    sample = (f"one layer-0 matrix per step in rotation ({len(layer0)} matrices), fp64 NumPy oracle, "
-              f"time scaled to the whole {len(shapes)}-matrix set by Newton-Schulz FLOP share")
+    sample = (f"one layer-0 matrix per step in rotation ({len(layer0)} matrices), fp64 NumPy oracle on "
+              f"{os.cpu_count()} host cores ({cores} BLAS threads); its Newton-Schulz time scaled to the whole "
+              f"{len(shapes)}-matrix set by NS FLOP share, its elementwise time by element share")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * full_step_s,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -339,6 +327,124 @@ def measure_aux(dev, stream, hbm_peak, matrix_params):
     }
 
 
+def time_set(shapes, wl, prec, groups, warmup, steps, dev, stream, seed, ns_form="auto"):
+    """One context over `shapes` with device-drawn inputs of the workload's
+    distributions: `warmup` untimed steps, then `steps` steps bracketed by
+    CUDA events on the launching stream with per-kernel timing on.  Returns
+    (ms per step, {phase: (ms, launches)} of the timed steps, {phase:
+    executed tensor FLOPs per step})."""
+    import torch
+    from pretraining_optimizer_b200 import MuonH
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    W = [torch.randn(s, generator=gen, device=dev) * 0.02 for s in shapes]
+    M = [torch.zeros_like(w) for w in W]
+    G = [torch.randn(s, generator=gen, device=dev) * 1e-3 for s in shapes]
+    opt = MuonH(W, M, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps, ns_coeffs=wl.ns_coeffs,
+                ns_precision=prec, groups=groups, ns_form=ns_form)
+    lrs = wl.lrs
+    for k in range(warmup):
+        opt.step(G, lrs[k % len(lrs)])
+    torch.cuda.synchronize()
+    opt.phase_times()
+    opt.enable_timing(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(steps):
+        opt.step(G, lrs[k % len(lrs)])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    opt.enable_timing(False)
+    phases = opt.phase_times()
+    flops = opt.phase_flops()
+    opt.device_status()
+    opt.close()
+    del W, M, G
+    torch.cuda.empty_cache()
+    return e0.elapsed_time(e1) / steps, phases, flops
+
+
+def ns_record(ms, phases, flops, steps, peak_t):
+    """Newton-Schulz rates of a timed set: executed TFLOP/s over the GEMM
+    phases, and the most time-consuming GEMM phase's TFLOP/s against the
+    sustained peak."""
+    ns = [k for k in NS_PHASES if phases[k][1] > 0]
+    ns_ms = sum(phases[k][0] for k in ns) / steps
+    dom = max(ns, key=lambda k: phases[k][0])
+    dom_t = flops[dom] / (phases[dom][0] / steps / 1000.0) / 1e12
+    return {"steps_per_s": 1000.0 / ms, "ms_per_step": ms, "ns_ms_per_step": ns_ms,
+            "ns_tflops_executed": sum(flops[k] for k in ns) / (ns_ms / 1000.0) / 1e12,
+            "dominant": dom, "dominant_tflops": dom_t, "dominant_frac": dom_t / peak_t}
+
+
+def side_records(dev, stream, peaks, args):
+    """Measurements beside the headline line, each its own context on fresh
+    device inputs (rank 0 of a single-GPU run):
+      elementwise_alone  the momentum and projection kernels of the Qwen3-1.7B
+                         set, each kind of tile on its own (tall: gate and up;
+                         wide: the rest) with the step in one group, so no
+                         launch overlaps another; against the burst HBM peak;
+      bf16               the Qwen3-1.7B set with bf16 Newton-Schulz operands;
+      qwen3_0.6b         the Qwen3-0.6B set (fp16 operands, its WSD schedule);
+      sweep              each shape of the roofline sweep in one group: the
+                         executed NS TFLOP/s and each elementwise kernel's GB/s."""
+    import synth
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    sampler = ClockSampler([torch_device_index(dev)])
+    out = {}
+    wl17, shapes17 = workload_desc("qwen3_1.7b")
+
+    def ew(phases, name, elems, per_elem):
+        t, cnt = phases[name]
+        ms = t / cnt
+        gbps = per_elem * elems / ms / 1e6
+        return {"ms_per_launch": ms, "launches": cnt, "gbps": gbps, "frac": gbps / hbm}
+
+    alone = {}
+    for kind, sub in (("tall", [s for s in shapes17 if s[0] > s[1]]), ("wide", [s for s in shapes17 if s[0] <= s[1]])):
+        ms, ph, _ = time_set(sub, wl17, "fp16", 1, 3, 5, dev, stream, seed=11)
+        el = sum(a * b for a, b in sub)
+        alone[kind] = {"matrices": len(sub), "elements": el,
+                       "momentum_norm": ew(ph, "momentum_norm", el, KERNEL_BYTES["momentum_norm"]),
+                       "project": ew(ph, "project", el, KERNEL_BYTES["project"])}
+    alone["peak"] = "hbm_gbs (burst copy): each launch runs alone"
+    out["elementwise_alone"] = alone
+
+    ms, ph, fl = time_set(shapes17, wl17, "bf16", 0, 3, 10, dev, stream, seed=12)
+    out["bf16"] = {"workload": "qwen3_1.7b", "ns_precision": "bf16", "ns_form": "y (bf16 runs the Y-space form)",
+                   **ns_record(ms, ph, fl, 10, peak_t)}
+
+    ms, ph, fl = time_set(shapes17, wl17, "fp16", 0, 3, 10, dev, stream, seed=15, ns_form="y")
+    out["fp16_y_space"] = {"workload": "qwen3_1.7b", "ns_precision": "fp16", "ns_form": "y",
+                           **ns_record(ms, ph, fl, 10, peak_t)}
+
+    wl06, shapes06 = workload_desc("qwen3_0.6b")
+    ms, ph, fl = time_set(shapes06, wl06, "fp16", 0, 5, 20, dev, stream, seed=13)
+    el06 = sum(a * b for a, b in shapes06)
+    ew06 = sum(ph[k][0] for k in ELEMENTWISE if k in ph) / 20
+    out["qwen3_0.6b"] = {"workload": "qwen3_0.6b", "matrices": len(shapes06), "params": el06,
+                         **ns_record(ms, ph, fl, 20, peak_t),
+                         "elementwise_gbps_algorithmic": ALGO_BYTES_PER_ELEM * el06 / (ew06 / 1000.0) / 1e9}
+
+    sweep = []
+    for r, c in synth.SWEEP_SHAPES:
+        wls, shs = workload_desc(f"sweep_{r}x{c}")
+        ms, ph, fl = time_set(shs, wls, "fp16", 1, 3, 3, dev, stream, seed=14)
+        el = sum(a * b for a, b in shs)
+        sweep.append({"shape": [r, c], "matrices": len(shs), **ns_record(ms, ph, fl, 3, peak_t),
+                      "momentum_norm_gbps": ew(ph, "momentum_norm", el, KERNEL_BYTES["momentum_norm"])["gbps"],
+                      "project_gbps": ew(ph, "project", el, KERNEL_BYTES["project"])["gbps"]})
+    out["sweep"] = sweep
+    out["side_clocks"] = sampler.stop()
+    return out
+
+
+def torch_device_index(dev):
+    return dev.index if dev.index is not None else 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -364,7 +470,7 @@ def run_ours(args):
     M = [torch.zeros_like(w) for w in W]
     G = [torch.randn(s, generator=gen, device=dev) * 1e-3 for s in shapes]
     opt = MuonH(W, M, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps, ns_coeffs=wl.ns_coeffs,
-                ns_precision=args.ns_precision)
+                ns_precision=args.ns_precision, ns_form=args.ns_form)
     lrs = wl.lrs
     stream = torch.cuda.current_stream()
 
@@ -474,22 +580,29 @@ def run_ours(args):
         if name in KERNEL_BYTES:
             entry["gbps"] = KERNEL_BYTES[name] * elems / (tms / args.steps / 1000.0) / 1e9
         kernels[name] = entry
-    # APPLY FLOPs of the timed region over the APPLY launches' summed device time
-    apply_ms, apply_n = phases["ns_apply"]
-    ap_flops = apply_flops(shapes) * wl.ns_steps * args.steps
-    achieved = ap_flops / (apply_ms / 1000.0) / 1e12
+    # Newton-Schulz rooflines from the FLOPs each phase's tiles execute (the
+    # library counts them per launch) over the phase's summed device time;
+    # the dominant kernel is the GEMM phase that takes the most time
+    flops = opt.phase_flops()
+    ns_phases = [k for k in NS_PHASES if phases[k][1] > 0]
+    for k in ns_phases:
+        kernels[k]["tflops_executed"] = flops[k] / (phases[k][0] / args.steps / 1000.0) / 1e12
+    dom = max(ns_phases, key=lambda k: phases[k][0])
+    achieved = kernels[dom]["tflops_executed"]
     peak_t = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    roofline = {"bound": "tensor", "kernel": "ns_apply", "achieved": achieved, "peak": peak_t,
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_t,
                 "unit": "TFLOP/s", "frac": achieved / peak_t,
-                "traffic": committed_traffic("muonh_ns_gemm.cu", args.workload, args.ns_precision),
-                "per": "one APPLY pass over the set (5 a step; one launch per matrix group)",
-                "algorithmic_bytes": apply_bytes(shapes),
+                "traffic": committed_traffic("muonh_ns_gemm.cu", dom, args.workload, args.ns_precision),
+                "per": f"the {dom} launches of one step ({phases[dom][1] // args.steps} a step)",
+                "flops_per_step": flops[dom],
                 "peak_source": f"bf16_tflops_sustained ({peak_src}); fp16 operands run at the bf16 rate"}
-    ns_ms = sum(phases[k][0] for k in ("ns_gram", "ns_square", "ns_apply")) / args.steps
+    ns_ms = sum(phases[k][0] for k in ns_phases) / args.steps
     ew_ms = sum(phases[k][0] for k in ELEMENTWISE) / args.steps
     summary = {
-        "ns_tflops_dense": ns_flops(shapes, wl.ns_steps) / (ns_ms / 1000.0) / 1e12,
-        "ns_tflops_executed": ns_flops_executed(shapes, wl.ns_steps, args.ns_precision) / (ns_ms / 1000.0) / 1e12,
+        "ns_form": args.ns_form,
+        "ns_tflops_method_dense": ns_flops(shapes, wl.ns_steps) / (ns_ms / 1000.0) / 1e12,
+        "ns_tflops_executed": sum(flops[k] for k in ns_phases) / (ns_ms / 1000.0) / 1e12,
+        "ns_flops_executed_per_step": sum(flops[k] for k in ns_phases),
         "ns_ms_per_step": ns_ms,
         "elementwise_ms_per_step": ew_ms,
         "elementwise_gbps_algorithmic": ALGO_BYTES_PER_ELEM * elems / (ew_ms / 1000.0) / 1e9,
@@ -501,15 +614,25 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_aux and args.workload == "qwen3_1.7b":
         aux = measure_aux(dev, stream, peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), elems)
 
+    # ---------------- side records (rank 0 of a single-GPU run of the headline set)
+    side = {}
+    if rank == 0 and world == 1 and not args.no_extra and args.workload == "qwen3_1.7b":
+        opt.close()
+        opt = None
+        del W, M, G
+        torch.cuda.empty_cache()
+        side = side_records(dev, stream, peaks, args)
+
     # ---------------- CPU baseline: the oracle on the leading matrices, rank 0, N = 1
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sample = cpu_sample(shapes, wl.ns_steps)
-        rate, dt, share = oracle_sample_rate(shapes, wl, sample)
-        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"the leading {len(sample)} of {n} matrices"
-                         f"{' (layer 0)' if args.workload.startswith('qwen3') else ''}, {share:.4f} of the NS "
-                         f"FLOPs, one fp64 step ({dt:.1f} s), scaled to the whole set"}
+        rate, dt, share, el_share = oracle_sample_rate(shapes, wl, sample)
+        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "nproc": os.cpu_count(), "kind": "oracle",
+               "sample": f"one measured fp64 step ({dt:.1f} s) of the leading {len(sample)} of {n} matrices"
+                         f"{' (layer 0)' if args.workload.startswith('qwen3') else ''}: {share:.4f} of the NS "
+                         f"FLOPs and {el_share:.4f} of the elements; Newton-Schulz and elementwise times "
+                         f"scaled to the whole set by their own shares"}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -520,9 +643,10 @@ def run_ours(args):
                 "config": bench_config(args, wl, shapes, world),
                 "roofline": roofline, "summary": summary, "kernels": kernels, "clocks": clocks,
                 "gpu_launches": launches_per_step * args.steps, "e2e": e2e, "cpu_baseline": cpu,
-                "aux_kernels": aux}
+                "aux_kernels": aux, **side}
         print(json.dumps(line), flush=True)
-    opt.close()
+    if opt is not None:
+        opt.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

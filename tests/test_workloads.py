@@ -45,16 +45,3 @@ def test_cpu_sample_stays_within_its_flop_bound(shape):
     assert len(idx) == 1 or flops <= bench.CPU_SAMPLE_FLOPS
     if len(idx) < 7:       # one more matrix would break the bound
         assert bench.ns_flops(shapes[:len(idx) + 1], wl.ns_steps) > bench.CPU_SAMPLE_FLOPS
-
-
-def test_executed_newton_schulz_flops():
-    """Upper-triangle tiles only: for r = c = 2048 (8 tile rows, 36 of 64
-    tiles) GRAM and SQUARE run 36/64 of their dense 2 r^3, APPLY all of its
-    2 r^3; a single tile row runs the dense count; FP32 mode runs three
-    products on the same tiles."""
-    r = 2048
-    assert bench.ns_flops_executed([(r, r)], 1) * 6 == bench.ns_flops([(r, r)], 1) * 4.25
-    assert bench.ns_flops_executed([(256, 512)], 5) == bench.ns_flops([(256, 512)], 5)
-    assert bench.ns_flops_executed([(256, 512)], 5, "fp32") == 3 * bench.ns_flops([(256, 512)], 5)
-    wl, shapes = bench.workload_desc("qwen3_1.7b")
-    assert round(bench.ns_flops_executed(shapes, wl.ns_steps) / 1e13, 2) == 5.04
