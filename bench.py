@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3_1.7b")
     ap.add_argument("--ns-precision", default="fp16", choices=["fp16", "bf16", "fp32"])
+    ap.add_argument("--groups", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="matrix groups of the step (0: the library's automatic choice)")
     ap.add_argument("--ns-form", default="auto", choices=["auto", "y", "gram"],
                     help="Newton-Schulz evaluation: Gram-space runs where they save FLOPs (auto), "
                          "Y-space everywhere, or Gram-space wherever fp16 allows")
@@ -241,6 +243,7 @@ def bench_config(args, wl, shapes, world):
     """The workload description both arms report."""
     return {"workload": args.workload, "matrices": len(shapes), "params": sum(a * b for a, b in shapes),
             "ns_steps": wl.ns_steps, "ns_precision": args.ns_precision, "ns_form": args.ns_form,
+            "groups": args.groups,
             "state": "fp32 W, M, G",
             "lr": "workload schedule", "l2": "inputs larger than L2 (no flush)",
             "parallelism": f"{world} independent replica(s)"}
@@ -470,7 +473,7 @@ def run_ours(args):
     M = [torch.zeros_like(w) for w in W]
     G = [torch.randn(s, generator=gen, device=dev) * 1e-3 for s in shapes]
     opt = MuonH(W, M, beta=wl.beta, nesterov=wl.nesterov, ns_steps=wl.ns_steps, ns_coeffs=wl.ns_coeffs,
-                ns_precision=args.ns_precision, ns_form=args.ns_form)
+                ns_precision=args.ns_precision, ns_form=args.ns_form, groups=args.groups)
     lrs = wl.lrs
     stream = torch.cuda.current_stream()
 

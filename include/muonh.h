@@ -115,13 +115,16 @@ typedef struct {
 
 /* Context-wide settings.
  *   groups  0: automatic.  A set of at least 16M elements on the 16-bit path
- *              then runs as two matrix groups, whose elementwise kernels
- *              overlap the other group's Newton-Schulz GEMMs on an internal
- *              stream.
+ *              then runs as two matrix groups of equal Newton-Schulz work,
+ *              whose elementwise kernels overlap the other group's GEMMs on
+ *              an internal stream.
  *           1: one group.  Every kernel runs on the caller's stream, one
  *              after another; the context creates no stream of its own.
+ *           2, 3: that many groups on the 16-bit path, whatever the size
+ *              (three groups take a quarter, a half and a quarter of the
+ *              work, so the two phases no GEMM hides are short).
  *           Other values are rejected (MUONH_ERR_INVALID_ARG).  The results
- *           are the same bit for bit either way.
+ *           are the same bit for bit whatever the grouping.
  *   ns_form  how the Newton-Schulz iteration is evaluated (MUONH_NS_FORM_*).
  *           Y-space: every iteration forms A = Y Y^T, B' = a I + b A + c A A
  *           and Y <- B' Y (three products, two of them over the r x c Y).
@@ -142,7 +145,7 @@ enum {
 typedef struct {
   int32_t ns_precision;   /* MUONH_NS_FP16 / _BF16 / _FP32                  */
   float eps;              /* Newton-Schulz input: X/(||X||_F + eps), >= 0    */
-  int32_t groups;         /* 0 = automatic, 1 = a single group              */
+  int32_t groups;         /* 0 = automatic, 1 = a single group, 2 or 3      */
   int32_t ns_form;        /* MUONH_NS_FORM_*                                */
 } muonh_config;
 

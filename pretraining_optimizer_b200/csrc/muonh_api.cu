@@ -58,7 +58,8 @@ constexpr int kRing = 4;
 // whose elementwise phases overlap the other groups' Newton-Schulz GEMMs;
 // below it the overlap cannot pay for the extra launches.
 constexpr int64_t kTwoGroupMinElems = int64_t(1) << 24;
-constexpr int kGroups = 2;
+constexpr int kGroups = 2;      // the automatic choice
+constexpr int kMaxGroups = 3;
 // Tiles per block of an elementwise launch that overlaps Newton-Schulz GEMMs:
 // short-lived blocks leave the SMs' resources to the GEMMs' blocks, which the
 // scheduler places first (they run on the highest-priority stream).
@@ -412,8 +413,8 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   if (cfg->ns_precision < 0 || cfg->ns_precision > 2)
     return fail(MUONH_ERR_INVALID_ARG, "ns_precision %d is not FP16, BF16 or FP32", cfg->ns_precision);
   if (!(cfg->eps >= 0.f) || !std::isfinite(cfg->eps)) return fail(MUONH_ERR_INVALID_ARG, "eps must be finite and >= 0");
-  if (cfg->groups < 0 || cfg->groups > 1)
-    return fail(MUONH_ERR_INVALID_ARG, "groups %d is not 0 (automatic) or 1 (one group)", cfg->groups);
+  if (cfg->groups < 0 || cfg->groups > kMaxGroups)
+    return fail(MUONH_ERR_INVALID_ARG, "groups %d is not 0 (automatic), 1, 2 or 3", cfg->groups);
   if (cfg->ns_form < MUONH_NS_FORM_AUTO || cfg->ns_form > MUONH_NS_FORM_GRAM)
     return fail(MUONH_ERR_INVALID_ARG, "ns_form %d is not MUONH_NS_FORM_AUTO, _Y or _GRAM", cfg->ns_form);
   for (int32_t i = 0; i < n; ++i) {
@@ -453,7 +454,8 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   ctx->sm_count = prop.multiProcessorCount;
   for (int k = 0; k < 4; ++k) ctx->ew_warp_grid[k] = ctx->sm_count * ew_warp_blocks_per_sm(k);
   ctx->pairs = cfg->ns_precision != P_FP32;
-  const bool single_group = cfg->groups == 1;
+  // matrix groups: 1, the automatic 2 for a large enough set, or as asked
+  const int want_groups = cfg->groups == 0 ? kGroups : cfg->groups;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ctx->last_stream = s;
 
@@ -552,8 +554,8 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       ctx->n_ns_slots += md.ns_slots;
     }
   }
-  // ---- matrix groups: with the CTA-pair path and enough elements, split
-  // the matrices into two index ranges of about equal Newton-Schulz work
+  // ---- matrix groups: with the CTA-pair path and enough elements (or when
+  // asked), split the matrices into index ranges of Newton-Schulz work
   {
     std::vector<double> work(n);
     double total = 0.0;
@@ -570,15 +572,22 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       elems += md.rows * md.cols;
     }
     // group g ends after the first matrix at which the running work reaches
-    // (g + 1) / kGroups of the total; every group keeps at least one matrix
+    // the group's share of the total: halves for two groups; for three, a
+    // quarter, a half and a quarter, so that the two exposed phases (the
+    // first group's momentum pass, the last group's projection) are short
+    // while the middle group's elementwise work hides under the GEMMs of
+    // its neighbours.  Every group keeps at least one matrix.
     std::vector<int32_t> bounds{0};
-    if (ctx->pairs && !single_group && n >= kGroups && elems >= kTwoGroupMinElems && total > 0.0) {
+    const int G = want_groups;
+    const bool big = cfg->groups > 1 || elems >= kTwoGroupMinElems;
+    if (ctx->pairs && G > 1 && n >= G && big && total > 0.0) {
+      const double ends2[2] = {0.5, 1.0}, ends3[3] = {0.25, 0.75, 1.0};
+      const double* ends = G == 2 ? ends2 : ends3;
       double acc = 0.0;
-      for (int32_t i = 0; i < n && static_cast<int>(bounds.size()) < kGroups; ++i) {
+      for (int32_t i = 0; i < n && static_cast<int>(bounds.size()) < G; ++i) {
         acc += work[i];
         const int g = static_cast<int>(bounds.size()) - 1;
-        if (acc >= total * (g + 1) / kGroups && i + 1 > bounds.back() && n - (i + 1) >= kGroups - g - 1)
-          bounds.push_back(i + 1);
+        if (acc >= total * ends[g] && i + 1 > bounds.back() && n - (i + 1) >= G - g - 1) bounds.push_back(i + 1);
       }
     }
     bounds.push_back(n);
@@ -706,7 +715,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part_ns),
                 std::max<int64_t>(1, 2 * ctx->n_ns_slots) * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_wmaps), n * sizeof(CUtensorMap)) != cudaSuccess ||
-      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), (1 + kGroups) * sizeof(int)) != cudaSuccess)   // err, any_rewrite[]
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_err), (1 + kMaxGroups) * sizeof(int)) != cudaSuccess)   // err, any_rewrite[]
     return fail(MUONH_ERR_OOM, "allocation of the device tables failed");
 
   std::vector<ClassDev> cdev;
@@ -734,7 +743,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   CUDA_TRY(cudaMemcpyAsync(ctx->d_classes, cdev.data(), cdev.size() * sizeof(ClassDev), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_et_mat, et_mat.data(), n_et * sizeof(int32_t), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_scal, scal.data(), n * sizeof(MatScal), cudaMemcpyHostToDevice, s));
-  CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, (1 + kGroups) * sizeof(int), s));
+  CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, (1 + kMaxGroups) * sizeof(int), s));
 
   // ---- Newton-Schulz tile lists: per group, one pair (upper-triangle tiles,
   // APPLY tiles) per iteration of the Y-space form (shared when equal), and

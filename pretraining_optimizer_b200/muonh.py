@@ -224,7 +224,7 @@ class MuonH:
     update_scale take one value for every matrix or a per-matrix sequence.
     groups=1 keeps every kernel of the step on the caller's stream (no
     overlap of elementwise and Newton-Schulz work); 0 lets the library split
-    a large set into two overlapping groups.  ns_form picks the evaluation
+    a large set into two overlapping groups; 2 or 3 asks for that many.  ns_form picks the evaluation
     of the Newton-Schulz iteration: "auto" (Gram-space runs where they save
     FLOPs), "y" (Y-space for every matrix) or "gram" (Gram-space wherever
     the fp16 path can run it)."""

@@ -56,7 +56,7 @@ def test_status_strings_and_argument_checks_without_a_gpu():
     cfg_bad = B.Config(7, 1e-7)
     d[0] = B.MatrixDesc(0x1000, 0x2000, 4, 8, 8, 0.0, 0.95, 1, 5, 3.4445, -4.775, 2.0315)
     assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(cfg_bad), None) == 1
-    assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(B.Config(0, 1e-7, 2)), None) == 1   # groups
+    assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(B.Config(0, 1e-7, 4)), None) == 1   # groups
     assert b"groups" in lib.muonh_last_error()
     assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(B.Config(0, 1e-7, 0, 3)), None) == 1   # ns_form
     assert b"ns_form" in lib.muonh_last_error()

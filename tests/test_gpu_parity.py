@@ -305,17 +305,18 @@ def test_two_group_schedule_with_general_path_matrices(prec, ns_tol, w_tol):
         assert st["flags"] == 0 and abs(st["post_norm"] - R0) <= NORM_TOL * R0 and abs(st["elr"] - lr) <= NORM_TOL * lr
 
 
-def test_single_group_gives_the_same_bits():
+def test_grouping_gives_the_same_bits():
     """groups=1 runs every kernel on the caller's stream, one after another;
-    a set large enough for the two-group overlap gives the same W, M and
-    stats bit for bit either way (fixed partial-sum slots, fixed order)."""
+    two and three groups overlap elementwise and GEMM work: a set large
+    enough for the overlap gives the same W, M and stats bit for bit
+    (fixed partial-sum slots, fixed order) whatever the grouping."""
     import torch
     from pretraining_optimizer_b200 import MuonH
     dev = torch.device("cuda:0")
     shapes = [(4096, 4096), (640, 384), (1000, 300), (1024, 2048)]
     W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
     runs = []
-    for groups in (0, 1):
+    for groups in (0, 1, 3):
         W = [torch.from_numpy(w).to(dev) for w in W0]
         M = [torch.zeros_like(w) for w in W]
         opt = MuonH(W, M, groups=groups)
@@ -326,11 +327,12 @@ def test_single_group_gives_the_same_bits():
         st = opt.stats()
         opt.close()
         runs.append(([w.cpu().numpy() for w in W], [m.cpu().numpy() for m in M], st, launches))
-    (Wa, Ma, sa, la), (Wb, Mb, sb, lb) = runs
-    assert la > lb          # the two-group schedule really ran in the automatic mode
-    for i in range(len(shapes)):
-        assert np.array_equal(Wa[i], Wb[i]) and np.array_equal(Ma[i], Mb[i]), i
-        assert sa[i] == sb[i], i
+    (Wa, Ma, sa, la), (Wb, Mb, sb, lb), (Wc, Mc, sc, lc) = runs
+    assert lc > la > lb     # three, two and one groups really ran
+    for W_, M_, s_ in ((Wb, Mb, sb), (Wc, Mc, sc)):
+        for i in range(len(shapes)):
+            assert np.array_equal(Wa[i], W_[i]) and np.array_equal(Ma[i], M_[i]), i
+            assert sa[i] == s_[i], i
 
 
 @pytest.mark.parametrize("prec", ["fp16", "bf16"])
