@@ -452,12 +452,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 // the leader's commits arrive on the matching barriers of both CTAs.  Each
 // CTA drains its own TMEM (its 128 rows) in the epilogue.
 //
-// Symmetric results (A, C, B') are computed on the 256 x 256 tiles of the
-// upper block triangle; the epilogue of an off-diagonal tile also writes its
-// transpose (a warp-level 32 x 32 transpose per store box), so SQUARE and
-// APPLY read A, C and B' as K-major operands.  (Reading a lower block
-// through its stored transpose as an MN-major operand instead ran SQUARE
-// about 30% slower on B200.)
+// Symmetric results (A, B', the Gram-space factors) are computed on the
+// 256 x 256 tiles of the upper block triangle; the epilogue of an
+// off-diagonal tile also writes its transpose (stmatrix.trans from the
+// accumulator fragments into a second store box), so SQUARE, SYMPROD and
+// APPLY read them as K-major operands.  (Reading a lower block through its
+// stored transpose as an MN-major operand instead ran SQUARE about 30%
+// slower on B200.)
 template <int PREC, int MODE>
 struct PairCfg {
   // the last APPLY gives staging space to the fp32 W boxes of its <W, O> partials
@@ -472,17 +473,12 @@ struct PairCfg {
   // Epilogue warps: one per TMEM lane quarter
   static constexpr int kEpiWarps = 4;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
-  // per-epilogue-warp 32 x 32 16-bit scratch for the mirrored copies (rows
-  // padded to 80 bytes: conflict-free 16-byte stores and 2-byte column reads)
-  static constexpr int kMirrorStride = 80;
-  static constexpr int kMirrorOffset = kBarOffset + 256;
-  static constexpr int kMirrorBytes = kEpiWarps * 32 * kMirrorStride;
   // Epilogue output staging: each epilogue warp owns kWarpBufs boxes of
   // 32 rows x 32 columns (16-bit, 64-byte swizzle) that it writes to global
   // memory with its own TMA stores
   static constexpr int kWarpBox = 32 * 32 * 2;
   static constexpr int kWarpBufs = kLast ? 2 : 4;
-  static constexpr int kStoreOffset = (kMirrorOffset + kMirrorBytes + 1023) / 1024 * 1024;
+  static constexpr int kStoreOffset = (kBarOffset + 256 + 1023) / 1024 * 1024;
   // Last APPLY: kWBufs fp32 W boxes (128 rows x 32 columns, or 32 x 128 for
   // a tall W) filled kWBufs chunks ahead, for the <W, O> partials
   static constexpr int kWBox = 128 * 32 * 4;
@@ -504,15 +500,17 @@ template <int kBufs>
 struct WarpStager {
   uint8_t* base;
   int count;   // boxes handed out so far
-  __device__ __forceinline__ void put(const CUtensorMap* map, int lane, const uint4 (&row)[4], int x, int y,
-                                      int z) {
+  // The next buffer, once the store issued from it kBufs puts ago has read it.
+  __device__ __forceinline__ uint8_t* acquire(int lane) {
     uint8_t* buf = base + (count % kBufs) * (32 * 32 * 2);
     if (count >= kBufs) {
       if (lane == 0) bulk_wait_read<kBufs - 1>();
       __syncwarp();
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + store_box_offset(lane, q)) = row[q];
+    return buf;
+  }
+  // Store the box the warp wrote into the acquired buffer.
+  __device__ __forceinline__ void commit(uint8_t* buf, const CUtensorMap* map, int lane, int x, int y, int z) {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -521,20 +519,34 @@ struct WarpStager {
     }
     ++count;
   }
+  __device__ __forceinline__ void put(const CUtensorMap* map, int lane, const uint4 (&row)[4], int x, int y,
+                                      int z) {
+    uint8_t* buf = acquire(lane);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(buf + store_box_offset(lane, q)) = row[q];
+    commit(buf, map, lane, x, y, z);
+  }
 };
 
-// Transpose a warp's 32 x 32 block of 16-bit values through its padded
-// shared-memory scratch: lane j passes row j, receives column j.
-template <int PREC, int kStride>
-__device__ __forceinline__ void warp_transpose32(uint8_t* scratch, int lane, const uint4 (&row)[4], uint4 (&col)[4]) {
-  using T16 = typename Store16<PREC>::T;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(scratch + lane * kStride + q * 16) = row[q];
-  __syncwarp();
-  T16* cv = reinterpret_cast<T16*>(col);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) cv[i] = *reinterpret_cast<const T16*>(scratch + i * kStride + lane * 2);
-  __syncwarp();
+// Two fp32 values to a packed pair of 16-bit values, the first in the low half.
+template <int PREC>
+__device__ __forceinline__ uint32_t pack_pair(float lo, float hi) {
+  if (PREC == P_BF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+template <int PREC>
+__device__ __forceinline__ float unpack_lo(uint32_t u) {
+  using T = typename Store16<PREC>::T;
+  return Store16<PREC>::back(*reinterpret_cast<const T*>(&u));
+}
+template <int PREC>
+__device__ __forceinline__ float unpack_hi(uint32_t u) {
+  using T = typename Store16<PREC>::T;
+  return Store16<PREC>::back(reinterpret_cast<const T*>(&u)[1]);
 }
 
 template <int PREC>
@@ -734,16 +746,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         const int r0 = td.bi * kPairM + static_cast<int>(rank) * 128;
         for (int b = 0; b < C::kWBufs; ++b) w_issue(td, md, cd, r0, b, b);   // first chunks while the MMAs run
       }
-      // SQUARE reads A[row][bj block] (written by GRAM, read-only here) for its
-      // b A term straight from L2, one 32-column chunk ahead
-      const uint16_t* arow = nullptr;
-      uint4 a_next[4];
+      // SQUARE reads A (written by GRAM, read-only here) for its b A term
+      // straight from L2, one 32-column chunk ahead, in the accumulator
+      // fragment layout of the epilogue: rows lane/4 + 8p + 16h of this
+      // warp's 32, columns 8k + 2 (lane % 4) (+1) of the chunk
+      const uint16_t* abase = nullptr;
+      uint32_t a_next[16];
       if (C::kSquare) {
-        const int row_a = td.bi * kPairM + static_cast<int>(rank) * 128 + lrow;
-        arow = static_cast<const uint16_t*>(cd.a[0]) + md.z * cd.a_stride + static_cast<int64_t>(row_a) * cd.r_pad +
-               td.bj * kBN;
+        const int frow = td.bi * kPairM + static_cast<int>(rank) * 128 + quarter * 32 + (lane >> 2);
+        abase = static_cast<const uint16_t*>(cd.a[0]) + md.z * cd.a_stride + static_cast<int64_t>(frow) * cd.r_pad +
+                td.bj * kBN + 2 * (lane & 3);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) a_next[q] = __ldg(reinterpret_cast<const uint4*>(arow + ch0 * 32) + q);
+        for (int hp = 0; hp < 4; ++hp)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            a_next[4 * hp + k] = __ldg(reinterpret_cast<const uint32_t*>(abase + static_cast<int64_t>(8 * hp) * cd.r_pad +
+                                                                         ch0 * 32 + 8 * k));
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
       tc_fence_after();
@@ -752,83 +770,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
       // iteration 0 reads X at the momentum kernel's scale: kappa corrects it
       const float kap = (MODE == M_GRAM && p.iter == 0) ? p.scal[td.mat].kappa : 1.f;
-      uint8_t* mirror_buf = smem + C::kMirrorOffset + epi * 32 * C::kMirrorStride;
       const bool mirror = td.bj > td.bi;   // off-diagonal block: also store its transpose
-      if (MODE == M_GRAM || MODE == M_SYMPROD) {
-        // GRAM: stored A = 2^ea Y Y^T from the stored Y (2^ex Y);
-        // SYMPROD: stored out = 2^e_out L R from the stored L and R
-        const float sa = MODE == M_GRAM
-                             ? kap * kap * exp2f(static_cast<float>(md.ea - 2 * md.ex))
-                             : exp2f(static_cast<float>(rr_exp(md, p.out_kind) - rr_exp(md, p.lhs_kind) -
-                                                        rr_exp(md, p.rhs_kind)));
+      if (MODE == M_GRAM || MODE == M_SYMPROD || MODE == M_SQUARE) {
+        // Symmetric outputs, drained in the accumulator fragment layout
+        // (tcgen05.ld.16x256b): the warp writes its 32 x 32 box with
+        // stmatrix and, for an off-diagonal tile, the mirrored box with
+        // stmatrix.trans, so the transpose costs no extra shared-memory pass.
+        //   GRAM:    stored A   = 2^ea Y Y^T from the stored Y (2^ex Y)
+        //   SYMPROD: stored out = 2^e_out L R from the stored L and R
+        //   SQUARE:  stored B'  = 2^eb (c A A + b A + a I) from the stored A
+        float sa = 1.f, s2 = 0.f, s1 = 0.f, diag = 0.f;
+        if (MODE == M_GRAM) sa = kap * kap * exp2f(static_cast<float>(md.ea - 2 * md.ex));
+        if (MODE == M_SYMPROD)
+          sa = exp2f(static_cast<float>(rr_exp(md, p.out_kind) - rr_exp(md, p.lhs_kind) - rr_exp(md, p.rhs_kind)));
+        if (MODE == M_SQUARE) {
+          s2 = md.c_coef * exp2f(static_cast<float>(md.eb - 2 * md.ea));
+          s1 = md.b * exp2f(static_cast<float>(md.eb - md.ea));
+          diag = md.a * exp2f(static_cast<float>(md.eb));
+        }
         const CUtensorMap* omap = p.tmaps + cd.tm_base + (MODE == M_GRAM ? TM_A_ST : tm_rr_st(p.out));
+        const int grow = row0 + wrow0_off;            // this warp's first row
+        const int frow = lane >> 2, fcol = 2 * (lane & 3);
         for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
           const int col0 = td.bj * kBN + ch * 32;
-          float v[32];
-          tmem_ld32(taddr + ch * 32, v);
+          uint32_t u[2][16];
+          tmem_ld16x32_nowait(taddr + ch * 32, u[0]);                       // rows 0..15 of the warp's 32
+          tmem_ld16x32_nowait(taddr + (16u << 16) + ch * 32, u[1]);         // rows 16..31
+          tmem_wait_ld();
           if (ch + kChStep >= kBN / 32) {   // this warp's last chunk of the tile
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader[acc]);   // accumulator drained
           }
+          uint32_t a_cur[16];
+          if (MODE == M_SQUARE) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= sa;
-          uint4 pv[4];
-          pack32<PREC>(v, pv);
-          stager.put(omap, lane, pv, col0, row0 + wrow0_off, md.z);
-          if (mirror) {
-            // the product is symmetric: out[col][row] = out[row][col]
-            uint4 cv[4];
-            warp_transpose32<PREC, C::kMirrorStride>(mirror_buf, lane, pv, cv);
-            stager.put(omap, lane, cv, row0 + wrow0_off, col0, md.z);
-          }
-        }
-      } else if (MODE == M_SQUARE) {
-        // stored B' = 2^eb (c A A + b A + a I), from the product of the stored
-        // A (2^ea A) with itself and the stored A of this chunk (read from L2)
-        const float s2 = md.c_coef * exp2f(static_cast<float>(md.eb - 2 * md.ea));
-        const float s1 = md.b * exp2f(static_cast<float>(md.eb - md.ea));
-        const float diag = md.a * exp2f(static_cast<float>(md.eb));
-        const CUtensorMap* omap = p.tmaps + cd.tm_base + tm_rr_st(p.out);
-        using T16 = typename Store16<PREC>::T;
-        for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
-          const int col0 = td.bj * kBN + ch * 32;
-          float v[32];
-          tmem_ld32(taddr + ch * 32, v);
-          if (ch + kChStep >= kBN / 32) {   // this warp's last chunk of the tile
-            tc_fence_before();
-            mbar_arrive_cluster(tempty_leader[acc]);
-          }
-          uint4 a_cur[4];
+            for (int q = 0; q < 16; ++q) a_cur[q] = a_next[q];
+            if (ch + kChStep < kBN / 32) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) a_cur[q] = a_next[q];
-          if (ch + kChStep < kBN / 32) {
+              for (int hp = 0; hp < 4; ++hp)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) a_next[q] = __ldg(reinterpret_cast<const uint4*>(arow + (ch + kChStep) * 32) + q);
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const T16* h = reinterpret_cast<const T16*>(&a_cur[q]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[8 * q + e] = fmaf(s2, v[8 * q + e], s1 * Store16<PREC>::back(h[e]));
-          }
-          const int dj = row - col0;
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (j == dj) {
-              v[j] += diag;
-              // bf16 keeps 8 significant bits of the diagonal (near a = 3.44
-              // in early iterations): APPLY adds back the rounding residual
-              if (PREC == P_BF16)
-                cd.bdiag[static_cast<int64_t>(md.z) * cd.r_pad + row] = v[j] - Store16<PREC>::back(Store16<PREC>::cvt(v[j]));
+                for (int k = 0; k < 4; ++k)
+                  a_next[4 * hp + k] = __ldg(reinterpret_cast<const uint32_t*>(
+                      abase + static_cast<int64_t>(8 * hp) * cd.r_pad + (ch + kChStep) * 32 + 8 * k));
             }
-          uint4 packed[4];
-          pack32<PREC>(v, packed);
-          stager.put(omap, lane, packed, col0, row0 + wrow0_off, md.z);
+          }
+          uint32_t w[2][2][4];   // [h][p][k]: rows 16h + 8p + lane/4, columns 8k + 2 (lane % 4) (+1)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                float v0 = __uint_as_float(u[h][4 * k + 2 * pp]), v1 = __uint_as_float(u[h][4 * k + 2 * pp + 1]);
+                if (MODE == M_SQUARE) {
+                  const uint32_t av = a_cur[4 * (2 * h + pp) + k];
+                  v0 = fmaf(s2, v0, s1 * unpack_lo<PREC>(av));
+                  v1 = fmaf(s2, v1, s1 * unpack_hi<PREC>(av));
+                  const int rg = grow + 16 * h + 8 * pp + frow, cg = col0 + 8 * k + fcol;
+                  if (rg == cg || rg == cg + 1) {
+                    float& vd = rg == cg ? v0 : v1;
+                    vd += diag;
+                    // bf16 keeps 8 significant bits of the diagonal (near a = 3.44
+                    // in early iterations): APPLY adds back the rounding residual
+                    if (PREC == P_BF16)
+                      cd.bdiag[static_cast<int64_t>(md.z) * cd.r_pad + rg] =
+                          vd - Store16<PREC>::back(Store16<PREC>::cvt(vd));
+                  }
+                } else {
+                  v0 *= sa;
+                  v1 *= sa;
+                }
+                w[h][pp][k] = pack_pair<PREC>(v0, v1);
+              }
+          // direct box: matrix (h, p, k) is box rows 16h + 8p .. +7, 16-byte piece k
+          uint8_t* buf = stager.acquire(lane);
+          const uint32_t sb = smem_u32(buf);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp)
+              stmatrix_x4(sb + store_box_offset(16 * h + 8 * pp + (lane & 7), lane >> 3), w[h][pp][0], w[h][pp][1],
+                          w[h][pp][2], w[h][pp][3]);
+          stager.commit(buf, omap, lane, col0, grow, md.z);
           if (mirror) {
-            // B'[col0 + lane][row0 + 32 quarter + j] = B'[row0 + 32 quarter + j][col0 + lane]
-            uint4 cv[4];
-            warp_transpose32<PREC, C::kMirrorStride>(mirror_buf, lane, packed, cv);
-            stager.put(omap, lane, cv, row0 + wrow0_off, col0, md.z);
+            // out[col][row] = out[row][col]: matrix (h, p, k) transposed is
+            // mirror-box rows 8k .. 8k+7, piece 2h + p; lane l addresses row l
+            uint8_t* mb = stager.acquire(lane);
+            const uint32_t smb = smem_u32(mb);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int pp = 0; pp < 2; ++pp)
+                stmatrix_x4_trans(smb + store_box_offset(lane, 2 * h + pp), w[h][pp][0], w[h][pp][1], w[h][pp][2],
+                                  w[h][pp][3]);
+            stager.commit(mb, omap, lane, grow, col0, md.z);
           }
         }
         if (werr) break;
