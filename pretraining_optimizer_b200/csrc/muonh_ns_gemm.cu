@@ -464,6 +464,8 @@ struct PairCfg {
   // the last APPLY gives staging space to the fp32 W boxes of its <W, O> partials
   static constexpr bool kLast = MODE == M_APPLY_LAST;
   static constexpr bool kSquare = MODE == M_SQUARE;
+  // operand ring of 32 KB stages (a sixth stage, where shared memory allows
+  // it, measured slower: SQUARE lost 4%)
   static constexpr int kStages = 5;
   static constexpr int kWBufs = 2;
   static constexpr int kABytes = 128 * kBK * 2;                 // 16 KB: this CTA's 128 rows
@@ -484,6 +486,8 @@ struct PairCfg {
   static constexpr int kWBox = 128 * 32 * 4;
   static constexpr int kWOffset = kStoreOffset + kEpiWarps * kWarpBufs * kWarpBox;
   static constexpr int kSmem = kWOffset + (kLast ? kWBufs * kWBox : 0) + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory of the pair kernel exceeds 227 KB");
+  static_assert(2 * kStages + 2 + 2 + 1 + 4 + 4 <= 31, "mbarriers exceed their 256-byte region");
 };
 
 // Row `r` (0..31) of a 32 x 32 16-bit box, 16-byte piece q, in the 64-byte
