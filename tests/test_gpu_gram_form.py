@@ -125,3 +125,48 @@ def test_executed_flops_of_each_form():
             exp_apply += (r // 256) * (c // 256) * tile * r
     assert (gf["ns_gram"], gf["ns_square"], gf["ns_apply"], gf["ns_product"]) == (exp_gram, exp_sq, exp_apply,
                                                                                    exp_prod)
+
+
+@pytest.mark.parametrize("ns_steps", [1, 2, 3, 4, 6, 7])
+def test_gram_form_run_lengths(ns_steps):
+    """Other step counts split into other runs ((1), (2), (3), (2, 2),
+    (3, 3), (3, 2, 2)); each matches the oracle, and the run structure
+    shows in the executed FLOPs: one Y Y^T and one Q Y per run."""
+    shape = (256, 768)
+    W0 = [synth.initial_weight(0, *shape)]
+    grad = lambda t, i: synth.gaussian_gradient(t, 0, *shape)
+    g = run_gpu(W0, grad, [0.01, 0.01], ns_steps=ns_steps, keep_updates=(1,), ns_form="gram")
+    o = run_oracle(W0, grad, [0.01, 0.01], ns_steps=ns_steps, keep_updates=(1,))
+    assert rel_fro(g["O"][1][0], o["O"][1][0]) <= FP16_NS_TOL, (ns_steps, rel_fro(g["O"][1][0], o["O"][1][0]))
+    assert np.linalg.norm(g["W"][0] - o["W"][0]) / o["R"][0] <= 1e-4
+    runs = -(-ns_steps // 3)
+    tile = 2 * 256 * 256
+    assert g["flops"]["ns_gram"] == runs * tile * 768            # one upper tile, K = 768
+    assert g["flops"]["ns_apply"] == runs * 3 * tile * 256       # three tiles, K = 256
+    assert g["flops"]["ns_square"] == ns_steps * tile * 256
+
+
+def test_gram_form_beside_y_space_matrices_of_the_same_class():
+    """Matrices with fewer Newton-Schulz steps than the context's largest
+    stay in the Y-space form, in the same shape class as Gram-form ones."""
+    shapes = [(256, 768)] * 3
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    steps = [5, 3, 5]
+    g = run_gpu(W0, grad, [0.01] * 3, ns_steps=steps, keep_updates=(2,), ns_form="gram")
+    for i in range(3):
+        o = run_oracle([W0[i]], lambda t, _: grad(t, i), [0.01] * 3, ns_steps=steps[i], keep_updates=(2,))
+        assert rel_fro(g["O"][2][i], o["O"][2][0]) <= FP16_NS_TOL, i
+        assert np.linalg.norm(g["W"][i] - o["W"][0]) / o["R"][0] <= 1e-4, i
+
+
+def test_gram_form_with_the_convergent_quintic():
+    """(15/8, -10/8, 3/8) has other bounds on the stored Q (its p(0) is 15/8)
+    and converges: 9 steps in the Gram form reach the oracle's output."""
+    coeffs = (15 / 8, -10 / 8, 3 / 8)
+    shape = (256, 768)
+    W0 = [synth.initial_weight(0, *shape)]
+    grad = lambda t, i: synth.gaussian_gradient(t, 0, *shape)
+    g = run_gpu(W0, grad, [0.01], ns_steps=9, coeffs=coeffs, keep_updates=(0,), ns_form="gram")
+    o = run_oracle(W0, grad, [0.01], ns_steps=9, coeffs=coeffs, keep_updates=(0,))
+    assert rel_fro(g["O"][0][0], o["O"][0][0]) <= FP16_NS_TOL
