@@ -184,6 +184,28 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
 muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* grads,
                         muonh_stats* stats, void* stream);
 
+/* Per-matrix arguments of one step, in device memory, for muonh_step_device
+ * (16 bytes: the gradient pointer, the effective LR, 4 bytes of padding). */
+typedef struct {
+  const float* grad;   /* fp32 device gradient, laid out like the matrix's w */
+  float lr;            /* the matrix's effective LR (eta^H) for this step     */
+  float pad_;
+} muonh_step_args;
+
+/* muonh_step with its per-matrix arguments in device memory: `args` is a
+ * device array of n muonh_step_args, read by the step's kernels when they
+ * run.  The call enqueues kernel launches and, for a grouped step, event
+ * records and waits between `stream` and the context's internal stream;
+ * it copies nothing from the host and never synchronises.  It can
+ * therefore be captured in a CUDA graph, and every replay uses whatever
+ * `args` and the gradients hold when it runs.  The library cannot inspect
+ * device-resident arguments: every grad must be non-NULL, 16-byte aligned
+ * and laid out like its matrix's w, and every lr finite, as muonh_step
+ * checks on the host.  `args` itself must be 16-byte aligned
+ * (MUONH_ERR_ALIGNMENT otherwise).  Results are bit-identical to
+ * muonh_step with the same arguments. */
+muonh_status muonh_step_device(muonh_ctx* ctx, const muonh_step_args* args, muonh_stats* stats, void* stream);
+
 /* Copy the last step's per-matrix stats to host memory (n entries);
  * synchronises the stream of the last step. */
 muonh_status muonh_get_stats(muonh_ctx* ctx, muonh_stats* host_out);

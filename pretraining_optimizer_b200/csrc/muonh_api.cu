@@ -233,6 +233,7 @@ struct muonh_ctx {
   ClassDev* d_classes = nullptr;
   MatScal* d_scal = nullptr;
   MatStep* d_step = nullptr;
+  const MatStep* step_src = nullptr;   // per-step arguments the next launches read (d_step or the caller's)
   int32_t* d_et_mat = nullptr;
   float* d_part = nullptr;
   double* d_part64 = nullptr;
@@ -276,7 +277,7 @@ struct muonh_ctx {
     p.m_first = g < 0 ? 0 : groups[g].m_first;
     p.m_count = g < 0 ? n : groups[g].m_count;
     p.mats = d_mats;
-    p.step = d_step;
+    p.step = step_src ? step_src : d_step;
     p.scal = d_scal;
     p.classes = d_classes;
     p.et_mat = d_et_mat;
@@ -296,6 +297,8 @@ struct muonh_ctx {
 };
 
 namespace {
+
+muonh_status enqueue_step(muonh_ctx* ctx, const MatStep* step_args, muonh_stats* stats, cudaStream_t s);
 
 cudaError_t dev_alloc(muonh_ctx* ctx, void** p, size_t bytes) {
   cudaError_t e = cudaMalloc(p, bytes);
@@ -854,7 +857,24 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
   for (int32_t i = 0; i < ctx->n; ++i) ctx->h_step[slot][i] = MatStep{grads[i], lr[i], 0.f};
   CUDA_TRY(cudaMemcpyAsync(ctx->d_step, ctx->h_step[slot], ctx->n * sizeof(MatStep), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaEventRecord(ctx->ev[slot], s));
+  return enqueue_step(ctx, ctx->d_step, stats, s);
+}
 
+muonh_status muonh_step_device(muonh_ctx* ctx, const muonh_step_args* args, muonh_stats* stats, void* stream) {
+  g_last_error.clear();
+  if (!ctx || !args) return fail(MUONH_ERR_INVALID_ARG, "ctx or args is NULL");
+  if (reinterpret_cast<uintptr_t>(args) & 15) return fail(MUONH_ERR_ALIGNMENT, "args not 16-byte aligned");
+  return enqueue_step(ctx, reinterpret_cast<const MatStep*>(args), stats, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Every launch of one step, reading the per-matrix (gradient, lr) table from
+// device memory `step_args`: kernels and event record/waits only.
+muonh_status enqueue_step(muonh_ctx* ctx, const MatStep* step_args, muonh_stats* stats, cudaStream_t s) {
+  ctx->step_src = step_args;
   int launches = 0;
   const int grid = ctx->sm_count * 8;
   // elementwise grids: one resident wave, or short blocks when the launch
@@ -1044,6 +1064,10 @@ muonh_status muonh_step(muonh_ctx* ctx, const float* lr, const float* const* gra
   ++ctx->step_count;
   return MUONH_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 muonh_status muonh_get_stats(muonh_ctx* ctx, muonh_stats* host_out) {
   g_last_error.clear();

@@ -22,7 +22,7 @@ FLAG_DEGENERATE = 8
 FLAG_TIMEOUT = 16
 
 EXPORTED_SYMBOLS = (
-    "muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
+    "muonh_init", "muonh_step", "muonh_step_device", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
     "muonh_export_state", "muonh_import_state", "muonh_device_status", "muonh_last_launch_count",
     "muonh_enable_timing", "muonh_phase_times", "muonh_phase_flops", "muonh_momentum_norm_noalloc",
     "muonh_average",
@@ -85,6 +85,7 @@ def library() -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     lib.muonh_init.argtypes = [POINTER(c_void_p), POINTER(MatrixDesc), c_int32, POINTER(Config), c_void_p]
     lib.muonh_step.argtypes = [c_void_p, POINTER(c_float), POINTER(c_void_p), c_void_p, c_void_p]
+    lib.muonh_step_device.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p]
     lib.muonh_get_stats.argtypes = [c_void_p, POINTER(Stats)]
     lib.muonh_get_update.argtypes = [c_void_p, c_int32, c_void_p, c_int64, c_void_p]
     lib.muonh_get_radius.argtypes = [c_void_p, POINTER(c_float)]
@@ -107,7 +108,7 @@ def library() -> ctypes.CDLL:
     lib.muonh_status_string.restype = c_char_p
     lib.muonh_last_error.argtypes = []
     lib.muonh_last_error.restype = c_char_p
-    for name in ("muonh_init", "muonh_step", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
+    for name in ("muonh_init", "muonh_step", "muonh_step_device", "muonh_get_stats", "muonh_get_update", "muonh_get_radius",
                  "muonh_export_state", "muonh_import_state", "muonh_device_status",
                  "muonh_enable_timing", "muonh_phase_times", "muonh_phase_flops", "muonh_momentum_norm_noalloc",
                  "muonh_average", "muonh_adamw_step", "muonh_check_wait_timeout"):
@@ -294,6 +295,41 @@ class MuonH:
                 raise ValueError("stats must be a CUDA tensor of at least 24*n bytes")
             sp = stats.data_ptr()
         _check(self._lib.muonh_step(self._ctx, self._lr, self._g, sp, _stream_handle(stream)))
+
+    def step_args(self, grads, lr):
+        """A CUDA tensor holding the device argument table of muonh_step_device
+        (one 16-byte record per matrix: gradient pointer, lr) for these
+        gradients and lr (float or per-matrix sequence).  Its lr fields are
+        also reachable as `args.view(torch.float32)[2::4]`, so a captured
+        graph can be given a new schedule value in place."""
+        import torch
+        n = self.n
+        if len(grads) != n:
+            raise ValueError("one gradient per weight")
+        rec = torch.zeros((n, 2), dtype=torch.int64)
+        lrs = torch.empty(n, dtype=torch.float32)
+        for i, g in enumerate(grads):
+            gp, r, c, ld = _matrix_view(g, f"grads[{i}]")
+            if (r, c, ld) != self.shapes[i]:
+                raise ValueError(f"grads[{i}] must match weights[{i}] in shape and stride")
+            if gp % 16:
+                raise ValueError(f"grads[{i}] must be 16-byte aligned")
+            rec[i, 0] = gp
+            lrs[i] = lr if isinstance(lr, (int, float)) else lr[i]
+        rec.view(torch.float32)[:, 2] = lrs
+        return rec.to(self.weights[0].device)
+
+    def step_device(self, args, stats=None, stream=None) -> None:
+        """One step reading its arguments from the device table `args` (see
+        step_args); enqueues kernels only, so it can be captured in a CUDA graph."""
+        if not args.is_cuda or args.numel() * args.element_size() < 16 * self.n:
+            raise ValueError("args must be a CUDA tensor of at least 16*n bytes")
+        sp = None
+        if stats is not None:
+            if not stats.is_cuda or stats.numel() * stats.element_size() < 24 * self.n:
+                raise ValueError("stats must be a CUDA tensor of at least 24*n bytes")
+            sp = stats.data_ptr()
+        _check(self._lib.muonh_step_device(self._ctx, args.data_ptr(), sp, _stream_handle(stream)))
 
     def step_raw(self, grad_ptrs, lr_values, stats_ptr=None, stream_handle=0) -> None:
         """Lowest-overhead step: pointers and values already marshalled."""

@@ -31,6 +31,9 @@ def test_struct_layouts_match_the_header():
     assert ctypes.sizeof(B.MatrixDesc) == 80
     assert ctypes.sizeof(B.Config) == 16 and B.Config.groups.offset == 8 and B.Config.ns_form.offset == 12
     assert ctypes.sizeof(B.Stats) == 24
+    # muonh_step_args: a device pointer and an fp32 lr, padded to 16 bytes (the kernels' own table layout)
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    assert re.search(r"typedef struct \{\s*const float\* grad;\s*float lr;\s*float pad_;\s*\} muonh_step_args;", text)
     assert B.MatrixDesc.radius.offset == 40 and B.MatrixDesc.ns_c.offset == 64
     assert B.MatrixDesc.update_rule.offset == 68 and B.MatrixDesc.update_scale.offset == 76
 
@@ -61,6 +64,7 @@ def test_status_strings_and_argument_checks_without_a_gpu():
     assert lib.muonh_init(ctypes.byref(ctx), d, 1, ctypes.byref(B.Config(0, 1e-7, 0, 3)), None) == 1   # ns_form
     assert b"ns_form" in lib.muonh_last_error()
     assert lib.muonh_step(None, None, None, None, None) == 1
+    assert lib.muonh_step_device(None, None, None, None) == 1
 
 
 def _desc(**kw):

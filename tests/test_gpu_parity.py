@@ -132,6 +132,29 @@ def test_per_matrix_nesterov_and_beta():
         assert np.linalg.norm(W[i].cpu().numpy() - o["W"][0]) / o["R"][0] <= 1e-4, i
 
 
+@pytest.mark.parametrize("prec,form,margin", [("fp16", "y", 5e-3), ("fp16", "gram", 5e-3), ("bf16", "y", 1e-2)])
+def test_output_spectrum_lies_in_the_band_of_the_quintic(prec, form, margin):
+    """The iteration maps each singular value s of the normalised input to
+    p^5(s), p(s) = a s + b s^3 + c s^5: the singular values of the GPU's O
+    lie in the image of p^5 over the input's singular values (evaluated on a
+    fine grid), up to a 16-bit margin."""
+    shape = (192, 448)
+    W0 = [synth.initial_weight(0, *shape)]
+    grad = lambda t, i: synth.gaussian_gradient(t, 0, *shape)
+    g = run_gpu(W0, grad, [0.01], prec=prec, keep_updates=(0,), ns_form=form)
+    _, X = oracle.momentum_update(np.zeros(shape), grad(0, 0), 0.95, True)
+    s_in = np.linalg.svd(X / np.linalg.norm(X), compute_uv=False)
+    grid = np.linspace(s_in.min(), s_in.max(), 100001)
+    a, b, c = oracle.QUINTIC
+    img = grid
+    for _ in range(5):
+        img = a * img + b * img ** 3 + c * img ** 5
+    s_out = np.linalg.svd(g["O"][0][0].astype(np.float64), compute_uv=False)
+    assert s_out.min() >= img.min() - margin and s_out.max() <= img.max() + margin, (s_out.min(), s_out.max(),
+                                                                                     img.min(), img.max())
+    assert 0.6 < s_out.min() and s_out.max() < 1.25
+
+
 def test_edge_cases_zero_nan_and_zero_lr():
     shapes = [(128, 256)] * 4
     W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
