@@ -214,27 +214,29 @@ def test_bitwise_deterministic():
     assert np.array_equal(a["W"][0], b["W"][0]) and np.array_equal(a["O"][2][0], b["O"][2][0])
 
 
-def test_checkpoint_resume_is_bitwise():
-    """10 straight steps == 5 steps, export/import into a new context, 5 steps."""
+@pytest.mark.parametrize("ns_form", ["auto", "gram"])
+def test_checkpoint_resume_is_bitwise(ns_form):
+    """10 straight steps == 5 steps, export/import into a new context, 5 steps
+    (in the Y-space form and, forced, in the Gram-space form)."""
     import torch
     from pretraining_optimizer_b200 import MuonH
     wl, W0 = _single()
     grads = [[torch.from_numpy(wl.grad(t, 0)).cuda()] for t in range(10)]
     W = [torch.from_numpy(W0[0]).cuda()]
-    opt = MuonH(W)
+    opt = MuonH(W, ns_form=ns_form)
     for t in range(10):
         opt.step(grads[t], wl.lrs[t])
     straight = W[0].cpu().numpy()
     opt.close()
     W2 = [torch.from_numpy(W0[0]).cuda()]
     M2 = [torch.zeros_like(W2[0])]
-    opt = MuonH(W2, M2)
+    opt = MuonH(W2, M2, ns_form=ns_form)
     for t in range(5):
         opt.step(grads[t], wl.lrs[t])
     blob = opt.export_state()
     w_ck, m_ck = W2[0].clone(), M2[0].clone()
     opt.close()
-    opt = MuonH([w_ck], [m_ck], radii=[1.0])       # radius replaced by the imported state
+    opt = MuonH([w_ck], [m_ck], radii=[1.0], ns_form=ns_form)   # radius replaced by the imported state
     opt.import_state(blob)
     for t in range(5, 10):
         opt.step(grads[t], wl.lrs[t])
