@@ -11,6 +11,9 @@
  *   O     = NS(X)                                   quintic Newton-Schulz:
  *           Y = X/(||X||_F + eps) on the wide orientation, then ns_steps times
  *           A = Y Y^T;  B = b A + c A A;  Y = a Y + B Y
+ *           (evaluated as written, or in runs of up to three iterations on
+ *           r x r matrices, A <- A p(A)^2 and one Y <- Q Y per run, which is
+ *           the same O in exact arithmetic; see muonh_config.ns_form)
  *   u^    = O/||O||_F                               Sec. 3.3, Eq. (1)
  *   W~    = W_t - lr R u^                           Sec. 3.3, Eq. (1)
  *   W_t+1 = R W~/||W~||_F                           Sec. 3.3, Eq. (1)
