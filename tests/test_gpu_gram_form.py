@@ -170,3 +170,26 @@ def test_gram_form_with_the_convergent_quintic():
     g = run_gpu(W0, grad, [0.01], ns_steps=9, coeffs=coeffs, keep_updates=(0,), ns_form="gram")
     o = run_oracle(W0, grad, [0.01], ns_steps=9, coeffs=coeffs, keep_updates=(0,))
     assert rel_fro(g["O"][0][0], o["O"][0][0]) <= FP16_NS_TOL
+
+
+@pytest.mark.parametrize("rule", ["decoupled_wd", "elr_aligned"])
+def test_ordinary_muon_rules_on_the_gram_form(rule):
+    """Eq. (3) and Eq. (5) read O from the buffer the last Gram-space run
+    wrote: wide and tall matrices, 4 steps, weight decay 0.1, u = 0.2 O."""
+    shapes = [(256, 768), (768, 256)]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    lrs = [0.02, 0.015, 0.01, 0.005]
+    kw = dict(rule=rule, weight_decay=0.1, update_scale=0.2)
+    g = run_gpu(W0, grad, lrs, keep_updates=(3,), ns_form="gram", **kw)
+    o = run_oracle(W0, grad, lrs, keep_updates=(3,), **kw)
+    for i in range(2):
+        assert rel_fro(g["O"][3][i], o["O"][3][i]) <= FP16_NS_TOL, i
+        assert np.linalg.norm(g["W"][i] - o["W"][i]) / np.linalg.norm(o["W"][i]) <= 2e-4, i
+        for t, lr in enumerate(lrs):
+            gs, os_ = g["stats"][t][i], o["stats"][t][i]
+            assert gs["flags"] == 0
+            if rule == "elr_aligned":
+                assert abs(gs["elr"] - lr) <= NORM_TOL * lr, (t, i)
+            else:
+                assert abs(gs["elr"] - os_["elr"]) <= FP16_NS_TOL * os_["elr"], (t, i)
