@@ -11,8 +11,9 @@ Pins (tests/test_oracle.py, run with -m "not gpu") tie every function to
 something other than itself: the singular-value form of the Newton-Schulz
 polynomial checked with a library SVD, convergence to the polar factor with
 a convergent coefficient set, the closed-form hyperball invariants
-(||W_{t+1}||_F = R, effective LR = lr), a hand-solved two-element example,
-and the geometric-sum form of the momentum buffer.  oracle.aux (checkpoint
+(||W_{t+1}||_F = R, effective LR = lr), hand-solved two-element examples
+and hand-solved radii R = ||W_0||_F, and the geometric-sum form of the
+momentum buffer, also carried across the steps of run_steps.  oracle.aux (checkpoint
 averaging, AdamW) and oracle.emulate (16-bit storage emulation of the
 iteration) are pinned in tests/test_oracle_aux.py and tests/test_oracle.py.
 """
