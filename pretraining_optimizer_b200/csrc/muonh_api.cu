@@ -216,10 +216,19 @@ struct muonh_ctx {
   // The step runs in one or kGroups matrix groups (contiguous index ranges
   // of about equal Newton-Schulz work): the elementwise phases of one group
   // overlap the Newton-Schulz GEMMs of its neighbours.
+  // The matrices of a group in one Newton-Schulz form (0: Y-space, 1:
+  // Gram-space): their elementwise tiles [e_first, e_end) (a group stores
+  // the Y-space matrices' tiles first) and their indices in d_mlist.
+  struct Subset {
+    int64_t e_first = 0, e_end = 0;
+    int32_t m_off = 0, m_count = 0;
+    bool any_unfused = false, any_general = false, any_wt[2] = {false, false};
+  };
   struct Group {
     int32_t m_first = 0, m_count = 0;
     int64_t e_first = 0, e_end = 0;
     bool any_unfused = false, any_general = false, any_wt[2] = {false, false};
+    Subset sub[2];
     std::vector<TileList> gram_lists, apply_lists;   // per Newton-Schulz iteration (Y-space form)
     bool any_gram = false;                           // Gram-space form: its upper and APPLY tiles
     TileList gram_upper, gram_apply;
@@ -227,6 +236,8 @@ struct muonh_ctx {
   std::vector<Group> groups;
   cudaStream_t ns_stream = nullptr;   // highest-priority stream for the GEMMs of a grouped step
   std::vector<cudaEvent_t> gev;       // grouped step: per group, front done (2g) and GEMMs done (2g+1)
+  cudaEvent_t split_ev[2] = {};       // grouped step: first group's Y-space front done; last group's
+                                      // Gram-space GEMMs done
   std::vector<void*> allocs;
 
   MatDev* d_mats = nullptr;
@@ -235,6 +246,8 @@ struct muonh_ctx {
   MatStep* d_step = nullptr;
   const MatStep* step_src = nullptr;   // per-step arguments the next launches read (d_step or the caller's)
   int32_t* d_et_mat = nullptr;
+  int32_t* d_mlist = nullptr;      // per group: Y-space matrix indices, then Gram-space ones
+  std::vector<int32_t> h_mlist;
   float* d_part = nullptr;
   double* d_part64 = nullptr;
   float* d_part_ns = nullptr;      // fused last-APPLY partials
@@ -270,12 +283,22 @@ struct muonh_ctx {
   }
 
   // whole-context launch (init) or one group's launch (g >= 0)
-  EwParams ew(muonh_stats* stats_out, int g = -1) const {
+  // Elementwise launch parameters: the whole set (g < 0), group g, or the
+  // matrices of group g in one form (sub 0: Y-space, 1: Gram-space)
+  EwParams ew(muonh_stats* stats_out, int g = -1, int sub = -1) const {
     EwParams p{};
     p.e_first = g < 0 ? 0 : groups[g].e_first;
     p.e_end = g < 0 ? n_et : groups[g].e_end;
     p.m_first = g < 0 ? 0 : groups[g].m_first;
     p.m_count = g < 0 ? n : groups[g].m_count;
+    if (g >= 0 && sub >= 0) {
+      const Subset& su = groups[g].sub[sub];
+      p.e_first = su.e_first;
+      p.e_end = su.e_end;
+      p.m_first = su.m_off;
+      p.m_count = su.m_count;
+      p.mlist = d_mlist;
+    }
     p.mats = d_mats;
     p.step = step_src ? step_src : d_step;
     p.scal = d_scal;
@@ -314,6 +337,11 @@ void release(muonh_ctx* ctx) {
   for (cudaEvent_t e : ctx->gev)
     if (e) cudaEventDestroy(e);
   ctx->gev.clear();
+  for (cudaEvent_t& e : ctx->split_ev)
+    if (e) {
+      cudaEventDestroy(e);
+      e = nullptr;
+    }
   for (int i = 0; i < kRing; ++i) {
     if (ctx->h_step[i]) cudaFreeHost(ctx->h_step[i]);
     if (ctx->ev[i]) cudaEventDestroy(ctx->ev[i]);
@@ -594,20 +622,36 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       }
     }
     bounds.push_back(n);
+    // elementwise tiles, group by group: a group's Y-space matrices first,
+    // then its Gram-space ones, so that the tiles of each form are one range
+    int64_t e = 0;
     for (size_t g = 0; g + 1 < bounds.size(); ++g) {
       muonh_ctx::Group gr;
       gr.m_first = bounds[g];
       gr.m_count = bounds[g + 1] - bounds[g];
-      const MatDev& last = ctx->mats[bounds[g + 1] - 1];
-      gr.e_first = ctx->mats[bounds[g]].et_begin;
-      gr.e_end = last.et_begin + static_cast<int64_t>(last.et_rows) * last.et_cols;
-      for (int32_t i = bounds[g]; i < bounds[g + 1]; ++i) {
-        const MatDev& md = ctx->mats[i];
-        gr.any_unfused |= !md.fused_dots;
-        gr.any_general |= md.warp_tiled == 0;
-        if (md.warp_tiled) gr.any_wt[md.transposed ? 1 : 0] = true;
-        gr.any_gram |= md.gram != 0;
+      gr.e_first = e;
+      for (int f = 0; f < 2; ++f) {
+        muonh_ctx::Subset& su = gr.sub[f];
+        su.e_first = e;
+        su.m_off = static_cast<int32_t>(ctx->h_mlist.size());
+        for (int32_t i = bounds[g]; i < bounds[g + 1]; ++i) {
+          MatDev& md = ctx->mats[i];
+          if ((md.gram != 0) != (f == 1)) continue;
+          md.et_begin = e;
+          e += static_cast<int64_t>(md.et_rows) * md.et_cols;
+          ctx->h_mlist.push_back(i);
+          su.any_unfused |= !md.fused_dots;
+          su.any_general |= md.warp_tiled == 0;
+          if (md.warp_tiled) su.any_wt[md.transposed ? 1 : 0] = true;
+        }
+        su.e_end = e;
+        su.m_count = static_cast<int32_t>(ctx->h_mlist.size()) - su.m_off;
+        gr.any_unfused |= su.any_unfused;
+        gr.any_general |= su.any_general;
+        for (int k = 0; k < 2; ++k) gr.any_wt[k] |= su.any_wt[k];
       }
+      gr.e_end = e;
+      gr.any_gram = gr.sub[1].m_count > 0;
       ctx->groups.push_back(gr);
     }
     if (ctx->groups.size() > 1) {
@@ -615,7 +659,8 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
       CUDA_TRY(cudaStreamCreateWithPriority(&ctx->ns_stream, cudaStreamNonBlocking, greatest));
       ctx->gev.assign(2 * ctx->groups.size(), nullptr);
-      for (cudaEvent_t& e : ctx->gev) CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+      for (cudaEvent_t& ev : ctx->gev) CUDA_TRY(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+      for (cudaEvent_t& ev : ctx->split_ev) CUDA_TRY(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
     }
   }
 
@@ -712,6 +757,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_scal), n * sizeof(MatScal)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_step), n * sizeof(MatStep)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_et_mat), n_et * sizeof(int32_t)) != cudaSuccess ||
+      dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_mlist), n * sizeof(int32_t)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part), 2 * n_et * sizeof(float)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part64), n_et * sizeof(double)) != cudaSuccess ||
       dev_alloc(ctx, reinterpret_cast<void**>(&ctx->d_part8), kStreamSlots * n_et * sizeof(float)) != cudaSuccess ||
@@ -745,6 +791,7 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
   CUDA_TRY(cudaMemcpyAsync(ctx->d_mats, ctx->mats.data(), n * sizeof(MatDev), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_classes, cdev.data(), cdev.size() * sizeof(ClassDev), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_et_mat, et_mat.data(), n_et * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemcpyAsync(ctx->d_mlist, ctx->h_mlist.data(), n * sizeof(int32_t), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemcpyAsync(ctx->d_scal, scal.data(), n * sizeof(MatScal), cudaMemcpyHostToDevice, s));
   CUDA_TRY(cudaMemsetAsync(ctx->d_err, 0, (1 + kMaxGroups) * sizeof(int), s));
 
@@ -879,19 +926,23 @@ muonh_status enqueue_step(muonh_ctx* ctx, const MatStep* step_args, muonh_stats*
   const int grid = ctx->sm_count * 8;
   // elementwise grids: one resident wave, or short blocks when the launch
   // overlaps the other group's GEMMs
-  auto ew_grid = [&](int kind, const muonh_ctx::Group& gr, bool overlap) {
+  auto ew_grid = [&](int kind, const EwParams& p, bool overlap) {
     if (!overlap) return ctx->ew_warp_grid[kind];
-    const int64_t tiles = gr.e_end - gr.e_first;
+    const int64_t tiles = p.e_end - p.e_first;
     return static_cast<int>(std::max<int64_t>(1, (tiles + kOverlapTilesPerBlock - 1) / kOverlapTilesPerBlock));
   };
-  auto front = [&](int g, cudaStream_t st, bool overlap) -> muonh_status {   // momentum, ||X||, X
+  // the elementwise work of group g, or of its matrices in one form (sub 0:
+  // Y-space, 1: Gram-space)
+  auto front = [&](int g, cudaStream_t st, bool overlap, int sub) -> muonh_status {   // momentum, ||X||, X
     const muonh_ctx::Group& gr = ctx->groups[g];
-    const EwParams p = ctx->ew(stats, g);
+    const EwParams p = ctx->ew(stats, g, sub);
+    const bool* any_wt = sub < 0 ? gr.any_wt : gr.sub[sub].any_wt;
+    const bool any_general = sub < 0 ? gr.any_general : gr.sub[sub].any_general;
     for (int tall = 0; tall < 2; ++tall)
-      if (gr.any_wt[tall])
-        STEP_LAUNCH_ON(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_warp(p, tall != 0, ew_grid(tall, gr, overlap), st),
+      if (any_wt[tall])
+        STEP_LAUNCH_ON(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_warp(p, tall != 0, ew_grid(tall, p, overlap), st),
                        "momentum_warp", st);
-    if (gr.any_general) STEP_LAUNCH_ON(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_norm(p, grid, st), "momentum_norm", st);
+    if (any_general) STEP_LAUNCH_ON(MUONH_PHASE_MOMENTUM_NORM, launch_momentum_norm(p, grid, st), "momentum_norm", st);
     STEP_LAUNCH_ON(MUONH_PHASE_FINALIZE_INPUT, launch_finalize_input(p, st), "finalize_input", st);
     STEP_LAUNCH_ON(MUONH_PHASE_WRITE_X, launch_write_x(p, grid, st), "write_x", st);
     return MUONH_OK;
@@ -899,7 +950,9 @@ muonh_status enqueue_step(muonh_ctx* ctx, const MatStep* step_args, muonh_stats*
   for (double& f : ctx->step_flops) f = 0.0;
   // tensor-core FLOPs of a launch over `sum_k` k-blocks of tiles (tile rows x 256 x 64 each)
   const double tile_flops = 2.0 * (ctx->pairs ? 2 * kBM : kBM) * kBN * kBK * (ctx->pairs ? 1 : 3);
-  auto newton_schulz = [&](int g, cudaStream_t st) -> muonh_status {
+  // the GEMMs of group g: its Y-space iterations (parts & 1) and its
+  // Gram-space runs (parts & 2)
+  auto newton_schulz = [&](int g, cudaStream_t st, int parts) -> muonh_status {
     const muonh_ctx::Group& gr = ctx->groups[g];
     NsParams base{};
     base.mats = ctx->d_mats;
@@ -912,7 +965,7 @@ muonh_status enqueue_step(muonh_ctx* ctx, const MatStep* step_args, muonh_stats*
     const int pairs_max = std::max(1, ctx->sm_count / 2);
     auto pair_grid = [&](int ntiles) { return std::min(pairs_max, std::max(1, ntiles)); };
     // ---- Y-space form: A = Y Y^T, B' = a I + b A + c A A, Y <- B' Y per iteration
-    for (int32_t k = 0; k < ctx->max_steps; ++k) {
+    for (int32_t k = 0; k < ((parts & 1) ? ctx->max_steps : 0); ++k) {
       NsParams np = base;
       np.src = k & 1;
       np.iter = k;
@@ -953,7 +1006,7 @@ muonh_status enqueue_step(muonh_ctx* ctx, const MatStep* step_args, muonh_stats*
     // iteration P = p(A) into B' or P1 (alternating); between iterations
     // T = A P, A = T P; the run's product Q = P1 P0 (into T) and P2 Q (into
     // P1); one Y <- Q Y (or P0 Y for a run of one) ends the run
-    if (gr.any_gram) {
+    if (gr.any_gram && (parts & 2)) {
       const TileList& up = gr.gram_upper;
       const TileList& ap = gr.gram_apply;
       int k0 = 0;
@@ -1019,45 +1072,80 @@ muonh_status enqueue_step(muonh_ctx* ctx, const MatStep* step_args, muonh_stats*
     }
     return MUONH_OK;
   };
-  auto back = [&](int g, cudaStream_t st, bool overlap) -> muonh_status {   // dots, projection, stats
+  auto back = [&](int g, cudaStream_t st, bool overlap, int sub) -> muonh_status {   // dots, projection, stats
     const muonh_ctx::Group& gr = ctx->groups[g];
-    const EwParams p = ctx->ew(stats, g);
-    if (gr.any_unfused) STEP_LAUNCH_ON(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, st), "update_dots", st);
+    const EwParams p = ctx->ew(stats, g, sub);
+    const bool* any_wt = sub < 0 ? gr.any_wt : gr.sub[sub].any_wt;
+    const bool any_general = sub < 0 ? gr.any_general : gr.sub[sub].any_general;
+    const bool any_unfused = sub < 0 ? gr.any_unfused : gr.sub[sub].any_unfused;
+    if (any_unfused) STEP_LAUNCH_ON(MUONH_PHASE_UPDATE_DOTS, launch_update_dots(p, grid, st), "update_dots", st);
     STEP_LAUNCH_ON(MUONH_PHASE_FINALIZE_UPDATE, launch_finalize_update(p, st), "finalize_update", st);
     for (int tall = 0; tall < 2; ++tall)
-      if (gr.any_wt[tall])
-        STEP_LAUNCH_ON(MUONH_PHASE_PROJECT, launch_project_warp(p, tall != 0, ew_grid(2 + tall, gr, overlap), st),
+      if (any_wt[tall])
+        STEP_LAUNCH_ON(MUONH_PHASE_PROJECT, launch_project_warp(p, tall != 0, ew_grid(2 + tall, p, overlap), st),
                        "project_warp", st);
-    if (gr.any_general) STEP_LAUNCH_ON(MUONH_PHASE_PROJECT, launch_project(p, grid, st), "project", st);
+    if (any_general) STEP_LAUNCH_ON(MUONH_PHASE_PROJECT, launch_project(p, grid, st), "project", st);
     STEP_LAUNCH_ON(MUONH_PHASE_FINALIZE_STEP, launch_finalize_step(p, st), "finalize_step", st);
     return MUONH_OK;
   };
   muonh_status st;
   if (ctx->groups.size() == 1) {
-    if ((st = front(0, s, false)) || (st = newton_schulz(0, s)) || (st = back(0, s, false))) return st;
+    if ((st = front(0, s, false, -1)) || (st = newton_schulz(0, s, 3)) || (st = back(0, s, false, -1))) return st;
   } else {
     // caller's stream: front(0) | front(1) | back(0), front(2) | ... | back(G-1)
     // GEMM stream:              | NS(0) ...| NS(1) ............| ... |
-    // group g's front work overlaps NS(g-1), its back work NS(g+1)
+    // group g's front work overlaps NS(g-1), its back work NS(g+1).  The two
+    // ends, where nothing else runs, are split by Newton-Schulz form when a
+    // group has both: the first group's Y-space GEMMs start after only the
+    // Y-space matrices' front work, and its Gram-space front work overlaps
+    // them; the last group runs its Gram-space GEMMs first, and their back
+    // work overlaps its Y-space GEMMs.
     cudaStream_t hs = ctx->ns_stream;
     const int G = static_cast<int>(ctx->groups.size());
-    if ((st = front(0, s, false))) return st;
+    auto both = [&](int g) { return ctx->groups[g].sub[0].m_count > 0 && ctx->groups[g].sub[1].m_count > 0; };
+    const bool split_first = both(0), split_last = both(G - 1);
+    if (split_first) {
+      if ((st = front(0, s, false, 0))) return st;
+      CUDA_TRY(cudaEventRecord(ctx->split_ev[0], s));
+      if ((st = front(0, s, true, 1))) return st;
+    } else if ((st = front(0, s, false, -1))) {
+      return st;
+    }
     CUDA_TRY(cudaEventRecord(ctx->gev[0], s));
     for (int g = 0; g < G; ++g) {
-      CUDA_TRY(cudaStreamWaitEvent(hs, ctx->gev[2 * g], 0));
-      if ((st = newton_schulz(g, hs))) return st;
+      if (g == 0 && split_first) {
+        CUDA_TRY(cudaStreamWaitEvent(hs, ctx->split_ev[0], 0));
+        if ((st = newton_schulz(g, hs, 1))) return st;
+        CUDA_TRY(cudaStreamWaitEvent(hs, ctx->gev[0], 0));
+        if ((st = newton_schulz(g, hs, 2))) return st;
+      } else if (g == G - 1 && split_last) {
+        CUDA_TRY(cudaStreamWaitEvent(hs, ctx->gev[2 * g], 0));
+        if ((st = newton_schulz(g, hs, 2))) return st;
+        CUDA_TRY(cudaEventRecord(ctx->split_ev[1], hs));
+        if ((st = newton_schulz(g, hs, 1))) return st;
+      } else {
+        CUDA_TRY(cudaStreamWaitEvent(hs, ctx->gev[2 * g], 0));
+        if ((st = newton_schulz(g, hs, 3))) return st;
+      }
       CUDA_TRY(cudaEventRecord(ctx->gev[2 * g + 1], hs));
       if (g + 1 < G) {
-        if ((st = front(g + 1, s, true))) return st;
+        if ((st = front(g + 1, s, true, -1))) return st;
         CUDA_TRY(cudaEventRecord(ctx->gev[2 * (g + 1)], s));   // before back(g - 1): NS(g + 1) need not wait for it
       }
       if (g >= 1) {
         CUDA_TRY(cudaStreamWaitEvent(s, ctx->gev[2 * (g - 1) + 1], 0));
-        if ((st = back(g - 1, s, true))) return st;
+        if ((st = back(g - 1, s, true, -1))) return st;
       }
     }
-    CUDA_TRY(cudaStreamWaitEvent(s, ctx->gev[2 * (G - 1) + 1], 0));
-    if ((st = back(G - 1, s, false))) return st;
+    if (split_last) {
+      CUDA_TRY(cudaStreamWaitEvent(s, ctx->split_ev[1], 0));
+      if ((st = back(G - 1, s, true, 1))) return st;
+      CUDA_TRY(cudaStreamWaitEvent(s, ctx->gev[2 * (G - 1) + 1], 0));
+      if ((st = back(G - 1, s, false, 0))) return st;
+    } else {
+      CUDA_TRY(cudaStreamWaitEvent(s, ctx->gev[2 * (G - 1) + 1], 0));
+      if ((st = back(G - 1, s, false, -1))) return st;
+    }
   }
   ctx->last_launches = launches;
   ctx->last_stream = s;

@@ -161,9 +161,11 @@ struct EwParams {
   const int32_t* et_mat;     // elementwise tile -> matrix
   int64_t n_et;
   // the part of the step one launch covers: elementwise tiles [e_first,
-  // e_end) and matrices [m_first, m_first + m_count) (one finalize block each)
+  // e_end) and matrices [m_first, m_first + m_count) (one finalize block
+  // each), or, with mlist, the matrices mlist[m_first .. m_first + m_count)
   int64_t e_first, e_end;
   int32_t m_first, m_count;
+  const int32_t* mlist;
   float* part;               // per-tile partials
   float* part8;              // warp-tiled kernels: one partial per (tile, warp), 8 per tile
   double* part64;
@@ -176,6 +178,11 @@ struct EwParams {
   int* any_rewrite;          // this matrix group: set by finalize_input when a matrix needs write_x,
                              // cleared by finalize_step
 };
+
+// Matrix of finalize block `b` of a launch.
+__device__ __forceinline__ int ew_matrix(const EwParams& p, int b) {
+  return p.mlist ? p.mlist[p.m_first + b] : p.m_first + b;
+}
 
 // -------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -603,7 +603,7 @@ __device__ double tile_partials(const EwParams& p, const MatDev& md, double* red
 
 __global__ void __launch_bounds__(kEwThreads) finalize_init_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = p.m_first + blockIdx.x;
+  const int mi = ew_matrix(p, blockIdx.x);
   const MatDev& md = p.mats[mi];
   const int64_t cnt = static_cast<int64_t>(md.et_rows) * md.et_cols;
   const double s = matrix_sum(p.part64, md.et_begin, cnt, 1, 0, red);
@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_init_kernel(const EwParam
 
 __global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = p.m_first + blockIdx.x;
+  const int mi = ew_matrix(p, blockIdx.x);
   const MatDev& md = p.mats[mi];
   const double s = tile_partials(p, md, red);
   if (threadIdx.x == 0) {
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_input_kernel(const EwPara
 
 __global__ void __launch_bounds__(kEwThreads) finalize_update_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = p.m_first + blockIdx.x;
+  const int mi = ew_matrix(p, blockIdx.x);
   const MatDev& md = p.mats[mi];
   double soo, swo;
   if (md.fused_dots) {
@@ -729,7 +729,7 @@ __global__ void __launch_bounds__(kEwThreads) finalize_update_kernel(const EwPar
 
 __global__ void __launch_bounds__(kEwThreads) finalize_step_kernel(const EwParams p) {
   __shared__ double red[kEwThreads / 32];
-  const int mi = p.m_first + blockIdx.x;
+  const int mi = ew_matrix(p, blockIdx.x);
   const MatDev& md = p.mats[mi];
   const double s = tile_partials(p, md, red);
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.any_rewrite = 0;   // write_x of this step has run
