@@ -193,3 +193,45 @@ def test_ordinary_muon_rules_on_the_gram_form(rule):
                 assert abs(gs["elr"] - lr) <= NORM_TOL * lr, (t, i)
             else:
                 assert abs(gs["elr"] - os_["elr"]) <= FP16_NS_TOL * os_["elr"], (t, i)
+
+
+def test_groups_split_by_form_give_the_same_bits():
+    """A set whose matrix groups hold both forms: with two groups the first
+    group's momentum pass and the last group's projection run in two parts
+    (Y-space matrices, then Gram-space ones) around the Gram-space and
+    Y-space GEMMs; with three groups the end groups hold one form each and
+    are not split; one group runs everything in sequence.  W, M and the
+    stats agree bit for bit, and the split schedule launches more kernels."""
+    import torch
+    from pretraining_optimizer_b200 import MuonH
+    dev = torch.device("cuda:0")
+    # NS work: the three 2048 x 6144 (Gram-space) matrices dominate, so two
+    # groups end after the second of them and each holds both forms
+    shapes = [(2048, 6144), (1024, 1024), (6144, 2048), (512, 768), (2048, 6144), (1024, 2048)]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    runs = []
+    for groups in (1, 2, 3):
+        W = [torch.from_numpy(w).to(dev) for w in W0]
+        M = [torch.zeros_like(w) for w in W]
+        opt = MuonH(W, M, groups=groups)
+        for t in range(2):
+            opt.step([torch.from_numpy(synth.gaussian_gradient(t, i, *s)).to(dev) for i, s in enumerate(shapes)],
+                     [0.01, 0.02, 0.01, 0.015, 0.01, 0.02])
+        launches = opt.last_launch_count()
+        st = opt.stats()
+        opt.device_status()
+        opt.close()
+        runs.append(([w.cpu().numpy() for w in W], [m.cpu().numpy() for m in M], st, launches))
+    (W1, M1, s1, l1), (W2, M2, s2, l2), (W3, M3, s3, l3) = runs
+    assert l2 > l1 and l3 > l1
+    for W_, M_, s_ in ((W2, M2, s2), (W3, M3, s3)):
+        for i in range(len(shapes)):
+            assert np.array_equal(W1[i], W_[i]) and np.array_equal(M1[i], M_[i]), i
+            assert s1[i] == s_[i], i
+    # and the result is the method's: the Gram-space matrices against the oracle
+    for i in (0, 2, 4):
+        R = oracle.radius(W0[i])
+        w, m = W0[i].astype(np.float64), np.zeros(shapes[i])
+        for t, lr in enumerate([0.01, 0.01]):
+            w, m, _, _ = oracle.muonh_step(w, m, synth.gaussian_gradient(t, i, *shapes[i]), lr, R)
+        assert rel_fro(W1[i], w) <= W_TOL_10, i
