@@ -354,6 +354,26 @@ void release(muonh_ctx* ctx) {
   delete ctx;
 }
 
+// 4-D 16-bit map over X (rows x inner, count matrices) as an MN-major
+// operand: dimensions (64 columns, rows, 64-column chunks, matrix) with the
+// chunk stride 128 bytes, so that a 64 x 64 x 2 box lands in shared memory
+// as two 64 x 64 chunks of 8 KB, one after the other (128-byte swizzle).
+muonh_status encode_map_mn2(CUtensorMap* out, void* base, int prec16_is_bf16, int64_t inner, int64_t rows,
+                            int64_t count) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(inner / 64),
+                              static_cast<cuuint64_t>(count)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(inner * 2), 128u, static_cast<cuuint64_t>(inner * rows * 2)};
+  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(kBK), 2u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(out, prec16_is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                  base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled (MN pair box) failed (%d)", static_cast<int>(r));
+  return MUONH_OK;
+}
+
 muonh_status encode_map(CUtensorMap* out, void* base, int prec16_is_bf16, int64_t inner, int64_t rows,
                         int64_t count, int box_rows, int box_inner = 64,
                         CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
@@ -719,6 +739,9 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
         if ((st = encode_map(&m[tm_x(TM_X_K256, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBN)))
           return st;
         if ((st = encode_map(&m[tm_x(TM_X_MN, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBK)))
+          return st;
+        if (part == 0 && ctx->pairs &&
+            (st = encode_map_mn2(&m[TM_X_MN2 + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count)))
           return st;
         if (part == 0 && (st = encode_map(&m[TM_X_ST + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count, 32, 32,
                                           CU_TENSOR_MAP_SWIZZLE_64B)))

@@ -53,7 +53,8 @@ enum TmSlot {
   TM_T_K128 = 23,  // Gram-space form: T, 128-row box
   TM_P1_ST = 24,   // P1 store box
   TM_T_ST = 25,    // T store box
-  TM_PER_CLASS = 26
+  TM_X_MN2 = 26,   // X[buf] as MN-major operand: the two 64-column chunks of a 128-column half, one 4-D box (+buf)
+  TM_PER_CLASS = 28
 };
 __host__ __device__ inline int tm_rr_k128(int buf) {
   return buf == RR_A ? TM_A_K128 : buf == RR_B ? TM_B_K128 : buf == RR_P1 ? TM_P1_K128 : TM_T_K128;
@@ -430,6 +431,16 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 }
 
 // TMA load into this CTA's shared memory that signals the pair leader's mbarrier.
+// 4-D tiled load for a CTA pair (see tma_load_3d_pair).
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y, int z) {
   asm volatile(

@@ -643,11 +643,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
             tma_load_3d_pair(sb, p.tmaps + cd.tm_base + tm_rr_k128(p.rhs), bar, k0, bcol, z);
           } else {
             // APPLY: rows of B' or Q (stored with its mirror, K-major) times Y,
-            // read as an MN-major operand
+            // read as an MN-major operand: both 64-column chunks of this CTA's
+            // half in one box (one TMA instruction fewer per stage: APPLY ran
+            // 4-5% faster than with a box per chunk)
             tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
-            const CUtensorMap* bm = p.tmaps + tm_x(cd.tm_base + TM_X_MN, p.src, 0);
-            tma_load_3d_pair(sb, bm, bar, bcol, k0, z);
-            tma_load_3d_pair(sb + 64 * kBK * 2, bm, bar, bcol + 64, k0, z);   // second 64-wide MN chunk
+            tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_MN2 + p.src, bar, 0, k0, bcol / 64, z);
           }
           issued[stage] = true;
           issued_parity[stage] = phase;
