@@ -354,18 +354,20 @@ void release(muonh_ctx* ctx) {
   delete ctx;
 }
 
-// 4-D 16-bit map over X (rows x inner, count matrices) as an MN-major
-// operand: dimensions (64 columns, rows, 64-column chunks, matrix) with the
-// chunk stride 128 bytes, so that a 64 x 64 x 2 box lands in shared memory
-// as two 64 x 64 chunks of 8 KB, one after the other (128-byte swizzle).
-muonh_status encode_map_mn2(CUtensorMap* out, void* base, int prec16_is_bf16, int64_t inner, int64_t rows,
-                            int64_t count) {
+// 4-D 16-bit map over a row-major buffer (rows x inner, count matrices):
+// dimensions (64 columns, rows, 64-column chunks, matrix), the chunk stride
+// 128 bytes, so that a 64 x box_rows x 2 box lands in shared memory as two
+// box_rows x 64 chunks one after the other (128-byte swizzle).  Read as a
+// K-major operand the chunks are two k-blocks; read as an MN-major one,
+// the two 64-wide column chunks of a 128-column half.
+muonh_status encode_map_chunks(CUtensorMap* out, void* base, int prec16_is_bf16, int64_t inner, int64_t rows,
+                               int64_t count, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MUONH_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(inner / 64),
                               static_cast<cuuint64_t>(count)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(inner * 2), 128u, static_cast<cuuint64_t>(inner * rows * 2)};
-  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(kBK), 2u, 1u};
+  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(box_rows), 2u, 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   CUresult r = fn(out, prec16_is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -741,7 +743,8 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
         if ((st = encode_map(&m[tm_x(TM_X_MN, buf, part)], cd.x[buf][part], bf, cd.c_pad, cd.r_pad, cd.count, kBK)))
           return st;
         if (part == 0 && ctx->pairs &&
-            (st = encode_map_mn2(&m[TM_X_MN2 + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count)))
+            ((st = encode_map_chunks(&m[TM_X_C64 + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count, kBK)) ||
+             (st = encode_map_chunks(&m[TM_X_C128 + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count, 2 * kBK))))
           return st;
         if (part == 0 && (st = encode_map(&m[TM_X_ST + buf], cd.x[buf][0], bf, cd.c_pad, cd.r_pad, cd.count, 32, 32,
                                           CU_TENSOR_MAP_SWIZZLE_64B)))
@@ -754,6 +757,10 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           (st = encode_map(&m[TM_C_K256 + part], cd.c[part], bf, cd.r_pad, cd.r_pad, cd.count, kBN)))
         return st;
       if (part == 0 && ctx->pairs) {
+        // two k-blocks of A or B' per TMA box
+        if ((st = encode_map_chunks(&m[TM_A_C128], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM)) ||
+            (st = encode_map_chunks(&m[TM_B_C128], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM)))
+          return st;
         // epilogue store boxes: 32 rows x 32 columns, one per epilogue warp
         if ((st = encode_map(&m[TM_A_ST], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
@@ -762,6 +769,9 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
         if (ctx->classes[ci].gram) {
           if ((st = encode_map(&m[TM_P1_K128], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
           if ((st = encode_map(&m[TM_T_K128], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
+          if ((st = encode_map_chunks(&m[TM_P1_C128], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, kBM)) ||
+              (st = encode_map_chunks(&m[TM_T_C128], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, kBM)))
+            return st;
           if ((st = encode_map(&m[TM_P1_ST], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, 32, 32,
                                CU_TENSOR_MAP_SWIZZLE_64B)))
             return st;

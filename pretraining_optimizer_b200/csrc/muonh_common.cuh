@@ -53,11 +53,21 @@ enum TmSlot {
   TM_T_K128 = 23,  // Gram-space form: T, 128-row box
   TM_P1_ST = 24,   // P1 store box
   TM_T_ST = 25,    // T store box
-  TM_X_MN2 = 26,   // X[buf] as MN-major operand: the two 64-column chunks of a 128-column half, one 4-D box (+buf)
-  TM_PER_CLASS = 28
+  // CTA pairs: 4-D maps (64 columns, rows, 64-column chunks, matrix) that
+  // load two 64-column chunks with one instruction
+  TM_X_C64 = 26,   // X[buf], 64 rows x 2 chunks: an MN-major k-block of a 128-column half (+buf)
+  TM_X_C128 = 28,  // X[buf], 128 rows x 2 chunks: two K-major k-blocks, or two MN-major ones (+buf)
+  TM_A_C128 = 30,  // A, B', P1, T: 128 rows x 2 chunks, two K-major k-blocks
+  TM_B_C128 = 31,
+  TM_P1_C128 = 32,
+  TM_T_C128 = 33,
+  TM_PER_CLASS = 34
 };
 __host__ __device__ inline int tm_rr_k128(int buf) {
   return buf == RR_A ? TM_A_K128 : buf == RR_B ? TM_B_K128 : buf == RR_P1 ? TM_P1_K128 : TM_T_K128;
+}
+__host__ __device__ inline int tm_rr_c128(int buf) {
+  return buf == RR_A ? TM_A_C128 : buf == RR_B ? TM_B_C128 : buf == RR_P1 ? TM_P1_C128 : TM_T_C128;
 }
 __host__ __device__ inline int tm_rr_st(int buf) {
   return buf == RR_A ? TM_A_ST : buf == RR_B ? TM_B_ST : buf == RR_P1 ? TM_P1_ST : TM_T_ST;

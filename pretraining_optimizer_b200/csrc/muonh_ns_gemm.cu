@@ -464,12 +464,15 @@ struct PairCfg {
   // the last APPLY gives staging space to the fp32 W boxes of its <W, O> partials
   static constexpr bool kLast = MODE == M_APPLY_LAST;
   static constexpr bool kSquare = MODE == M_SQUARE;
-  // operand ring of 32 KB stages (a sixth stage, where shared memory allows
-  // it, measured slower: SQUARE lost 4%)
-  static constexpr int kStages = 5;
+  // Operand ring: stages of kKB k-blocks, each operand of a stage one TMA
+  // box (two 64-column chunks of a 4-D map): 3 stages of 64 KB, or, in the
+  // last APPLY, which also stages W, 5 stages of one k-block (32 KB)
+  static constexpr int kKB = kLast ? 1 : 2;
+  static constexpr int kStages = kLast ? 5 : 3;
   static constexpr int kWBufs = 2;
-  static constexpr int kABytes = 128 * kBK * 2;                 // 16 KB: this CTA's 128 rows
-  static constexpr int kBBytes = 128 * kBK * 2;                 // 16 KB: this CTA's half of N
+  static constexpr int kABlock = 128 * kBK * 2;                 // 16 KB: one k-block of this CTA's 128 rows
+  static constexpr int kABytes = kKB * kABlock;
+  static constexpr int kBBytes = kKB * kABlock;                 // this CTA's half of N
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = kStages * kStageBytes;
   // Epilogue warps: one per TMEM lane quarter
@@ -625,14 +628,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         const int abase = td.bi * kPairM, bbase = td.bj * kBN;                // tile origin
         const int arow = abase + static_cast<int>(rank) * 128;              // this CTA's A rows
         const int bcol = bbase + static_cast<int>(rank) * 128;              // this CTA's B half
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk; kb += C::kKB) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
           const uint32_t bar = map_shared_rank(&full[stage], 0);
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           const int k0 = kb * kBK;
-          if (MODE == M_GRAM) {
+          if (C::kKB == 2) {
+            // one 4-D box per operand and stage: K-major operands as the two
+            // 64-column chunks (k-blocks) kb, kb + 1 of this CTA's 128 rows;
+            // in APPLY, Y's rows k0 .. k0+127 in this CTA's two 64-column
+            // chunks (read MN-major).  Half the TMA instructions of one box
+            // per k-block.
+            if (MODE == M_GRAM) {
+              const CUtensorMap* xm = p.tmaps + cd.tm_base + TM_X_C128 + p.src;
+              tma_load_4d_pair(sa, xm, bar, 0, arow, kb, z);
+              tma_load_4d_pair(sb, xm, bar, 0, bcol, kb, z);
+            } else if (MODE == M_SQUARE || MODE == M_SYMPROD) {
+              tma_load_4d_pair(sa, p.tmaps + cd.tm_base + tm_rr_c128(p.lhs), bar, 0, arow, kb, z);
+              tma_load_4d_pair(sb, p.tmaps + cd.tm_base + tm_rr_c128(p.rhs), bar, 0, bcol, kb, z);
+            } else {
+              tma_load_4d_pair(sa, p.tmaps + cd.tm_base + tm_rr_c128(p.lhs), bar, 0, arow, kb, z);
+              tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_C128 + p.src, bar, 0, k0, bcol / 64, z);
+            }
+          } else if (MODE == M_GRAM) {
             tma_load_3d_pair(sa, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, arow, z);
             tma_load_3d_pair(sb, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, bcol, z);
           } else if (MODE == M_SQUARE || MODE == M_SYMPROD) {
@@ -647,7 +667,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
             // half in one box (one TMA instruction fewer per stage: APPLY ran
             // 4-5% faster than with a box per chunk)
             tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
-            tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_MN2 + p.src, bar, 0, k0, bcol / 64, z);
+            tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_C64 + p.src, bar, 0, k0, bcol / 64, z);
           }
           issued[stage] = true;
           issued_parity[stage] = phase;
@@ -682,17 +702,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk; kb += C::kKB) {
           if (!mbar_wait(&full[stage], phase, p.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t sb = sa + C::kABytes;
+          const uint32_t s0 = smem_u32(smem + stage * C::kStageBytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t adesc = sdesc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t bdesc = kApply ? sdesc_sw128(sb + k * 16 * 128, 64 * kBK * 2, 1024)
-                                          : sdesc_sw128(sb + k * 32, 16, 1024);
-            umma_f16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          for (int j = 0; j < C::kKB; ++j) {
+            // k-block kb + j: A chunk j; B chunk j (K-major), or rows 64 j ..
+            // of both 64-column chunks (MN-major APPLY: chunk stride kKB x 8 KB)
+            const uint32_t sa = s0 + j * C::kABlock;
+            const uint32_t sb = s0 + C::kABytes + j * (kApply ? 64 * 128 : C::kABlock);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t adesc = sdesc_sw128(sa + k * 32, 16, 1024);
+              const uint64_t bdesc = kApply ? sdesc_sw128(sb + k * 16 * 128, C::kKB * 64 * 128, 1024)
+                                            : sdesc_sw128(sb + k * 32, 16, 1024);
+              umma_f16_pair(d_tmem, adesc, bdesc, kIdesc, ((kb + j) | k) != 0 ? 1u : 0u);
+            }
           }
           umma_commit_pair(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
