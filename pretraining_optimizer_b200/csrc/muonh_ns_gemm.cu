@@ -477,7 +477,8 @@ struct PairCfg {
   static constexpr int kBarOffset = kStages * kStageBytes;
   // Epilogue warps: one per TMEM lane quarter
   static constexpr int kEpiWarps = 4;
-  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kProducerB = 2 + kEpiWarps;   // the B-operand producer warp, after the epilogue warps
+  static constexpr int kThreads = 96 + 32 * kEpiWarps;
   // Epilogue output staging: each epilogue warp owns kWarpBufs boxes of
   // 32 rows x 32 columns (16-bit, 64-byte swizzle) that it writes to global
   // memory with its own TMA stores
@@ -610,8 +611,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
+  if (warp == 0 || warp == C::kProducerB) {
+    // ------------------------------------------------------------ TMA producers (both CTAs)
+    // warp 0 loads the A operand of every stage (and, in the leader, sets
+    // the stage's expected bytes); warp kProducerB loads the B operand, so
+    // that the two boxes of a stage are issued from two warps at once
+    const bool role_a = warp == 0;
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -630,7 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         const int bcol = bbase + static_cast<int>(rank) * 128;              // this CTA's B half
         for (int kb = 0; kb < nk; kb += C::kKB) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) { ok = false; break; }
-          if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
+          if (rank == 0 && role_a) mbar_expect_tx(&full[stage], 2 * C::kStageBytes);
           const uint32_t bar = map_shared_rank(&full[stage], 0);
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
@@ -643,38 +648,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
             // per k-block.
             if (MODE == M_GRAM) {
               const CUtensorMap* xm = p.tmaps + cd.tm_base + TM_X_C128 + p.src;
-              tma_load_4d_pair(sa, xm, bar, 0, arow, kb, z);
-              tma_load_4d_pair(sb, xm, bar, 0, bcol, kb, z);
+              if (role_a) tma_load_4d_pair(sa, xm, bar, 0, arow, kb, z);
+              if (!role_a) tma_load_4d_pair(sb, xm, bar, 0, bcol, kb, z);
             } else if (MODE == M_SQUARE || MODE == M_SYMPROD) {
-              tma_load_4d_pair(sa, p.tmaps + cd.tm_base + tm_rr_c128(p.lhs), bar, 0, arow, kb, z);
-              tma_load_4d_pair(sb, p.tmaps + cd.tm_base + tm_rr_c128(p.rhs), bar, 0, bcol, kb, z);
+              if (role_a) tma_load_4d_pair(sa, p.tmaps + cd.tm_base + tm_rr_c128(p.lhs), bar, 0, arow, kb, z);
+              if (!role_a) tma_load_4d_pair(sb, p.tmaps + cd.tm_base + tm_rr_c128(p.rhs), bar, 0, bcol, kb, z);
             } else {
-              tma_load_4d_pair(sa, p.tmaps + cd.tm_base + tm_rr_c128(p.lhs), bar, 0, arow, kb, z);
-              tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_C128 + p.src, bar, 0, k0, bcol / 64, z);
+              if (role_a) tma_load_4d_pair(sa, p.tmaps + cd.tm_base + tm_rr_c128(p.lhs), bar, 0, arow, kb, z);
+              if (!role_a) tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_C128 + p.src, bar, 0, k0, bcol / 64, z);
             }
           } else if (MODE == M_GRAM) {
-            tma_load_3d_pair(sa, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, arow, z);
-            tma_load_3d_pair(sb, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, bcol, z);
+            if (role_a) tma_load_3d_pair(sa, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, arow, z);
+            if (!role_a) tma_load_3d_pair(sb, p.tmaps + tm_x(cd.tm_base + TM_X_K128, p.src, 0), bar, k0, bcol, z);
           } else if (MODE == M_SQUARE || MODE == M_SYMPROD) {
             // A A (SQUARE) or L R (SYMPROD) with both operands stored whole
             // (every block and its mirror): both K-major; the right operand is
             // symmetric, so its rows serve as the N x K operand
-            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
-            tma_load_3d_pair(sb, p.tmaps + cd.tm_base + tm_rr_k128(p.rhs), bar, k0, bcol, z);
+            if (role_a) tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
+            if (!role_a) tma_load_3d_pair(sb, p.tmaps + cd.tm_base + tm_rr_k128(p.rhs), bar, k0, bcol, z);
           } else {
             // APPLY: rows of B' or Q (stored with its mirror, K-major) times Y,
             // read as an MN-major operand: both 64-column chunks of this CTA's
             // half in one box (one TMA instruction fewer per stage: APPLY ran
             // 4-5% faster than with a box per chunk)
-            tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
-            tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_C64 + p.src, bar, 0, k0, bcol / 64, z);
+            if (role_a) tma_load_3d_pair(sa, p.tmaps + cd.tm_base + tm_rr_k128(p.lhs), bar, k0, arow, z);
+            if (!role_a) tma_load_4d_pair(sb, p.tmaps + cd.tm_base + TM_X_C64 + p.src, bar, 0, k0, bcol / 64, z);
           }
           issued[stage] = true;
           issued_parity[stage] = phase;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok && rank == 0) {
+      if (!ok && rank == 0 && role_a) {
         for (int s = 0; s < C::kStages; ++s)
           if (issued[s]) {
             const uint64_t t0 = globaltimer();
