@@ -369,6 +369,15 @@ __device__ __forceinline__ void stmatrix_x4(uint32_t addr, uint32_t a, uint32_t 
                "r"(c), "r"(d)
                : "memory");
 }
+// Inverse of stmatrix_x4: four 8 x 8 16-bit matrices from shared memory into
+// MMA fragments (thread t: row t/4, columns 2(t%4), 2(t%4)+1 of each);
+// thread t gives the address of row t%8 of matrix t/8.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(addr)
+               : "memory");
+}
 __device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a),
                "r"(b), "r"(c), "r"(d)

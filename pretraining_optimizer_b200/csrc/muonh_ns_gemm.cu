@@ -483,15 +483,19 @@ struct PairCfg {
   // 32 rows x 32 columns (16-bit, 64-byte swizzle) that it writes to global
   // memory with its own TMA stores
   static constexpr int kWarpBox = 32 * 32 * 2;
-  static constexpr int kWarpBufs = kLast ? 2 : 4;
+  static constexpr int kWarpBufs = (kLast || kSquare) ? 2 : 4;
   static constexpr int kStoreOffset = (kBarOffset + 256 + 1023) / 1024 * 1024;
+  // SQUARE: each epilogue warp stages A's 32 x 32 box of its next chunk (for
+  // the b A term) by TMA, two buffers, and reads it back with ldmatrix
+  static constexpr int kABoxOffset = kStoreOffset + kEpiWarps * kWarpBufs * kWarpBox;
+  static constexpr int kABoxBytes = kSquare ? kEpiWarps * 2 * kWarpBox : 0;
   // Last APPLY: kWBufs fp32 W boxes (128 rows x 32 columns, or 32 x 128 for
   // a tall W) filled kWBufs chunks ahead, for the <W, O> partials
   static constexpr int kWBox = 128 * 32 * 4;
-  static constexpr int kWOffset = kStoreOffset + kEpiWarps * kWarpBufs * kWarpBox;
+  static constexpr int kWOffset = kABoxOffset + kABoxBytes;
   static constexpr int kSmem = kWOffset + (kLast ? kWBufs * kWBox : 0) + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory of the pair kernel exceeds 227 KB");
-  static_assert(2 * kStages + 2 + 2 + 1 + 4 + 4 <= 31, "mbarriers exceed their 256-byte region");
+  static_assert(2 * kStages + 2 + 2 + 1 + 4 + 4 + 8 <= 31, "mbarriers exceed their 256-byte region");
 };
 
 // Row `r` (0..31) of a 32 x 32 16-bit box, 16-byte piece q, in the 64-byte
@@ -580,7 +584,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
   uint64_t* drain = tempty + 2;
   uint64_t* wfull = drain + 1;                       // last APPLY / SQUARE: staged boxes landed
   uint64_t* wempty = wfull + 4;                      // ... and consumed by the 4 epilogue warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty + 4);
+  uint64_t* abar = wempty + 4;                       // SQUARE: A boxes landed, per epilogue warp and buffer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(abar + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -602,6 +607,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
       mbar_init(&wfull[b], 1);
       mbar_init(&wempty[b], C::kEpiWarps);
     }
+    for (int b = 0; b < 8; ++b) mbar_init(&abar[b], 1);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
@@ -748,6 +754,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
     const uint32_t tempty_leader[2] = {map_shared_rank(&tempty[0], 0), map_shared_rank(&tempty[1], 0)};
     WarpStager<C::kWarpBufs> stager{smem + C::kStoreOffset + epi * C::kWarpBufs * C::kWarpBox, 0};
     const int wrow0_off = quarter * 32;   // this warp's rows inside the CTA's 128
+    // SQUARE: A boxes of this warp (two buffers), their landing barriers and
+    // phases, and whether a box is still in flight (for the give-up path)
+    uint8_t* const abox = smem + C::kABoxOffset + epi * 2 * C::kWarpBox;
+    uint64_t* const abar_w = abar + 2 * epi;
+    uint32_t aphase[2] = {0u, 0u};
+    bool a_inflight[2] = {false, false};
+    int a_count = 0;   // A boxes issued so far; box i lands in buffer i % 2
+    auto a_issue = [&](const CUtensorMap* amap, int x, int y, int z) {
+      const int b = a_count & 1;
+      if (lane == 0) {
+        fence_proxy_async_smem();   // the buffer's previous box was read with ldmatrix
+        mbar_expect_tx(&abar_w[b], C::kWarpBox);
+        tma_load_3d(abox + b * C::kWarpBox, amap, &abar_w[b], x, y, z);
+      }
+      a_inflight[b] = true;
+      ++a_count;
+    };
     uint32_t wphase[C::kWBufs] = {};   // phases of the staging buffers
     int w_pending[C::kWBufs] = {};     // thread 64: staged loads issued and not yet consumed
     int w_issued[C::kWBufs] = {};      // thread 64: loads issued into each buffer so far
@@ -781,23 +804,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
         const int r0 = td.bi * kPairM + static_cast<int>(rank) * 128;
         for (int b = 0; b < C::kWBufs; ++b) w_issue(td, md, cd, r0, b, b);   // first chunks while the MMAs run
       }
-      // SQUARE reads A (written by GRAM, read-only here) for its b A term
-      // straight from L2, one 32-column chunk ahead, in the accumulator
-      // fragment layout of the epilogue: rows lane/4 + 8p + 16h of this
-      // warp's 32, columns 8k + 2 (lane % 4) (+1) of the chunk
-      const uint16_t* abase = nullptr;
-      uint32_t a_next[16];
-      if (C::kSquare) {
-        const int frow = td.bi * kPairM + static_cast<int>(rank) * 128 + quarter * 32 + (lane >> 2);
-        abase = static_cast<const uint16_t*>(cd.a[0]) + md.z * cd.a_stride + static_cast<int64_t>(frow) * cd.r_pad +
-                td.bj * kBN + 2 * (lane & 3);
-#pragma unroll
-        for (int hp = 0; hp < 4; ++hp)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            a_next[4 * hp + k] = __ldg(reinterpret_cast<const uint32_t*>(abase + static_cast<int64_t>(8 * hp) * cd.r_pad +
-                                                                         ch0 * 32 + 8 * k));
-      }
+      // SQUARE reads A (written by GRAM, read-only here) for its b A term:
+      // the 32 x 32 box of this warp's rows and the chunk's columns, staged
+      // by TMA one chunk ahead and read with ldmatrix straight into the
+      // accumulator fragment layout (rows lane/4 + 8p + 16h of the warp's
+      // 32, columns 8k + 2 (lane % 4) (+1) of the chunk)
+      const CUtensorMap* amap = p.tmaps + cd.tm_base + TM_A_ST;
+      const int arow_w = td.bi * kPairM + static_cast<int>(rank) * 128 + quarter * 32;
+      if (C::kSquare) a_issue(amap, td.bj * kBN + ch0 * 32, arow_w, md.z);
       if (!mbar_wait(&tfull[acc], acc_phase, p.err)) break;
       tc_fence_after();
       const int row0 = td.bi * kPairM + static_cast<int>(rank) * 128;   // this CTA's first row
@@ -838,16 +852,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
           }
           uint32_t a_cur[16];
           if (MODE == M_SQUARE) {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) a_cur[q] = a_next[q];
-            if (ch + kChStep < kBN / 32) {
-#pragma unroll
-              for (int hp = 0; hp < 4; ++hp)
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  a_next[4 * hp + k] = __ldg(reinterpret_cast<const uint32_t*>(
-                      abase + static_cast<int64_t>(8 * hp) * cd.r_pad + (ch + kChStep) * 32 + 8 * k));
+            const int b = (a_count - 1) & 1;   // this chunk's box (the latest issued)
+            if (ch + kChStep < kBN / 32) a_issue(amap, col0 + kChStep * 32, arow_w, md.z);
+            if (!mbar_wait(&abar_w[b], aphase[b], p.err)) {
+              werr = true;
+              break;
             }
+            aphase[b] ^= 1u;
+            a_inflight[b] = false;
+            const uint32_t ab = smem_u32(abox + b * C::kWarpBox);
+#pragma unroll
+            for (int hp = 0; hp < 4; ++hp)
+              ldmatrix_x4(ab + store_box_offset(8 * hp + (lane & 7), lane >> 3), a_cur[4 * hp], a_cur[4 * hp + 1],
+                          a_cur[4 * hp + 2], a_cur[4 * hp + 3]);
           }
           uint32_t w[2][2][4];   // [h][p][k]: rows 16h + 8p + lane/4, columns 8k + 2 (lane % 4) (+1)
 #pragma unroll
@@ -1002,6 +1019,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
       }
     }
     if (lane == 0) bulk_wait_all();   // every TMA store of this warp has completed
+    // on a give-up path, let this warp's A boxes in flight land before the CTA exits
+    for (int b = 0; b < 2; ++b)
+      if (C::kSquare && a_inflight[b]) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&abar_w[b], aphase[b]) && globaltimer() - t0 < kWaitLimitNs) {
+        }
+      }
     if (threadIdx.x == 64) {
       // on a give-up path, let issued W loads land before the CTA exits
       for (int b = 0; b < C::kWBufs; ++b)
