@@ -134,14 +134,14 @@ typedef struct {
  *           Gram-space: runs of up to three iterations are carried on r x r
  *           matrices, A_{k+1} = A_k p(A_k)^2 with p(A) = a I + b A + c A A,
  *           and each run ends with one Y <- Q Y, Q the product of the run's
- *           p(A_k) (fewer FLOPs where c >= 3r; a restart every three
+ *           p(A_k) (fewer FLOPs where c >= 2r; a restart every three
  *           iterations keeps fp16 storage accurate).  In exact arithmetic
  *           both give the same O; their fp16 rounding differs.  The Gram
  *           form needs FP16 operands and ns_steps equal to the largest
  *           ns_steps of the context; other matrices use the Y-space form.
  *           Values outside MUONH_NS_FORM_* are rejected. */
 enum {
-  MUONH_NS_FORM_AUTO = 0,    /* Gram form for classes with r >= 2048, c >= 3r  */
+  MUONH_NS_FORM_AUTO = 0,    /* Gram form for classes with r >= 1024, c >= 2r  */
   MUONH_NS_FORM_Y = 1,       /* Y-space form for every matrix                   */
   MUONH_NS_FORM_GRAM = 2     /* Gram form for every matrix that can take it     */
 };
