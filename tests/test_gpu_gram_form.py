@@ -127,6 +127,32 @@ def test_executed_flops_of_each_form():
                                                                                    exp_prod)
 
 
+def test_automatic_form_choice():
+    """The automatic choice takes the Gram-space form where it saves FLOPs,
+    c >= 2r with r >= 1024 (here 1024 x 2048 and its tall transpose), and the
+    Y-space form for a square class and for r < 1024: the per-phase FLOPs
+    are the sum of each matrix's own form."""
+    shapes = [(1024, 2048), (2048, 2048), (512, 1536), (2048, 1024)]
+    W0 = [synth.initial_weight(i, *s) for i, s in enumerate(shapes)]
+    grad = lambda t, i: synth.gaussian_gradient(t, i, *shapes[i])
+    f = run_gpu(W0, grad, [0.01])["flops"]
+    tile = 2 * 256 * 256
+    exp = {"ns_gram": 0, "ns_square": 0, "ns_apply": 0, "ns_product": 0}
+    for rows, cols in shapes:
+        r, c = min(rows, cols), max(rows, cols)
+        if r >= 1024 and c >= 2 * r:
+            for g in (3, 2):
+                exp["ns_gram"] += _upper(r) * tile * c
+                exp["ns_square"] += g * _upper(r) * tile * r
+                exp["ns_product"] += (3 * g - 3) * _upper(r) * tile * r
+                exp["ns_apply"] += (r // 256) * (c // 256) * tile * r
+        else:
+            exp["ns_gram"] += 5 * _upper(r) * tile * c
+            exp["ns_square"] += 5 * _upper(r) * tile * r
+            exp["ns_apply"] += 5 * (r // 256) * (c // 256) * tile * r
+    assert {k: f[k] for k in exp} == exp
+
+
 @pytest.mark.parametrize("ns_steps", [1, 2, 3, 4, 6, 7])
 def test_gram_form_run_lengths(ns_steps):
     """Other step counts split into other runs ((1), (2), (3), (2, 2),
