@@ -20,11 +20,13 @@
 // triangle and store each off-diagonal block twice, directly and mirrored,
 // so that every consumer reads its operands K-major.
 //
-// Per CTA: warp 0 issues TMA loads into a ring of shared-memory stages,
-// warp 1 (one thread) issues tcgen05.mma into one of two TMEM accumulators
-// (128 lanes x 256 fp32 columns each), warps 2-5 drain the other
-// accumulator with tcgen05.ld, apply the polynomial epilogue and store.
-// Every wait is bounded (muonh::mbar_wait) and records a timeout in *err.
+// Per CTA: producer warps issue TMA loads into a ring of shared-memory
+// stages (one warp in the FP32-mode kernel; in the CTA-pair kernel warp 0
+// loads the A boxes and warp 6 the B boxes), warp 1 (one thread) issues
+// tcgen05.mma into one of two TMEM accumulators (128 lanes x 256 fp32
+// columns each), warps 2-5 drain the other accumulator with tcgen05.ld,
+// apply the polynomial epilogue and store.  Every wait is bounded
+// (muonh::mbar_wait) and records a timeout in *err.
 //
 // Storage: fp16 operands hold the value times 2^e (e per matrix and per
 // operand, chosen on the host so that no entry can overflow); products of
@@ -447,10 +449,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) ns_gemm_kernel(const __grid_c
 // computes a 256 x 256 tile with tcgen05.mma.cta_group::2.  Each CTA loads
 // its own 128 rows of the A operand and its own 128-column half of the B
 // operand (no multicast), so a pair moves a third less operand data per
-// FLOP than two single-CTA 128 x 256 tiles.  The leader CTA (rank 0) issues
-// the MMAs; both CTAs' TMA loads complete on the leader's stage barrier, and
-// the leader's commits arrive on the matching barriers of both CTAs.  Each
-// CTA drains its own TMEM (its 128 rows) in the epilogue.
+// FLOP than two single-CTA 128 x 256 tiles.  Each operand of a stage is one
+// 4-D TMA box covering two k-blocks, issued by one of two producer warps:
+// a TMA instruction holds its issuing thread for a few hundred cycles, and
+// one box per operand and k-block from a single thread starved the MMAs.
+// The leader CTA (rank 0) issues the MMAs; both CTAs' TMA loads complete on
+// the leader's stage barrier, and the leader's commits arrive on the
+// matching barriers of both CTAs.  Each CTA drains its own TMEM (its 128
+// rows) in the epilogue.
 //
 // Symmetric results (A, B', the Gram-space factors) are computed on the
 // 256 x 256 tiles of the upper block triangle; the epilogue of an
