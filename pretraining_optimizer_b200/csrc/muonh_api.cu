@@ -762,6 +762,12 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
         if ((st = encode_map_chunks(&m[TM_A_C128], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM)) ||
             (st = encode_map_chunks(&m[TM_B_C128], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, kBM)))
           return st;
+        // GRAM and SYMPROD store boxes: 32 x 64 direct, 64 x 32 mirrored
+        if ((st = encode_map(&m[TM_A_ST2], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+            (st = encode_map(&m[TM_A_STM], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, 64, 32, CU_TENSOR_MAP_SWIZZLE_64B)) ||
+            (st = encode_map(&m[TM_B_ST2], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+            (st = encode_map(&m[TM_B_STM], cd.b[0], bf, cd.r_pad, cd.r_pad, cd.count, 64, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
+          return st;
         // epilogue store boxes: 32 rows x 32 columns, one per epilogue warp
         if ((st = encode_map(&m[TM_A_ST], cd.a[0], bf, cd.r_pad, cd.r_pad, cd.count, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
           return st;
@@ -772,6 +778,11 @@ muonh_status muonh_init(muonh_ctx** out, const muonh_matrix_desc* mats, int32_t 
           if ((st = encode_map(&m[TM_T_K128], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, kBM))) return st;
           if ((st = encode_map_chunks(&m[TM_P1_C128], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, kBM)) ||
               (st = encode_map_chunks(&m[TM_T_C128], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, kBM)))
+            return st;
+          if ((st = encode_map(&m[TM_P1_ST2], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+              (st = encode_map(&m[TM_P1_STM], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, 64, 32, CU_TENSOR_MAP_SWIZZLE_64B)) ||
+              (st = encode_map(&m[TM_T_ST2], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+              (st = encode_map(&m[TM_T_STM], cd.t, bf, cd.r_pad, cd.r_pad, cd.count, 64, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
             return st;
           if ((st = encode_map(&m[TM_P1_ST], cd.p1, bf, cd.r_pad, cd.r_pad, cd.count, 32, 32,
                                CU_TENSOR_MAP_SWIZZLE_64B)))

@@ -61,13 +61,29 @@ enum TmSlot {
   TM_B_C128 = 31,
   TM_P1_C128 = 32,
   TM_T_C128 = 33,
-  TM_PER_CLASS = 34
+  // CTA pairs, GRAM and SYMPROD outputs: 32 x 64 direct boxes (128-byte
+  // swizzle) and 64 x 32 mirror boxes (64-byte swizzle) of A, B', P1, T
+  TM_A_ST2 = 34,
+  TM_B_ST2 = 35,
+  TM_P1_ST2 = 36,
+  TM_T_ST2 = 37,
+  TM_A_STM = 38,
+  TM_B_STM = 39,
+  TM_P1_STM = 40,
+  TM_T_STM = 41,
+  TM_PER_CLASS = 42
 };
 __host__ __device__ inline int tm_rr_k128(int buf) {
   return buf == RR_A ? TM_A_K128 : buf == RR_B ? TM_B_K128 : buf == RR_P1 ? TM_P1_K128 : TM_T_K128;
 }
 __host__ __device__ inline int tm_rr_c128(int buf) {
   return buf == RR_A ? TM_A_C128 : buf == RR_B ? TM_B_C128 : buf == RR_P1 ? TM_P1_C128 : TM_T_C128;
+}
+__host__ __device__ inline int tm_rr_st2(int buf) {
+  return buf == RR_A ? TM_A_ST2 : buf == RR_B ? TM_B_ST2 : buf == RR_P1 ? TM_P1_ST2 : TM_T_ST2;
+}
+__host__ __device__ inline int tm_rr_stm(int buf) {
+  return buf == RR_A ? TM_A_STM : buf == RR_B ? TM_B_STM : buf == RR_P1 ? TM_P1_STM : TM_T_STM;
 }
 __host__ __device__ inline int tm_rr_st(int buf) {
   return buf == RR_A ? TM_A_ST : buf == RR_B ? TM_B_ST : buf == RR_P1 ? TM_P1_ST : TM_T_ST;

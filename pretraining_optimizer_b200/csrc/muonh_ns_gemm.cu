@@ -488,8 +488,11 @@ struct PairCfg {
   // Epilogue output staging: each epilogue warp owns kWarpBufs boxes of
   // 32 rows x 32 columns (16-bit, 64-byte swizzle) that it writes to global
   // memory with its own TMA stores
-  static constexpr int kWarpBox = 32 * 32 * 2;
-  static constexpr int kWarpBufs = (kLast || kSquare) ? 2 : 4;
+  // GRAM and SYMPROD store two chunks per box (a 32 x 64 direct box, a 64 x
+  // 32 mirror box): half the TMA stores
+  static constexpr bool kPairStore = MODE == M_GRAM || MODE == M_SYMPROD;
+  static constexpr int kWarpBox = kPairStore ? 32 * 64 * 2 : 32 * 32 * 2;
+  static constexpr int kWarpBufs = (kLast || kSquare || kPairStore) ? 2 : 4;
   static constexpr int kStoreOffset = (kBarOffset + 256 + 1023) / 1024 * 1024;
   // SQUARE: each epilogue warp stages A's 32 x 32 box of its next chunk (for
   // the b A term) by TMA, two buffers, and reads it back with ldmatrix
@@ -501,26 +504,34 @@ struct PairCfg {
   static constexpr int kWOffset = kABoxOffset + kABoxBytes;
   static constexpr int kSmem = kWOffset + (kLast ? kWBufs * kWBox : 0) + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory of the pair kernel exceeds 227 KB");
+  static_assert(!kPairStore || kEpiWarps == 4, "a box of two consecutive chunks needs one warp per lane quarter");
   static_assert(2 * kStages + 2 + 2 + 1 + 4 + 4 + 8 <= 31, "mbarriers exceed their 256-byte region");
 };
 
-// Row `r` (0..31) of a 32 x 32 16-bit box, 16-byte piece q, in the 64-byte
-// swizzle pattern of the TMA store box.
+// Row `r` of a 16-bit box with 64-byte rows (32 columns; 32 or 64 rows),
+// 16-byte piece q, in the 64-byte swizzle pattern of the TMA box.
 __device__ __forceinline__ uint32_t store_box_offset(int r, int q) {
   return static_cast<uint32_t>(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
 }
 
-// TMA-store staging private to one epilogue warp: lane j supplies row j of
-// a 32 x 32 box; lane 0 issues the store.  A buffer is reused only after the
-// store issued from it kBufs puts earlier has read it, so the warps never
-// wait on one another.
-template <int kBufs>
+// Row `r` (0..31) of a 32 x 64 16-bit box, 16-byte piece q (0..7), in the
+// 128-byte swizzle pattern of the TMA store box.
+__device__ __forceinline__ uint32_t store_box_offset128(int r, int q) {
+  return static_cast<uint32_t>(r * 128 + ((q ^ (r & 7)) << 4));
+}
+
+// TMA-store staging private to one epilogue warp: the warp writes a box of
+// kBox bytes into an acquired buffer and lane 0 issues its store.  Acquire
+// and commit alternate; a buffer is reused only after the store issued from
+// it kBufs boxes earlier has read it, so the warps never wait on one
+// another.
+template <int kBufs, int kBox>
 struct WarpStager {
   uint8_t* base;
   int count;   // boxes handed out so far
   // The next buffer, once the store issued from it kBufs puts ago has read it.
   __device__ __forceinline__ uint8_t* acquire(int lane) {
-    uint8_t* buf = base + (count % kBufs) * (32 * 32 * 2);
+    uint8_t* buf = base + (count % kBufs) * kBox;
     if (count >= kBufs) {
       if (lane == 0) bulk_wait_read<kBufs - 1>();
       __syncwarp();
@@ -758,7 +769,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
     const int ch0 = epi / 4;
     const int lrow = quarter * 32 + lane;
     const uint32_t tempty_leader[2] = {map_shared_rank(&tempty[0], 0), map_shared_rank(&tempty[1], 0)};
-    WarpStager<C::kWarpBufs> stager{smem + C::kStoreOffset + epi * C::kWarpBufs * C::kWarpBox, 0};
+    WarpStager<C::kWarpBufs, C::kWarpBox> stager{smem + C::kStoreOffset + epi * C::kWarpBufs * C::kWarpBox, 0};
     const int wrow0_off = quarter * 32;   // this warp's rows inside the CTA's 128
     // SQUARE: A boxes of this warp (two buffers), their landing barriers and
     // phases, and whether a box is still in flight (for the give-up path)
@@ -844,6 +855,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
           diag = md.a * exp2f(static_cast<float>(md.eb));
         }
         const CUtensorMap* omap = p.tmaps + cd.tm_base + (MODE == M_GRAM ? TM_A_ST : tm_rr_st(p.out));
+        // GRAM, SYMPROD: 32 x 64 direct and 64 x 32 mirror boxes of two chunks
+        const CUtensorMap* omap2 = p.tmaps + cd.tm_base + (MODE == M_GRAM ? TM_A_ST2 : tm_rr_st2(p.out));
+        const CUtensorMap* omapm = p.tmaps + cd.tm_base + (MODE == M_GRAM ? TM_A_STM : tm_rr_stm(p.out));
+        uint32_t wprev[2][2][4];   // the first chunk of a pair, held for its box
         const int grow = row0 + wrow0_off;            // this warp's first row
         const int frow = lane >> 2, fcol = 2 * (lane & 3);
         for (int ch = ch0; ch < kBN / 32; ch += kChStep) {
@@ -900,6 +915,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PREC, MODE>:
                 }
                 w[h][pp][k] = pack_pair<PREC>(v0, v1);
               }
+          if (C::kPairStore) {
+            const int c = ch & 1;   // chunk of the pair (every warp walks every chunk)
+            if (c == 0) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) wprev[h][pp][k] = w[h][pp][k];
+              continue;
+            }
+            // direct box: chunk cc's matrix (h, p, k) is rows 16h + 8p .. +7, 16-byte piece 4 cc + k
+            uint8_t* buf = stager.acquire(lane);
+            const uint32_t sb = smem_u32(buf);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int pp = 0; pp < 2; ++pp) {
+                stmatrix_x4(sb + store_box_offset128(16 * h + 8 * pp + (lane & 7), lane >> 3), wprev[h][pp][0],
+                            wprev[h][pp][1], wprev[h][pp][2], wprev[h][pp][3]);
+                stmatrix_x4(sb + store_box_offset128(16 * h + 8 * pp + (lane & 7), 4 + (lane >> 3)), w[h][pp][0],
+                            w[h][pp][1], w[h][pp][2], w[h][pp][3]);
+              }
+            stager.commit(buf, omap2, lane, col0 - 32, grow, md.z);
+            if (mirror) {
+              // chunk cc transposed: mirror-box rows 32 cc + 8k .. +7, piece 2h + p
+              uint8_t* mb = stager.acquire(lane);
+              const uint32_t smb = smem_u32(mb);
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp) {
+                  stmatrix_x4_trans(smb + store_box_offset(lane, 2 * h + pp), wprev[h][pp][0], wprev[h][pp][1],
+                                    wprev[h][pp][2], wprev[h][pp][3]);
+                  stmatrix_x4_trans(smb + store_box_offset(32 + lane, 2 * h + pp), w[h][pp][0], w[h][pp][1],
+                                    w[h][pp][2], w[h][pp][3]);
+                }
+              stager.commit(mb, omapm, lane, grow, col0 - 32, md.z);
+            }
+            continue;
+          }
           // direct box: matrix (h, p, k) is box rows 16h + 8p .. +7, 16-byte piece k
           uint8_t* buf = stager.acquire(lane);
           const uint32_t sb = smem_u32(buf);
